@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Throughput of the TurboQuant hot path on B200 (one JSON line on rank 0).
+
+Default workload ("sweep"): TurboQuant_mse quantize + dequantize of N = 2^20
+bf16 vectors, d = 128, per-channel lognormal(0, 1) scales with 4 of 128
+channels x20 outliers, for b = 1, 2, 3, 4.  One step = quantize and dequantize
+the batch at every b; the metric counts vectors quantized per second.  The
+decode-attention workload over a compressed K/V cache (B = 8, 32 q-heads,
+8 kv-heads, d = 128, context 131072, K prod 4-bit, V mse 4-bit) is measured in
+the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sweep|decode]
+
+For N > 1 (torchrun, one rank per GPU) every rank processes its own batch:
+the path has no exchange step, so there is no collective in the data path
+("scaling": "weak"); the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+D = 128
+SWEEP_N = 1 << 20
+SWEEP_BITS = (1, 2, 3, 4)
+DEC = dict(B=8, Hq=32, Hkv=8, T=131072)
+METRIC = "vectors quantized/s; packed-KV logits keys/s and % of HBM-bandwidth roofline"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9 and parts[1].isdigit():
+                        rows.append(parts)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(int(r[2]) for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- oracle baseline
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sweep_rate(n_sample: int, bits=SWEEP_BITS, seed: int = 0):
+    """The oracle (as it stands) on a bounded sample of the sweep workload:
+    quantize + pack + dequantize n_sample rows at each b.  Returns vectors/s."""
+    from oracle import codebook as ocb
+    from oracle import turboquant as oq
+    G = synth.gaussian_matrix(D, D, seed, synth.ROT_K)
+    Pi = oq.haar_rotation(G)
+    books = {b: ocb.lloyd_max(b, D) for b in bits}
+    x = synth.to_bf16_exact(synth.scaled_gaussian_rows(n_sample, D, 1.0, seed=seed, outliers=4)).astype(np.float64)
+    t0 = time.perf_counter()
+    for b in bits:
+        c, t = books[b]
+        idx, n, _ = oq.quant_mse(x, Pi, t)
+        oq.pack_codes_vec(idx, b)
+        oq.dequant_mse(idx, n, Pi, c)
+    dt = time.perf_counter() - t0
+    return n_sample * len(bits) / dt, dt
+
+
+def oracle_decode_rate(T_sample: int, seed: int = 0):
+    """Oracle decode for one (batch, kv-head) slice of T_sample tokens and its
+    4 q-heads (logits, softmax, value sum).  Returns keys/s."""
+    from oracle import codebook as ocb
+    from oracle import turboquant as oq
+    Pk = oq.haar_rotation(synth.gaussian_matrix(D, D, seed, synth.ROT_K))
+    Sk = synth.gaussian_matrix(D, D, seed, synth.QJL_K)
+    Pv = oq.haar_rotation(synth.gaussian_matrix(D, D, seed, synth.ROT_V))
+    c3, t3 = ocb.lloyd_max(3, D)
+    c4, t4 = ocb.lloyd_max(4, D)
+    k = synth.kv_head_rows(T_sample, D, 0, 0, 0, seed=seed)
+    v = synth.kv_head_rows(T_sample, D, 1, 0, 0, seed=seed)
+    ks = oq.quant_prod(k, 4, Pk, Sk, t3, c3)
+    vi, vn, _ = oq.quant_mse(v, Pv, t4)
+    q = synth.decode_queries(1, 4, D, seed=seed)
+    t0 = time.perf_counter()
+    vhat = oq.dequant_mse(vi, vn, Pv, c4)
+    oq.attention_decode(q, lambda b, h, qs: oq.prod_estimate(qs, ks["idx"], ks["norms"], ks["signs"], ks["rnorms"],
+                                                             Pk, Sk, c3, 4), lambda b, h: vhat, 1)
+    dt = time.perf_counter() - t0
+    return T_sample / dt, dt
+
+
+# ----------------------------------------------------------------- GPU workloads
+
+class Sweep:
+    """Config: N = 2^20 bf16 vectors (256 MiB > L2), d = 128, b = 1..4."""
+
+    def __init__(self, tq, torch, rank, dev):
+        self.tq, self.torch, self.dev = tq, torch, dev
+        self.N = SWEEP_N
+        G = synth.gaussian_matrix(D, D, 0, synth.ROT_K)
+        Pi = tq.tq_make_rotation(G)
+        self.h = {b: tq.tq_create(D, b, tq.TQ_MSE, Pi) for b in SWEEP_BITS}
+        g = torch.Generator(device=dev).manual_seed(1000 + rank)
+        s = synth.lognormal_channel_scales(D, 1.0, 0)
+        s[synth.outlier_channels(D, 4, 0)] *= 20.0
+        scale = torch.tensor(s, dtype=torch.float32, device=dev)
+        self.x = (torch.randn((self.N, D), generator=g, device=dev) * scale).to(torch.bfloat16)
+        self.codes = {b: torch.empty((self.N, self.h[b].words), dtype=torch.int32, device=dev) for b in SWEEP_BITS}
+        self.norms = {b: torch.empty(self.N, dtype=torch.float32, device=dev) for b in SWEEP_BITS}
+        self.xh = torch.empty((self.N, D), dtype=torch.float32, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.kern = {"quant_mse": [], "dequant_mse": []}
+        self.launches_per_step = 2 * len(SWEEP_BITS)
+
+    def step(self, record=False):
+        tq, torch = self.tq, self.torch
+        for b in SWEEP_BITS:
+            if record:
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(self.stream)
+            tq.tq_quant_mse(self.h[b], self.x, self.codes[b], self.norms[b])
+            if record:
+                e1.record(self.stream)
+            tq.tq_dequant_mse(self.h[b], self.codes[b], self.norms[b], self.xh)
+            if record:
+                e2.record(self.stream)
+                self.kern["quant_mse"].append((e0, e1, b))
+                self.kern["dequant_mse"].append((e1, e2, b))
+
+    def kernel_stats(self):
+        out = {}
+        for name, evs in self.kern.items():
+            ms = [a.elapsed_time(bb) for a, bb, _ in evs]
+            if name == "quant_mse":
+                bytes_ = [self.N * (D * 2 + 16 * b + 4) for _, _, b in evs]
+            else:
+                bytes_ = [self.N * (16 * b + 4 + D * 4) for _, _, b in evs]
+            out[name] = dict(ms_total=sum(ms), launches=len(ms), bytes_total=sum(bytes_))
+        return out
+
+    def units_per_step(self):
+        return self.N * len(SWEEP_BITS)
+
+    # ---- end to end through host buffers
+    def e2e(self, steps, warmup):
+        tq, torch = self.tq, self.torch
+        xh_host = self.x.cpu().pin_memory()
+        outs = {b: (torch.empty(self.codes[b].shape, dtype=torch.int32).pin_memory(),
+                    torch.empty(self.N, dtype=torch.float32).pin_memory()) for b in SWEEP_BITS}
+        xd = torch.empty_like(self.x)
+
+        def one():
+            xd.copy_(xh_host, non_blocking=True)
+            for b in SWEEP_BITS:
+                tq.tq_quant_mse(self.h[b], xd, self.codes[b], self.norms[b])
+                tq.tq_dequant_mse(self.h[b], self.codes[b], self.norms[b], self.xh)
+                outs[b][0].copy_(self.codes[b], non_blocking=True)
+                outs[b][1].copy_(self.norms[b], non_blocking=True)
+
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            one()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / steps
+        h2d = self.x.numel() * 2
+        d2h = sum(self.codes[b].numel() * 4 + self.N * 4 for b in SWEEP_BITS)
+        return ms, h2d, d2h
+
+
+class Decode:
+    """Config: B = 8, Hq = 32, Hkv = 8, d = 128, T = 131072; K prod 4b (3+1), V mse 4b."""
+
+    def __init__(self, tq, torch, rank, dev):
+        self.tq, self.torch, self.dev = tq, torch, dev
+        B, Hq, Hkv, T = DEC["B"], DEC["Hq"], DEC["Hkv"], DEC["T"]
+        self.B, self.Hq, self.Hkv, self.T = B, Hq, Hkv, T
+        Pk = tq.tq_make_rotation(synth.gaussian_matrix(D, D, 0, synth.ROT_K))
+        Sk = synth.gaussian_matrix(D, D, 0, synth.QJL_K)
+        Pv = tq.tq_make_rotation(synth.gaussian_matrix(D, D, 0, synth.ROT_V))
+        self.hk = tq.tq_create(D, 4, tq.TQ_PROD, Pk, Sk)
+        self.hv = tq.tq_create(D, 4, tq.TQ_MSE, Pv)
+        rows = B * Hkv * T
+        self.kcodes = torch.empty((rows, self.hk.words), dtype=torch.int32, device=dev)
+        self.ksigns = torch.empty((rows, tq.sign_words(D)), dtype=torch.int32, device=dev)
+        self.knorms = torch.empty(rows, dtype=torch.float32, device=dev)
+        self.krnorms = torch.empty(rows, dtype=torch.float32, device=dev)
+        self.vcodes = torch.empty((rows, self.hv.words), dtype=torch.int32, device=dev)
+        self.vnorms = torch.empty(rows, dtype=torch.float32, device=dev)
+        g = torch.Generator(device=dev).manual_seed(2000 + rank)
+        chunk = T  # one (batch, kv-head) slice at a time: bounded temporary memory
+        for bh in range(B * Hkv):
+            h = bh % Hkv
+            for kind in (0, 1):
+                s = torch.tensor(synth.lognormal_channel_scales(D, 1.0, 0, 10 + kind, h), dtype=torch.float32,
+                                 device=dev)
+                x = (torch.randn((chunk, D), generator=g, device=dev) * s).to(torch.bfloat16)
+                sl = slice(bh * T, (bh + 1) * T)
+                if kind == 0:
+                    tq.tq_quant_prod(self.hk, x, self.kcodes[sl], self.ksigns[sl], self.knorms[sl], self.krnorms[sl])
+                else:
+                    tq.tq_quant_mse(self.hv, x, self.vcodes[sl], self.vnorms[sl])
+        sq = torch.tensor(synth.lognormal_channel_scales(D, 1.0, 0, 20), dtype=torch.float32, device=dev)
+        self.q = (torch.randn((B, Hq, D), generator=g, device=dev) * sq).to(torch.bfloat16)
+        self.out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, tq.tq_attn_decode_workspace(self.hk, B, Hq, Hkv, T)), dtype=torch.uint8,
+                              device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.kern = []
+        self.scale = 1.0 / math.sqrt(D)
+
+    def step(self, record=False):
+        tq, torch = self.tq, self.torch
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+        tq.tq_attn_decode(self.hk, self.hv, self.q, self.Hkv, self.T, self.T, self.kcodes, self.ksigns, self.knorms,
+                          self.krnorms, self.vcodes, self.vnorms, self.scale, self.out, self.ws)
+        if record:
+            e1.record(self.stream)
+            self.kern.append((e0, e1))
+
+    def bytes_per_step(self):
+        # packed K (48 B codes + 16 B signs + 4 + 4 B norms) + V (64 B codes + 4 B norm) per token
+        return self.B * self.Hkv * self.T * (48 + 16 + 8 + 64 + 4)
+
+    def units_per_step(self):
+        return self.B * self.Hkv * self.T
+
+
+# ----------------------------------------------------------------- driver
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import compressed_kv_cache_turboquant_b200 as tq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device(dev))
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    hbm, bf16, peak_kind = peaks()
+    wl_cls = Sweep if args.workload == "sweep" else Decode
+    wl = wl_cls(tq, torch, rank, dev)
+    for _ in range(args.warmup):
+        wl.step()
+    barrier()
+    with ClockSampler(local) as clk:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            wl.step(record=True)
+        e.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(s.elapsed_time(e) / args.steps)
+    units = wl.units_per_step() * world
+    value = units / (ms / 1e3)
+
+    if args.workload == "sweep":
+        ks = wl.kernel_stats()
+        dom = max(ks, key=lambda k: ks[k]["ms_total"])
+        unit_name = "vectors/s"
+        config = {"workload": "TurboQuant_mse quant+dequant sweep b=1..4, N=2^20 bf16, d=128, lognormal(0,1) "
+                              "channel scales, 4 channels x20 outliers",
+                  "N": SWEEP_N, "d": D, "bits": list(SWEEP_BITS), "input_dtype": "bf16",
+                  "dequant_dtype": "f32", "l2": "inputs larger than L2 (256 MiB bf16 per step per b)",
+                  "parallelism": f"dp{world} (independent batches, no collective)"}
+        launches = wl.launches_per_step * args.steps
+    else:
+        k_ms = sum(a.elapsed_time(b) for a, b in wl.kern)
+        ks = {"attn_decode": dict(ms_total=k_ms, launches=len(wl.kern), bytes_total=wl.bytes_per_step() * len(wl.kern))}
+        dom = "attn_decode"
+        unit_name = "keys/s"
+        config = {"workload": "decode attention over TurboQuant K/V: B=8, Hq=32, Hkv=8, d=128, T=131072, "
+                              "K prod 4b (3+1 QJL), V mse 4b, bf16 queries",
+                  "B": DEC["B"], "Hq": DEC["Hq"], "Hkv": DEC["Hkv"], "T": DEC["T"], "d": D,
+                  "l2": "packed cache 1.17 GB > L2", "parallelism": f"dp{world} (independent caches)"}
+        launches = 3 * args.steps
+    dk = ks[dom]
+    achieved = dk["bytes_total"] / (dk["ms_total"] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
+                "traffic": None,
+                "bytes_per_launch": dk["bytes_total"] / dk["launches"]}
+    kernels = {k: {"avg_ms": v["ms_total"] / v["launches"],
+                   "GBps": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9,
+                   "frac_hbm": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9 / hbm} for k, v in ks.items()}
+
+    e2e = None
+    if args.workload == "sweep":
+        e_ms, h2d, d2h = wl.e2e(max(2, args.steps // 2), 1)
+        e_ms = max_over_ranks(e_ms)
+        e2e = {"value": units / (e_ms / 1e3), "unit": unit_name, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms}
+
+    result = {"metric": METRIC, "value": value, "unit": unit_name, "n_gpus": world, "steps": args.steps,
+              "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+              "vs_baseline": None, "dtype": "f32 (bf16 in, fp32 accumulate)", "data": "synthetic",
+              "config": config, "roofline": roofline, "kernels": kernels, "e2e": e2e,
+              "gpu_launches": launches, "clocks": clk.summary()}
+
+    if args.workload == "sweep" and not args.no_decode:
+        del wl
+        torch.cuda.empty_cache()
+        dl = Decode(tq, torch, rank, dev)
+        for _ in range(args.warmup):
+            dl.step()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(args.steps):
+            dl.step(record=True)
+        e2.record()
+        torch.cuda.synchronize()
+        dms = max_over_ranks(s2.elapsed_time(e2) / args.steps)
+        kms = sum(a.elapsed_time(b) for a, b in dl.kern) / len(dl.kern)
+        gbs = dl.bytes_per_step() / (kms / 1e3) / 1e9
+        result["decode"] = {"value": dl.units_per_step() * world / (dms / 1e3), "unit": "keys/s",
+                            "ms_per_step": dms, "GBps": gbs, "frac_hbm": gbs / hbm,
+                            "bytes_per_step": dl.bytes_per_step(),
+                            "config": "B=8, Hq=32, Hkv=8, d=128, T=131072, K prod 4b, V mse 4b"}
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        if args.workload == "sweep":
+            rate, dt = oracle_sweep_rate(args.cpu_sample)
+            sample = f"{args.cpu_sample} vectors of the sweep workload at each b=1..4 ({dt:.1f} s)"
+        else:
+            rate, dt = oracle_decode_rate(args.cpu_sample)
+            sample = f"one (batch, kv-head) slice of {args.cpu_sample} tokens, 4 q-heads ({dt:.1f} s)"
+        result["cpu_baseline"] = {"value": rate, "unit": unit_name, "cores": cpu_threads(), "kind": "oracle",
+                                  "sample": sample}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    fn = oracle_sweep_rate if args.workload == "sweep" else oracle_decode_rate
+    for i in range(args.warmup + args.steps):
+        rate, dt = fn(args.ref_sample)
+        if i >= args.warmup:
+            times.append(dt)
+    per = args.ref_sample * (len(SWEEP_BITS) if args.workload == "sweep" else 1)
+    value = per / (sum(times) / len(times))
+    unit = "vectors/s" if args.workload == "sweep" else "keys/s"
+    cores = cpu_threads()
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample_per_step": args.ref_sample},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.ref_sample} units per step of the {args.workload} workload"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["sweep", "decode"], default="sweep")
+    ap.add_argument("--cpu-sample", type=int, default=None)
+    ap.add_argument("--ref-sample", type=int, default=None)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.cpu_sample is None:
+        args.cpu_sample = 1 << 19 if args.workload == "sweep" else 1 << 17
+    if args.ref_sample is None:
+        args.ref_sample = 1 << 14 if args.workload == "sweep" else 1 << 13
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,169 @@
+"""Thin Python binding of the C ABI (include/tq.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls and forwards
+device pointers of torch tensors (``data_ptr()``) and the current CUDA
+stream.  No arithmetic of the method happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import (TQ_BF16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQError, check, lib)
+
+__all__ = [
+    "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQError", "Handle", "code_words", "sign_words",
+    "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
+    "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
+]
+
+
+def code_words(b: int, d: int) -> int:
+    return ((d + 31) // 32) * b
+
+
+def sign_words(d: int) -> int:
+    return (d + 31) // 32
+
+
+def _dptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor (this library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype == torch.bfloat16:
+        return TQ_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def tq_version() -> str:
+    return lib.tq_version().decode()
+
+
+def tq_make_codebook(b: int, d: int) -> tuple[np.ndarray, np.ndarray]:
+    c = np.zeros(2 ** b)
+    t = np.zeros(2 ** b - 1)
+    check("tq_make_codebook", lib.tq_make_codebook(b, d, _dptr(c), _dptr(t)))
+    return c, t
+
+
+def tq_make_rotation(G: np.ndarray) -> np.ndarray:
+    G = np.ascontiguousarray(G, dtype=np.float64)
+    d = G.shape[0]
+    Pi = np.zeros((d, d))
+    check("tq_make_rotation", lib.tq_make_rotation(d, _dptr(G), _dptr(Pi)))
+    return Pi
+
+
+class Handle:
+    """Owns a tq_handle (device constants); destroyed with the object."""
+
+    def __init__(self, ptr: int, d: int, b: int, variant: int):
+        self.ptr = ptr
+        self.d, self.b, self.variant = d, b, variant
+        self.bm = b if variant == TQ_MSE else b - 1
+
+    @property
+    def words(self) -> int:
+        return code_words(self.bm, self.d)
+
+    def close(self):
+        if self.ptr:
+            check("tq_destroy", lib.tq_destroy(self.ptr))
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def tq_create(d: int, b: int, variant: int, Pi: np.ndarray, S: np.ndarray | None = None,
+              centroids: np.ndarray | None = None) -> Handle:
+    Pi = np.ascontiguousarray(Pi, dtype=np.float64)
+    Sa = None if S is None else np.ascontiguousarray(S, dtype=np.float64)
+    ca = None if centroids is None else np.ascontiguousarray(centroids, dtype=np.float64)
+    h = ctypes.c_void_p()
+    check("tq_create", lib.tq_create(ctypes.byref(h), d, b, variant, _dptr(Pi),
+                                     None if Sa is None else _dptr(Sa), None if ca is None else _dptr(ca)))
+    return Handle(h.value, d, b, variant)
+
+
+def tq_quant_mse(h: Handle, x: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
+                 out_stride: int = 1, stream=None) -> None:
+    N = x.shape[0]
+    check("tq_quant_mse", lib.tq_quant_mse(h.ptr, _ptr(x), _dtype_code(x), N, x.shape[1], _ptr(codes),
+                                           _ptr(norms), out_stride, _stream(stream)))
+
+
+def tq_dequant_mse(h: Handle, codes: torch.Tensor, norms: torch.Tensor, out: torch.Tensor,
+                   stream=None) -> None:
+    check("tq_dequant_mse", lib.tq_dequant_mse(h.ptr, _ptr(codes), _ptr(norms), codes.shape[0], _ptr(out),
+                                               _dtype_code(out), _stream(stream)))
+
+
+def tq_quant_prod(h: Handle, x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor,
+                  norms: torch.Tensor, rnorms: torch.Tensor, out_stride: int = 1, stream=None) -> None:
+    N = x.shape[0]
+    check("tq_quant_prod", lib.tq_quant_prod(h.ptr, _ptr(x), _dtype_code(x), N, x.shape[1], _ptr(codes),
+                                             _ptr(signs), _ptr(norms), _ptr(rnorms), out_stride,
+                                             _stream(stream)))
+
+
+def tq_ip_scores_workspace(h: Handle, nq: int, N: int, topk: int = 0) -> int:
+    return int(lib.tq_ip_scores_workspace(h.ptr, nq, N, topk))
+
+
+def tq_ip_scores(h: Handle, q: torch.Tensor, codes: torch.Tensor, signs, norms: torch.Tensor, rnorms,
+                 scores=None, topk: int = 0, top_idx=None, top_val=None, workspace=None,
+                 stream=None) -> None:
+    nq, N = q.shape[0], codes.shape[0]
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_ip_scores_workspace(h, nq, N, topk)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_ip_scores", lib.tq_ip_scores(h.ptr, _ptr(q), nq, _ptr(codes), _ptr(signs), _ptr(norms),
+                                           _ptr(rnorms), N, _ptr(scores), topk, _ptr(top_idx),
+                                           _ptr(top_val), _ptr(workspace), workspace.numel(),
+                                           _stream(stream)))
+
+
+def tq_attn_decode_workspace(hk: Handle, B: int, Hq: int, Hkv: int, T: int) -> int:
+    return int(lib.tq_attn_decode_workspace(hk.ptr, B, Hq, Hkv, T))
+
+
+def tq_attn_decode(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, kv_stride: int,
+                   kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale: float, out: torch.Tensor,
+                   workspace=None, stream=None) -> None:
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_attn_decode_workspace(hk, B, Hq, Hkv, T)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_attn_decode", lib.tq_attn_decode(hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T,
+                                               kv_stride, _ptr(kcodes), _ptr(ksigns), _ptr(knorms),
+                                               _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale),
+                                               _ptr(out), _ptr(workspace), workspace.numel(),
+                                               _stream(stream)))

@@ -1,0 +1,334 @@
+// C ABI of the TurboQuant hot path: argument checks, handle management and
+// dispatch to the kernels.  The operations are defined in include/tq.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "tq_internal.h"
+
+namespace tqi {
+
+static thread_local char g_err[512] = "";
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int clear_error() {
+  g_err[0] = '\0';
+  return TQ_OK;
+}
+
+static int cuda_error(const char* where, int e) {
+  return set_error(TQ_ECUDA, "%s: %s", where, cudaGetErrorString((cudaError_t)e));
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define TQ_CHECK_ALIGN(p, name)                                                        \
+  do {                                                                                 \
+    if ((p) && !aligned16(p)) return set_error(TQ_EALIGN, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// decode attention: context splits per (batch, q-head)
+static int decode_splits(int B, int Hq, int64_t T, int sm_count) {
+  // enough CTAs to fill the machine a few times, each split >= 512 tokens
+  int64_t want = (int64_t)sm_count * 4 / std::max(1, B * Hq);
+  int64_t cap = (T + 511) / 512;
+  int64_t s = std::max<int64_t>(1, std::min<int64_t>(want > 0 ? want : 1, cap));
+  return (int)std::min<int64_t>(s, 256);
+}
+
+}  // namespace tqi
+
+using namespace tqi;
+
+extern "C" const char* tq_last_error(void) { return g_err; }
+extern "C" const char* tq_version(void) { return "tq-b200 0.1 (sm_100a)"; }
+
+extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double* Pi,
+                         const double* S, const double* centroids) {
+  if (!out || !Pi) return set_error(TQ_EINVAL, "tq_create: NULL handle or rotation");
+  *out = nullptr;
+  if (variant != TQ_MSE && variant != TQ_PROD)
+    return set_error(TQ_EUNSUPPORTED, "tq_create: unknown variant %d", variant);
+  if (d < 8 || d > TQ_MAX_DIM || d % 8 != 0)
+    return set_error(TQ_EUNSUPPORTED, "tq_create: d = %d (need 8 <= d <= %d, d %% 8 == 0)", d,
+                     TQ_MAX_DIM);
+  const int bm = (variant == TQ_MSE) ? b : b - 1;
+  if (bm < 1 || bm > kMaxMseBits)
+    return set_error(TQ_EUNSUPPORTED, "tq_create: b = %d unsupported for this variant", b);
+  if (variant == TQ_PROD && !S) return set_error(TQ_EINVAL, "tq_create: TQ_PROD needs S");
+
+  tq_ctx* h = new (std::nothrow) tq_ctx();
+  if (!h) return set_error(TQ_ENOMEM, "tq_create: out of host memory");
+  h->d = d;
+  h->b = b;
+  h->variant = variant;
+  h->bm = bm;
+  const int K = 1 << bm;
+  if (centroids) {
+    for (int k = 0; k < K; ++k) h->host_centroids[k] = centroids[k];
+    for (int k = 0; k + 1 < K; ++k) {
+      if (!(centroids[k] < centroids[k + 1])) {
+        delete h;
+        return set_error(TQ_EINVAL, "tq_create: centroids must be strictly ascending");
+      }
+      h->host_thresholds[k] = 0.5 * (centroids[k] + centroids[k + 1]);
+    }
+  } else {
+    int rc = tq_make_codebook(bm, d, h->host_centroids, h->host_thresholds);
+    if (rc != TQ_OK) {
+      delete h;
+      return rc;
+    }
+  }
+  int e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_error("tq_create", e);
+  }
+
+  // host staging of every constant (float32), then one upload
+  const size_t dd = (size_t)d * d;
+  std::vector<float> Pf(dd), PTf(dd), Sf, TTf;
+  for (int j = 0; j < d; ++j)
+    for (int i = 0; i < d; ++i) {
+      Pf[(size_t)j * d + i] = (float)Pi[(size_t)j * d + i];
+      PTf[(size_t)i * d + j] = (float)Pi[(size_t)j * d + i];
+    }
+  if (variant == TQ_PROD) {
+    Sf.resize(dd);
+    TTf.resize(dd);
+    for (size_t k = 0; k < dd; ++k) Sf[k] = (float)S[k];
+    // T = S Pi^T in float64: T[j][i] = sum_k S[j][k] Pi[i][k]; stored as TT[i][j]
+    std::vector<double> row(d);
+    for (int j = 0; j < d; ++j)
+      for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        const double* s = S + (size_t)j * d;
+        const double* p = Pi + (size_t)i * d;
+        for (int k = 0; k < d; ++k) acc += s[k] * p[k];
+        TTf[(size_t)i * d + j] = (float)acc;
+      }
+  }
+  std::vector<float> cf(K), tf(K);
+  for (int k = 0; k < K; ++k) cf[k] = (float)h->host_centroids[k];
+  for (int k = 0; k + 1 < K; ++k) tf[k] = (float)h->host_thresholds[k];
+
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t oPi = take(dd * 4), oPT = take(dd * 4);
+  const size_t oS = (variant == TQ_PROD) ? take(dd * 4) : 0;
+  const size_t oTT = (variant == TQ_PROD) ? take(dd * 4) : 0;
+  const size_t oC = take(64 * 4), oT = take(64 * 4);
+  h->block_bytes = off;
+  e = cudaMalloc(&h->block, h->block_bytes);
+  if (e != cudaSuccess) {
+    delete h;
+    return set_error(TQ_ENOMEM, "tq_create: cudaMalloc of %zu bytes failed", off);
+  }
+  char* base = (char*)h->block;
+  h->dev.Pi = (float*)(base + oPi);
+  h->dev.PiT = (float*)(base + oPT);
+  h->dev.centroids = (float*)(base + oC);
+  h->dev.thresholds = (float*)(base + oT);
+  if (variant == TQ_PROD) {
+    h->dev.S = (float*)(base + oS);
+    h->dev.TT = (float*)(base + oTT);
+  }
+  e = cudaMemcpy(h->dev.Pi, Pf.data(), dd * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->dev.PiT, PTf.data(), dd * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->dev.centroids, cf.data(), K * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && K > 1)
+    e = cudaMemcpy(h->dev.thresholds, tf.data(), (K - 1) * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && variant == TQ_PROD) {
+    e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
+  }
+  if (e != cudaSuccess) {
+    cudaFree(h->block);
+    delete h;
+    return cuda_error("tq_create upload", e);
+  }
+  *out = h;
+  return clear_error();
+}
+
+extern "C" int tq_destroy(tq_handle h) {
+  if (!h) return clear_error();
+  int e = cudaDeviceSynchronize();
+  int e2 = cudaFree(h->block);
+  delete h;
+  if (e != cudaSuccess) return cuda_error("tq_destroy", e);
+  if (e2 != cudaSuccess) return cuda_error("tq_destroy", e2);
+  return clear_error();
+}
+
+extern "C" int tq_handle_info(tq_handle h, int* d, int* b, int* variant, int* mse_bits) {
+  if (!h) return set_error(TQ_EINVAL, "tq_handle_info: NULL handle");
+  if (d) *d = h->d;
+  if (b) *b = h->b;
+  if (variant) *variant = h->variant;
+  if (mse_bits) *mse_bits = h->bm;
+  return clear_error();
+}
+
+static int check_quant_args(const char* fn, tq_handle h, int want_variant, const void* x, int dtype,
+                            int64_t N, int64_t x_stride, const void* codes, const void* norms,
+                            int64_t out_stride) {
+  if (!h) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
+  if (h->variant != want_variant) return set_error(TQ_EINVAL, "%s: wrong handle variant", fn);
+  if (N < 0) return set_error(TQ_EINVAL, "%s: N < 0", fn);
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return set_error(TQ_EUNSUPPORTED, "%s: dtype %d", fn, dtype);
+  if (x_stride < h->d || x_stride % 8 != 0)
+    return set_error(TQ_EINVAL, "%s: x_stride %lld (need >= d and a multiple of 8)", fn,
+                     (long long)x_stride);
+  if (out_stride < 1) return set_error(TQ_EINVAL, "%s: out_stride < 1", fn);
+  if (N > 0 && (!x || !codes || !norms)) return set_error(TQ_EINVAL, "%s: NULL pointer", fn);
+  TQ_CHECK_ALIGN(x, "x");
+  TQ_CHECK_ALIGN(codes, "codes");
+  TQ_CHECK_ALIGN(norms, "norms");
+  return TQ_OK;
+}
+
+extern "C" int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                            uint32_t* codes, float* norms, int64_t out_stride, void* stream) {
+  int rc = check_quant_args("tq_quant_mse", h, TQ_MSE, x, dtype, N, x_stride, codes, norms, out_stride);
+  if (rc) return rc;
+  if (N == 0) return clear_error();
+  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream);
+  return e ? cuda_error("tq_quant_mse", e) : clear_error();
+}
+
+extern "C" int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                             uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
+                             int64_t out_stride, void* stream) {
+  int rc = check_quant_args("tq_quant_prod", h, TQ_PROD, x, dtype, N, x_stride, codes, norms, out_stride);
+  if (rc) return rc;
+  if (N > 0 && (!signs || !rnorms)) return set_error(TQ_EINVAL, "tq_quant_prod: NULL pointer");
+  TQ_CHECK_ALIGN(signs, "signs");
+  TQ_CHECK_ALIGN(rnorms, "rnorms");
+  if (N == 0) return clear_error();
+  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream);
+  return e ? cuda_error("tq_quant_prod", e) : clear_error();
+}
+
+extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* norms, int64_t N,
+                              void* out, int out_dtype, void* stream) {
+  if (!h) return set_error(TQ_EINVAL, "tq_dequant_mse: NULL handle");
+  if (N < 0) return set_error(TQ_EINVAL, "tq_dequant_mse: N < 0");
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16)
+    return set_error(TQ_EUNSUPPORTED, "tq_dequant_mse: out_dtype %d", out_dtype);
+  if (N > 0 && (!codes || !norms || !out)) return set_error(TQ_EINVAL, "tq_dequant_mse: NULL pointer");
+  TQ_CHECK_ALIGN(codes, "codes");
+  TQ_CHECK_ALIGN(norms, "norms");
+  TQ_CHECK_ALIGN(out, "out");
+  if (N == 0) return clear_error();
+  int e = launch_dequant_simple(h, codes, norms, N, out, out_dtype, stream);
+  return e ? cuda_error("tq_dequant_mse", e) : clear_error();
+}
+
+// workspace of tq_ip_scores: rotated + projected queries, and the score matrix
+// when only the top-k is requested
+extern "C" size_t tq_ip_scores_workspace(tq_handle h, int64_t nq, int64_t N, int topk) {
+  if (!h || nq < 0 || N < 0) return 0;
+  size_t bytes = align_up((size_t)nq * h->d * 4, 256) * 2;
+  if (topk > 0) bytes += align_up((size_t)nq * N * 4, 256);
+  return bytes;
+}
+
+extern "C" int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint32_t* codes,
+                            const uint32_t* signs, const float* norms, const float* rnorms,
+                            int64_t N, float* scores, int topk, int32_t* top_idx, float* top_val,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return set_error(TQ_EINVAL, "tq_ip_scores: NULL handle");
+  if (nq < 0 || N < 0) return set_error(TQ_EINVAL, "tq_ip_scores: negative size");
+  if (topk < 0 || topk > TQ_MAX_TOPK || (topk > 0 && topk > N && N > 0))
+    return set_error(TQ_EINVAL, "tq_ip_scores: topk %d (need 0..min(N, %d))", topk, TQ_MAX_TOPK);
+  const bool prod = h->variant == TQ_PROD;
+  if (nq > 0 && N > 0) {
+    if (!q || !codes || !norms || (prod && (!signs || !rnorms)))
+      return set_error(TQ_EINVAL, "tq_ip_scores: NULL input");
+    if (!scores && topk == 0) return set_error(TQ_EINVAL, "tq_ip_scores: no output requested");
+    if (topk > 0 && (!top_idx || !top_val)) return set_error(TQ_EINVAL, "tq_ip_scores: NULL top-k output");
+  }
+  for (const void* p : {(const void*)q, (const void*)codes, (const void*)signs, (const void*)norms,
+                        (const void*)rnorms, (const void*)scores, (const void*)top_idx,
+                        (const void*)top_val, (const void*)workspace})
+    TQ_CHECK_ALIGN(p, "a device pointer");
+  if (nq == 0 || N == 0) return clear_error();
+  const size_t need = tq_ip_scores_workspace(h, nq, N, topk);
+  if (!workspace || ws_bytes < need)
+    return set_error(TQ_EWORKSPACE, "tq_ip_scores: workspace %zu < %zu bytes", ws_bytes, need);
+  char* ws = (char*)workspace;
+  float* qrot = (float*)ws;
+  float* qproj = (float*)(ws + align_up((size_t)nq * h->d * 4, 256));
+  float* sc = scores;
+  if (topk > 0 && !scores) sc = (float*)(ws + 2 * align_up((size_t)nq * h->d * 4, 256));
+  int e = launch_query_prep(h, q, TQ_F32, nq, qrot, prod ? qproj : nullptr, stream);
+  if (!e) e = launch_scores_simple(h, qrot, qproj, nq, codes, signs, norms, rnorms, N, sc, stream);
+  if (!e && topk > 0) e = launch_topk_simple(sc, nq, N, topk, top_idx, top_val, stream);
+  return e ? cuda_error("tq_ip_scores", e) : clear_error();
+}
+
+extern "C" size_t tq_attn_decode_workspace(tq_handle hk, int B, int Hq, int Hkv, int64_t T) {
+  if (!hk || B < 0 || Hq < 0 || Hkv <= 0 || T < 0) return 0;
+  const int splits = decode_splits(B, Hq, T, hk->sm_count);
+  const size_t q = align_up((size_t)B * Hq * hk->d * 4, 256);
+  return 2 * q + align_up((size_t)B * Hq * splits * (hk->d + 2) * 4, 256);
+}
+
+extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq,
+                              int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
+                              const uint32_t* ksigns, const float* knorms, const float* krnorms,
+                              const uint32_t* vcodes, const float* vnorms, float scale, float* out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!hk || !hv) return set_error(TQ_EINVAL, "tq_attn_decode: NULL handle");
+  if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)
+    return set_error(TQ_EINVAL, "tq_attn_decode: need a TQ_PROD key handle and a TQ_MSE value handle");
+  if (hk->d != hv->d) return set_error(TQ_EINVAL, "tq_attn_decode: key and value d differ");
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16)
+    return set_error(TQ_EUNSUPPORTED, "tq_attn_decode: q_dtype %d", q_dtype);
+  if (B < 0 || Hq < 0 || Hkv <= 0 || (Hq % Hkv) != 0 || T < 1 || kv_stride < T)
+    return set_error(TQ_EINVAL, "tq_attn_decode: bad shape (B=%d Hq=%d Hkv=%d T=%lld stride=%lld)", B,
+                     Hq, Hkv, (long long)T, (long long)kv_stride);
+  if (!std::isfinite(scale)) return set_error(TQ_EINVAL, "tq_attn_decode: scale is not finite");
+  if (B == 0 || Hq == 0) return clear_error();
+  if (!q || !kcodes || !ksigns || !knorms || !krnorms || !vcodes || !vnorms || !out)
+    return set_error(TQ_EINVAL, "tq_attn_decode: NULL pointer");
+  for (const void* p : {(const void*)q, (const void*)kcodes, (const void*)ksigns, (const void*)knorms,
+                        (const void*)krnorms, (const void*)vcodes, (const void*)vnorms,
+                        (const void*)out, (const void*)workspace})
+    TQ_CHECK_ALIGN(p, "a device pointer");
+  const size_t need = tq_attn_decode_workspace(hk, B, Hq, Hkv, T);
+  if (!workspace || ws_bytes < need)
+    return set_error(TQ_EWORKSPACE, "tq_attn_decode: workspace %zu < %zu bytes", ws_bytes, need);
+  const int splits = decode_splits(B, Hq, T, hk->sm_count);
+  char* ws = (char*)workspace;
+  const size_t qb = align_up((size_t)B * Hq * hk->d * 4, 256);
+  float* qrot = (float*)ws;
+  float* qproj = (float*)(ws + qb);
+  float* partials = (float*)(ws + 2 * qb);
+  int e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)B * Hq, qrot, qproj, stream);
+  if (!e)
+    e = launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms,
+                             krnorms, vcodes, vnorms, scale, splits, partials, out, stream);
+  return e ? cuda_error("tq_attn_decode", e) : clear_error();
+}

@@ -1,0 +1,68 @@
+// Internal declarations shared by the host API and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "tq.h"
+
+namespace tqi {
+
+// Thread-local error text behind tq_last_error(); returns `code` for chaining.
+int set_error(int code, const char* fmt, ...);
+int clear_error();
+
+constexpr int kMaxMseBits = 4;
+
+// Device-resident constants of one quantizer instance (one cudaMalloc block).
+struct DevConsts {
+  float* Pi = nullptr;          // [d][d] row-major, y = Pi x
+  float* PiT = nullptr;         // [d][d] row-major transpose of Pi
+  float* S = nullptr;           // [d][d] QJL projection (prod), for the query side S q
+  float* TT = nullptr;          // [d][d] transpose of T = S Pi^T (prod): [i][j] = T[j][i]
+  float* centroids = nullptr;   // [2^bm]
+  float* thresholds = nullptr;  // [2^bm - 1]
+  // tensor-core operands: rotation / projection split into bf16 pieces,
+  // pre-arranged in the shared-memory layout the MMA kernels consume
+  uint16_t* Pi_bf16 = nullptr;  // [pieces][d*d]
+  uint16_t* T_bf16 = nullptr;   // [pieces][d*d]
+  // decode tables
+  uint32_t* lut_f16 = nullptr;  // packed fp16 centroid byte tables
+};
+
+}  // namespace tqi
+
+struct tq_ctx {
+  int d = 0, b = 0, variant = 0, bm = 0;  // bm: mse bits (b for MSE, b-1 for PROD)
+  int device = 0;
+  int sm_count = 0;
+  void* block = nullptr;  // the single device allocation
+  size_t block_bytes = 0;
+  tqi::DevConsts dev;
+  // host copies (float64) kept for diagnostics
+  double host_centroids[16] = {0};
+  double host_thresholds[15] = {0};
+};
+
+namespace tqi {
+
+// ---- launchers (kernels_*.cu); all return cudaError_t as int ----
+int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                        uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
+                        int64_t out_stride, void* stream);
+int launch_dequant_simple(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_t N,
+                          void* out, int out_dtype, void* stream);
+int launch_query_prep(const tq_ctx* h, const float* q, int q_dtype, int64_t nq, float* qrot,
+                      float* qproj, void* stream);
+int launch_scores_simple(const tq_ctx* h, const float* qrot, const float* qproj, int64_t nq,
+                         const uint32_t* codes, const uint32_t* signs, const float* norms,
+                         const float* rnorms, int64_t N, float* scores, void* stream);
+int launch_topk_simple(const float* scores, int64_t nq, int64_t N, int k, int32_t* top_idx,
+                       float* top_val, void* stream);
+int launch_decode_simple(const tq_ctx* hk, const tq_ctx* hv, const float* qrot,
+                         const float* qproj, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
+                         const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
+                         const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                         float scale, int splits, float* partials, float* out, void* stream);
+
+}  // namespace tqi

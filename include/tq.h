@@ -1,0 +1,258 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) TurboQuant hot path.
+ *
+ * TurboQuant is an online, data-oblivious vector quantizer.  Pages cited below:
+ *   [ttakun]  "KV缓存52GB瞬间爆内存？TurboQuant随机旋转+标量量化如何把LLM长上下文推理成本
+ *             砍到1/16且失真逼近理论极限" (ttakun.com/news/45354)
+ *   [tmdm]    "谷歌悄悄扔下一颗“性能核弹”：KV缓存压缩6倍，推理提速8倍，还不用重训模型"
+ *             (tmdm.cn/turboquant-kv-compression)
+ *   [admirer] m.admirer.cn report on "TurboQuant: Online Vector Quantization with
+ *             Near-optimal Distortion Rate" (arXiv 2504.19874)
+ *   [tq.net]  turboquant.net/zh, "TurboQuant 最近的进展和外溢影响"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Return value: TQ_OK (0) or one of the TQ_E* codes below.  On error the
+ *   call has launched nothing; tq_last_error() returns a message for the
+ *   calling thread.
+ * - Device pointers ("dev") are caller-owned device memory on the handle's
+ *   device; the library never allocates, frees or retains them.  Host
+ *   pointers ("host") are read or written before the call returns.
+ * - Every device call is asynchronous on `stream` (a cudaStream_t, NULL = the
+ *   legacy default stream) and does not synchronise.  Outputs are complete
+ *   when the stream reaches the call.
+ * - Alignment: every device pointer must be 16-byte aligned (TQ_EALIGN).
+ * - A handle holds only constants (rotation, projection, codebook) uploaded
+ *   by tq_create to the device that was current at that time.  Concurrent
+ *   calls on one handle from several streams are safe; destroying a handle
+ *   while work that uses it is in flight is not.
+ *
+ * Packed code layout (the pages say only that 32-bit coordinates become 2- or
+ * 4-bit integers, [ttakun, "为什么随机旋转是整个算法的底层杠杆"]).  A vector's d rotated
+ * coordinates form G = ceil(d/32) groups of 32 (coordinates past d are zero);
+ * group g owns the b consecutive uint32 words g*b .. g*b+b-1, so one vector
+ * takes TQ_CODE_WORDS(b, d) = G*b words.  Inside a group, for local coordinate i:
+ *   b = 1: word 0 bit i = idx_i
+ *   b = 2: word k bits 2j..2j+1 = idx_{16k+j}          (k < 2, j < 16)
+ *   b = 3: word k bits 4j..4j+2 = idx_{8k+j}           (k < 3, j < 8)
+ *          word k bit  4j+3     = bit k of idx_{24+j}
+ *   b = 4: word k bits 4j..4j+3 = idx_{8k+j}           (k < 4, j < 8)
+ * QJL sign bits use the b = 1 layout (bit set <=> (S r)_i >= 0).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define TQ_OK 0
+#define TQ_EINVAL 1        /* NULL pointer, negative size, inconsistent shapes */
+#define TQ_EUNSUPPORTED 2  /* b, d, dtype or variant outside the supported set */
+#define TQ_EALIGN 3        /* a device pointer is not 16-byte aligned */
+#define TQ_ECUDA 4         /* a CUDA runtime call or launch failed (see tq_last_error) */
+#define TQ_ENOMEM 5        /* tq_create could not allocate the handle's constants */
+#define TQ_EWORKSPACE 6    /* the workspace passed is smaller than required */
+
+/* element types */
+#define TQ_F32 0
+#define TQ_BF16 1
+
+/* variants */
+#define TQ_MSE 0  /* TurboQuant_mse: b bits per coordinate */
+#define TQ_PROD 1 /* TurboQuant_prod: (b-1)-bit mse + 1-bit QJL of the residual */
+
+#define TQ_MAX_DIM 4096
+#define TQ_CODE_WORDS(b, d) ((((d) + 31) / 32) * (b))
+#define TQ_SIGN_WORDS(d) (((d) + 31) / 32)
+
+typedef struct tq_ctx* tq_handle;
+
+/* ---------------------------------------------------------------- host setup */
+
+/*
+ * tq_make_codebook -- Lloyd-Max scalar quantizer for one rotated coordinate.
+ * [ttakun, "为什么随机旋转是整个算法的底层杠杆"]: after the rotation each coordinate
+ * follows a known Beta-shaped law and is quantized with a precomputed Lloyd-Max
+ * quantizer; the law is f(x) = Gamma(d/2)/(sqrt(pi) Gamma((d-1)/2)) (1-x^2)^((d-3)/2)
+ * on [-1, 1] [tq.net, "TurboQuant 两阶段算法", 坐标分布公式]; computed once offline
+ * [tq.net, "实现步骤草图", 预计算 Lloyd-Max 质心].
+ *   b           bits, 1..4
+ *   d           dimension, 3..TQ_MAX_DIM
+ *   centroids   host out, [2^b] ascending, float64, symmetric (c_k = -c_{2^b-1-k})
+ *   thresholds  host out, [2^b - 1], midpoints of adjacent centroids (may be NULL)
+ * Iterates to the float64 fixed point.  Pure host code; needs no GPU.
+ * Errors: TQ_EINVAL (NULL centroids), TQ_EUNSUPPORTED (b or d out of range).
+ */
+TQ_API int tq_make_codebook(int b, int d, double* centroids, double* thresholds);
+
+/*
+ * tq_make_rotation -- random orthogonal rotation from a Gaussian matrix.
+ * [ttakun, "为什么随机旋转是整个算法的底层杠杆"]: the rotation is obtained from the QR
+ * decomposition of a random Gaussian matrix; [tq.net, "实现步骤草图", 生成随机旋转矩阵].
+ *   d    dimension, 1..TQ_MAX_DIM
+ *   G    host in, [d*d] row-major float64 (caller's N(0,1) draws)
+ *   Pi   host out, [d*d] row-major float64: Q of G = Q R (Householder), with
+ *        column j multiplied by sign(R_jj) so that R has a positive diagonal
+ *        (Haar distributed).  The quantizer uses y = Pi x.
+ * Pure host code.  Errors: TQ_EINVAL, TQ_EUNSUPPORTED (d), TQ_ENOMEM.
+ */
+TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
+
+/*
+ * tq_create -- upload the constants of one quantizer instance.
+ *   h          host out, the new handle
+ *   d          dimension; supported: 8..TQ_MAX_DIM with d % 8 == 0
+ *   b          total bits per coordinate: TQ_MSE 1..4, TQ_PROD 2..4
+ *              (TQ_PROD spends b-1 bits on the mse stage and 1 on QJL)
+ *   variant    TQ_MSE or TQ_PROD
+ *   Pi         host in, [d*d] row-major float64 orthogonal rotation (y = Pi x)
+ *   S          host in, [d*d] row-major float64 QJL projection (m = d rows);
+ *              NULL for TQ_MSE.  Reading: the pages never give S's shape; the
+ *              estimator's sqrt(pi/2)/d factor implies m = d.
+ *   centroids  host in, [2^bm] ascending (bm = b for TQ_MSE, b-1 for TQ_PROD),
+ *              or NULL to use tq_make_codebook(bm, d)
+ * Allocates device memory for the constants on the current device (the only
+ * allocation the library makes) and synchronises with it.
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
+ */
+TQ_API int tq_create(tq_handle* h, int d, int b, int variant, const double* Pi, const double* S,
+              const double* centroids);
+
+/* tq_destroy -- free the handle's device constants (synchronises the device). NULL is a no-op. */
+TQ_API int tq_destroy(tq_handle h);
+
+/* tq_handle_info -- d, b, variant and bm (mse bits) of a handle; any out pointer may be NULL. */
+TQ_API int tq_handle_info(tq_handle h, int* d, int* b, int* variant, int* mse_bits);
+
+/* ---------------------------------------------------------------- hot path */
+
+/*
+ * tq_quant_mse -- TurboQuant_mse quantization of N vectors
+ * ([ttakun, "TurboQuant_mse vs TurboQuant_prod两个变体的精确分工"]: store the norm as
+ * float32, rotate, quantize every coordinate independently against the
+ * precomputed codebook; [tq.net, "实现步骤草图", quant 原语]).
+ * n_i = ||x_i||, y = Pi x_i / n_i, idx_j = #{k : y_j >= t_k} (ties go up),
+ * codes packed as described at the top of this file.  x_i = 0 gives n_i = 0
+ * and the codes of y = 0.
+ *   h         handle with variant TQ_MSE
+ *   x         dev in, N rows of d elements of `dtype` (TQ_F32 or TQ_BF16),
+ *             row i at x + i*x_stride elements; x_stride >= d, x_stride % 8 == 0
+ *   N         number of vectors (0 is a no-op)
+ *   codes     dev out, row i at codes + i*out_stride*TQ_CODE_WORDS(b, d)
+ *   norms     dev out, float32, norms[i*out_stride]
+ *   out_stride  >= 1; 1 for dense outputs (a larger stride writes every
+ *             out_stride-th slot, e.g. one token slot per head of a KV cache)
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                 uint32_t* codes, float* norms, int64_t out_stride, void* stream);
+
+/*
+ * tq_dequant_mse -- x_hat_i = n_i * Pi^T c[idx_i]
+ * ([ttakun, same section]: rebuild by rotating back and rescaling;
+ * [tq.net, "实现步骤草图", dequant 原语]).
+ *   h       handle with variant TQ_MSE (or TQ_PROD: dequantizes its mse stage)
+ *   codes   dev in, [N][TQ_CODE_WORDS(bm, d)]
+ *   norms   dev in, [N] float32
+ *   out     dev out, [N][d] of out_dtype (TQ_F32 or TQ_BF16)
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* norms, int64_t N, void* out,
+                   int out_dtype, void* stream);
+
+/*
+ * tq_quant_prod -- TurboQuant_prod quantization
+ * ([ttakun, "TurboQuant_mse vs TurboQuant_prod两个变体的精确分工"]: (b-1)-bit mse gives
+ * x_hat and the residual r, then 1-bit QJL of r; [tmdm, "双剑合璧：PolarQuant + QJL",
+ * ✦ QJL]; [admirer, "第二步：1 bit 算力帶來的「神級校準」"]).
+ * Computes the mse stage as tq_quant_mse with bm = b-1 bits, then in the
+ * rotated frame u = y - c[idx] (so r = n Pi^T u), sign bits of (S r)_j =
+ * n (S Pi^T u)_j (bit set <=> >= 0), and rn = ||r|| = n ||u||.
+ *   x, N, x_stride, out_stride   as tq_quant_mse
+ *   codes    dev out, [N][TQ_CODE_WORDS(b-1, d)]
+ *   signs    dev out, [N][TQ_SIGN_WORDS(d)]
+ *   norms    dev out, [N] float32 ||x||
+ *   rnorms   dev out, [N] float32 ||r||
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                  uint32_t* codes, uint32_t* signs, float* norms, float* rnorms, int64_t out_stride,
+                  void* stream);
+
+/*
+ * tq_ip_scores -- estimated inner products of nq queries with N quantized vectors
+ * ([tmdm, "双剑合璧", ✦ QJL]: the unbiased estimator corrects the quantization error
+ * while the score is computed; [admirer, "內存價格能下來嗎？": nearest-neighbour search).
+ *   TQ_PROD: s = n <Pi q, c[idx]> + rn sqrt(pi/2)/d <S q, sigma>, sigma_j = +-1
+ *   TQ_MSE:  s = n <Pi q, c[idx]>
+ * Each query is rotated (and projected) once.
+ *   q        dev in, [nq][d] float32
+ *   codes, signs, norms, rnorms   dev in, as written by tq_quant_* (signs and
+ *            rnorms are ignored for TQ_MSE and may be NULL)
+ *   scores   dev out, [nq][N] float32, or NULL when topk > 0 and only the
+ *            top-k is wanted
+ *   topk     0, or 1..TQ_MAX_TOPK: also write the topk largest scores per query
+ *            to top_idx [nq][topk] int32 and top_val [nq][topk] float32, by
+ *            score descending (ties: lower index first)
+ *   workspace, ws_bytes   dev scratch of at least tq_ip_scores_workspace(...) bytes
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
+ */
+#define TQ_MAX_TOPK 64
+TQ_API int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint32_t* codes,
+                 const uint32_t* signs, const float* norms, const float* rnorms, int64_t N,
+                 float* scores, int topk, int32_t* top_idx, float* top_val, void* workspace,
+                 size_t ws_bytes, void* stream);
+TQ_API size_t tq_ip_scores_workspace(tq_handle h, int64_t nq, int64_t N, int topk);
+
+/*
+ * tq_attn_decode -- one decode step of attention over a TurboQuant K/V cache
+ * ([tq.net, "实现步骤草图", 集成到 attention]: K and V are stored in TurboQuant form and
+ * QJL is used inside attention; [tmdm, "实测数据"]: attention logits over a 4-bit cache).
+ * For batch b, query head j (kv-head h = j / (Hq/Hkv)):
+ *   logit_t = scale * est(q_bj, k_t)        (TQ_PROD estimator with handle hk)
+ *   out_bj  = sum_t softmax(logit)_t * n_t Pi_V^T c_V[idx_t]   (values with hv, TQ_MSE)
+ * The value sum runs in the rotated frame and Pi_V^T is applied once per output.
+ *   hk, hv      TQ_PROD key handle and TQ_MSE value handle, same d
+ *   q           dev in, [B][Hq][d] of q_dtype (TQ_F32 or TQ_BF16)
+ *   B, Hq, Hkv  batch, query heads, kv-heads (Hq % Hkv == 0)
+ *   T           context length (>= 1)
+ *   kv_stride   token slots per (batch, kv-head) in the cache arrays (>= T):
+ *               token t of (b, h) is row (b*Hkv + h)*kv_stride + t of
+ *   kcodes [..][TQ_CODE_WORDS(bk-1, d)], ksigns [..][TQ_SIGN_WORDS(d)],
+ *   knorms [..], krnorms [..], vcodes [..][TQ_CODE_WORDS(bv, d)], vnorms [..]
+ *   scale       logit scale; Reading: the pages give none, callers pass 1/sqrt(d)
+ *   out         dev out, [B][Hq][d] float32
+ *   workspace   dev scratch of at least tq_attn_decode_workspace(...) bytes
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
+ */
+TQ_API int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                   int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                   const float* knorms, const float* krnorms, const uint32_t* vcodes,
+                   const float* vnorms, float scale, float* out, void* workspace, size_t ws_bytes,
+                   void* stream);
+TQ_API size_t tq_attn_decode_workspace(tq_handle hk, int B, int Hq, int Hkv, int64_t T);
+
+/* ---------------------------------------------------------------- diagnostics */
+
+/* tq_last_error -- message of the last failing call on this thread ("" if none). */
+TQ_API const char* tq_last_error(void);
+
+/* tq_version -- library version string. */
+TQ_API const char* tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

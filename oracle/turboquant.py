@@ -229,10 +229,41 @@ def unpack_codes(words: np.ndarray, b: int, d: int) -> np.ndarray:
     return out[:, :d]
 
 
+def pack_codes_vec(idx: np.ndarray, b: int) -> np.ndarray:
+    """Same layout as ``pack_codes`` (b <= 4), vectorised over rows with numpy
+    shifts for large inputs.  Pinned to ``pack_codes`` by equality tests."""
+    idx = np.atleast_2d(np.asarray(idx)).astype(np.uint32)
+    N, d = idx.shape
+    G = (d + 31) // 32
+    full = np.zeros((N, G * 32), dtype=np.uint32)
+    full[:, :d] = idx
+    grp = full.reshape(N, G, 32)
+    out = np.zeros((N, G, b), dtype=np.uint32)
+    if b == 1:
+        for i in range(32):
+            out[:, :, 0] |= grp[:, :, i] << np.uint32(i)
+    elif b == 2:
+        for k in range(2):
+            for j in range(16):
+                out[:, :, k] |= grp[:, :, 16 * k + j] << np.uint32(2 * j)
+    elif b == 4:
+        for k in range(4):
+            for j in range(8):
+                out[:, :, k] |= grp[:, :, 8 * k + j] << np.uint32(4 * j)
+    elif b == 3:
+        for k in range(3):
+            for j in range(8):
+                out[:, :, k] |= grp[:, :, 8 * k + j] << np.uint32(4 * j)
+                out[:, :, k] |= ((grp[:, :, 24 + j] >> np.uint32(k)) & np.uint32(1)) << np.uint32(4 * j + 3)
+    else:
+        raise ValueError("pack_codes_vec handles b <= 4")
+    return out.reshape(N, G * b)
+
+
 def pack_signs(bits: np.ndarray) -> np.ndarray:
     """QJL sign bits [N, m] (True = non-negative) -> uint32 [N, ceil(m/32)], bit i of
     word g = coordinate 32g + i (the b = 1 layout)."""
-    return pack_codes(np.asarray(bits, dtype=np.int64), 1)
+    return pack_codes_vec(np.asarray(bits, dtype=np.int64), 1)
 
 
 def unpack_signs(words: np.ndarray, m: int) -> np.ndarray:

@@ -1,0 +1,258 @@
+"""GPU parity of every hot-path call against the float64 oracle.
+
+Codes: bit-exact except coordinates whose oracle rotated value lies within
+1e-5/sqrt(d) of a decision threshold (at most 1e-4 of all coordinates).
+QJL signs: bit-exact on vectors whose mse codes match, except |(S r)_j| <=
+1e-5 ||r||.  Reconstructions: relative L2 <= 1e-5.  Scores: |delta| <=
+1e-4 ||q|| ||k|| against the oracle estimator on the same (oracle) codes.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import turboquant as oq
+
+from cases import (DEV, Instance, bf16_exact, compare_codes, compare_signs, rel_err, rel_l2_rows,
+                   to_device, upload_words, words_u32)
+
+import compressed_kv_cache_turboquant_b200 as tq
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+NORM_RTOL = 1e-5
+
+
+def _check_quant(inst: Instance, x64: np.ndarray, out: dict, rows=None):
+    rows = np.arange(x64.shape[0]) if rows is None else rows
+    ref = inst.oracle_quant(x64[rows])
+    codes = words_u32(out["codes"])[rows]
+    exact, _ = compare_codes(codes, ref["idx"], ref["y"], inst.t_o, inst.d, inst.bm)
+    norms = out["norms"].cpu().numpy()[rows]
+    assert np.max(rel_err(norms, ref["norms"])) <= NORM_RTOL
+    if inst.prod:
+        compare_signs(words_u32(out["signs"])[rows], ref["signs"], ref["Sr"], ref["rnorms"], exact)
+        rn = out["rnorms"].cpu().numpy()[rows]
+        assert np.max(rel_err(rn[exact], ref["rnorms"][exact])) <= NORM_RTOL
+    return ref, exact
+
+
+# ------------------------------------------------------------------ quantize
+
+@pytest.mark.parametrize("variant,b", [(tq.TQ_MSE, 2), (tq.TQ_PROD, 3), (tq.TQ_MSE, 1), (tq.TQ_MSE, 4)])
+def test_pr1_fp32_quantize(variant, b):
+    """N = 4096 fp32, d = 128, N(0,1) x lognormal(0, 0.5) channel scales, seed 0."""
+    inst = Instance(128, b, variant)
+    x64 = synth.scaled_gaussian_rows(4096, 128, 0.5, seed=0)
+    out = inst.alloc_outputs(4096)
+    inst.gpu_quant(to_device(x64, torch.float32), out)
+    torch.cuda.synchronize()
+    _check_quant(inst, x64, out)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_sweep_bf16_full_size_sampled(b):
+    """N = 2^20 bf16, d = 128, lognormal(0, 1) scales, 4 channels x20 outliers;
+    the whole batch on the GPU, the oracle on sampled rows and the tail."""
+    N, d = 1 << 20, 128
+    inst = Instance(d, b, tq.TQ_MSE)
+    x64 = bf16_exact(synth.scaled_gaussian_rows(N, d, 1.0, seed=0, outliers=4))
+    out = inst.alloc_outputs(N)
+    inst.gpu_quant(to_device(x64, torch.bfloat16), out)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([synth.rng(9, b).choice(N, 3000, replace=False), np.arange(N - 40, N)]))
+    _check_quant(inst, x64, out, rows)
+    # dequantized batch on the GPU: mean relative MSE close to the closed-form D(b, d)
+    xh = torch.empty((N, d), dtype=torch.float32, device=DEV)
+    tq.tq_dequant_mse(inst.h, out["codes"], out["norms"], xh)
+    xt = to_device(x64, torch.float32)
+    rel = ((xt - xh).square().sum(1) / xt.square().sum(1)).mean().item()
+    from oracle import codebook as ocb
+    D = ocb.distortion(inst.c_o, d)
+    assert abs(rel / D - 1) < 0.05, (rel, D)
+
+
+@pytest.mark.parametrize("d", [64, 128, 200])
+@pytest.mark.parametrize("N", [1, 33, 1000])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_shapes(d, N, dtype):
+    for variant, b in [(tq.TQ_MSE, 3), (tq.TQ_PROD, 4), (tq.TQ_PROD, 2)]:
+        inst = Instance(d, b, variant, seed=d + N)
+        x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=N)
+        if dtype == torch.bfloat16:
+            x64 = bf16_exact(x64)
+        out = inst.alloc_outputs(N)
+        inst.gpu_quant(to_device(x64, dtype), out)
+        torch.cuda.synchronize()
+        _check_quant(inst, x64, out)
+
+
+def test_zero_vectors_strides_and_slots():
+    d, N, stride, slots = 128, 50, 136, 3
+    inst = Instance(d, 4, tq.TQ_PROD, seed=5)
+    x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=5)
+    x64[[0, 17, 49]] = 0.0
+    xp = np.zeros((N, stride))
+    xp[:, :d] = x64
+    out = inst.alloc_outputs(N, slots=N * slots)
+    inst.gpu_quant(to_device(xp, torch.float32), out, out_stride=slots)
+    torch.cuda.synchronize()
+    sub = {k: v[::slots] for k, v in out.items()}
+    ref, _ = _check_quant(inst, x64, sub)
+    assert np.all(sub["norms"].cpu().numpy()[[0, 17, 49]] == 0)
+    assert np.all(sub["rnorms"].cpu().numpy()[[0, 17, 49]] == 0)
+    # untouched slots stay zero
+    other = out["codes"].view(N, slots, -1)[:, 1:]
+    assert int(other.abs().sum()) == 0
+
+
+def test_fp32_d1536_prod_sampled():
+    d, N = 1536, 300
+    inst = Instance(d, 4, tq.TQ_PROD, seed=3)
+    x64 = synth.unit_rows(N, d, 3)
+    out = inst.alloc_outputs(N)
+    inst.gpu_quant(to_device(x64, torch.float32), out)
+    torch.cuda.synchronize()
+    _check_quant(inst, x64, out)
+
+
+# ------------------------------------------------------------------ dequant
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", [64, 128, 200])
+def test_dequant_matches_oracle(b, d):
+    N = 777
+    inst = Instance(d, b, tq.TQ_MSE, seed=b)
+    x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=b)
+    idx, n, _ = oq.quant_mse(x64, inst.Pi_o, inst.t_o)
+    ref = oq.dequant_mse(idx, n, inst.Pi_o, inst.c_o)
+    codes = upload_words(oq.pack_codes_vec(idx, b))
+    norms = torch.tensor(n, device=DEV)
+    out = torch.empty((N, d), dtype=torch.float32, device=DEV)
+    tq.tq_dequant_mse(inst.h, codes, norms, out)
+    outb = torch.empty((N, d), dtype=torch.bfloat16, device=DEV)
+    tq.tq_dequant_mse(inst.h, codes, norms, outb)
+    torch.cuda.synchronize()
+    assert np.max(rel_l2_rows(out.cpu().numpy(), ref)) <= 1e-5
+    assert np.max(rel_l2_rows(outb.float().cpu().numpy(), ref)) <= 2 ** -8
+
+
+# ------------------------------------------------------------------ scores
+
+def _score_case(inst, N, nq, seed, topk=0):
+    d = inst.d
+    x64 = synth.scaled_gaussian_rows(N, d, 0.5, seed=seed)
+    q64 = synth.gaussian_queries(nq, d, seed=seed)
+    st = inst.oracle_quant(x64)
+    if inst.prod:
+        ref = oq.prod_estimate(q64, st["idx"], st["norms"], st["signs"], st["rnorms"], inst.Pi_o, inst.S,
+                               inst.c_o, inst.b)
+    else:
+        ref = oq.mse_estimate(q64, st["idx"], st["norms"], inst.Pi_o, inst.c_o)
+    codes = upload_words(oq.pack_codes_vec(st["idx"], inst.bm))
+    norms = torch.tensor(st["norms"], device=DEV)
+    signs = upload_words(oq.pack_signs(st["signs"])) if inst.prod else None
+    rnorms = torch.tensor(st["rnorms"], device=DEV) if inst.prod else None
+    q = to_device(q64, torch.float32)
+    scores = torch.empty((nq, N), dtype=torch.float32, device=DEV)
+    kw = {}
+    if topk:
+        kw = dict(topk=topk, top_idx=torch.empty((nq, topk), dtype=torch.int32, device=DEV),
+                  top_val=torch.empty((nq, topk), dtype=torch.float32, device=DEV))
+    tq.tq_ip_scores(inst.h, q, codes, signs, norms, rnorms, scores=scores, **kw)
+    torch.cuda.synchronize()
+    tol = 1e-4 * np.linalg.norm(q64, axis=1)[:, None] * np.linalg.norm(x64, axis=1)[None, :]
+    err = np.abs(scores.cpu().numpy() - ref)
+    assert np.all(err <= tol), float(np.max(err / tol))
+    return ref, tol, kw
+
+
+@pytest.mark.parametrize("variant,b", [(tq.TQ_MSE, 2), (tq.TQ_PROD, 3)])
+def test_pr1_scores(variant, b):
+    """64 seeded Gaussian queries against all 4096 PR1 vectors."""
+    _score_case(Instance(128, b, variant), 4096, 64, 0)
+
+
+@pytest.mark.parametrize("d,b", [(64, 4), (200, 2), (200, 4), (128, 4)])
+def test_scores_shapes_and_topk(d, b):
+    ref, tol, kw = _score_case(Instance(d, b, tq.TQ_PROD, seed=d), 2500, 9, d, topk=10)
+    ti = kw["top_idx"].cpu().numpy()
+    tv = kw["top_val"].cpu().numpy()
+    oi, ov = oq.topk(ref, 10)
+    for r in range(ref.shape[0]):
+        # returned values are the oracle's scores of the returned keys (within tolerance),
+        # sorted, and no excluded key beats the k-th by more than the tolerance
+        assert np.all(np.abs(tv[r] - ref[r, ti[r]]) <= tol[r, ti[r]])
+        assert np.all(np.diff(tv[r]) <= 0)
+        assert len(set(ti[r].tolist())) == 10
+        rest = np.setdiff1d(np.arange(ref.shape[1]), ti[r])
+        assert np.max(ref[r, rest]) <= tv[r, -1] + 2 * np.max(tol[r])
+        assert np.allclose(np.sort(tv[r]), np.sort(ov[r]), atol=2 * np.max(tol[r]))
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
+    """Quantize K (prod 4b) and V (mse 4b) with the oracle for the sampled
+    (batch, kv-head) slices, random valid codes elsewhere; decode on the GPU
+    and compare the sampled outputs with the oracle's attention."""
+    hk = Instance(d, 4, tq.TQ_PROD, seed=seed)
+    hv = Instance(d, 4, tq.TQ_MSE, seed=seed, rot_stream=synth.ROT_V)
+    S = T + stride_extra
+    rows = B * Hkv * S
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    kcodes = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, hk.h.words), dtype=torch.int32, device=DEV, generator=g)
+    ksigns = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, tq.sign_words(d)), dtype=torch.int32, device=DEV, generator=g)
+    vcodes = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, hv.h.words), dtype=torch.int32, device=DEV, generator=g)
+    knorms = torch.rand(rows, device=DEV, generator=g) * 10 + 1
+    krnorms = knorms * 0.2
+    vnorms = torch.rand(rows, device=DEV, generator=g) * 10 + 1
+    q64 = bf16_exact(synth.decode_queries(B, Hq, d, seed=seed))
+    refs = {}
+    for (b, h) in sample:
+        k64 = synth.kv_head_rows(T, d, 0, b, h, seed=seed)
+        v64 = synth.kv_head_rows(T, d, 1, b, h, seed=seed)
+        kst = hk.oracle_quant(k64)
+        vidx, vn, _ = oq.quant_mse(v64, hv.Pi_o, hv.t_o)
+        r0 = (b * Hkv + h) * S
+        kcodes[r0:r0 + T] = upload_words(oq.pack_codes_vec(kst["idx"], 3))
+        ksigns[r0:r0 + T] = upload_words(oq.pack_signs(kst["signs"]))
+        knorms[r0:r0 + T] = torch.tensor(kst["norms"], device=DEV)
+        krnorms[r0:r0 + T] = torch.tensor(kst["rnorms"], device=DEV)
+        vcodes[r0:r0 + T] = upload_words(oq.pack_codes_vec(vidx, 4))
+        vnorms[r0:r0 + T] = torch.tensor(vn, device=DEV)
+        refs[(b, h)] = (kst, oq.dequant_mse(vidx, vn, hv.Pi_o, hv.c_o))
+    q = to_device(q64, torch.bfloat16)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=DEV)
+    scale = 1.0 / math.sqrt(d)
+    tq.tq_attn_decode(hk.h, hv.h, q, Hkv, T, S, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    gsz = Hq // Hkv
+    for (b, h), (kst, vhat) in refs.items():
+        qs = q64[b, h * gsz:(h + 1) * gsz]
+        est = oq.prod_estimate(qs, kst["idx"], kst["norms"], kst["signs"], kst["rnorms"], hk.Pi_o, hk.S,
+                               hk.c_o, 4)
+        logits = est * scale
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        ref = p @ vhat
+        # logit tolerance of the score bound, propagated through the softmax
+        eps = scale * 1e-4 * np.linalg.norm(qs, axis=1)[:, None] * (np.asarray(kst["norms"], dtype=np.float64)[None, :])
+        spread = np.linalg.norm(vhat[None, :, :] - ref[:, None, :], axis=2)
+        tol = 2 * np.sum(p * eps * spread, axis=1) + 1e-3 * np.linalg.norm(ref, axis=1)
+        err = np.linalg.norm(got[b, h * gsz:(h + 1) * gsz] - ref, axis=1)
+        assert np.all(err <= tol), (b, h, err, tol)
+
+
+def test_decode_small_ragged():
+    _decode_case(B=2, Hq=8, Hkv=2, T=1531, d=128, sample=[(0, 0), (0, 1), (1, 0), (1, 1)], seed=1,
+                 stride_extra=5)
+
+
+def test_decode_cfg4_full_size_sampled():
+    """B = 8, Hq = 32, Hkv = 8, d = 128, T = 131072: full launch, sampled slices."""
+    _decode_case(B=8, Hq=32, Hkv=8, T=131072, d=128, sample=[(0, 0), (7, 7), (3, 5)], seed=0)

@@ -322,6 +322,13 @@ def test_packing_roundtrip_and_padding(b, d):
     assert np.all(full[:, d:] == 0)
 
 
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("d", [32, 64, 100, 200])
+def test_vectorised_packer_equals_field_by_field_packer(b, d):
+    idx = synth.rng(10 + b, d).integers(0, 2 ** b, size=(7, d))
+    assert np.array_equal(tq.pack_codes_vec(idx, b), tq.pack_codes(idx, b))
+
+
 # --------------------------------------------------------------------- attention
 
 def test_attention_uniform_and_dominant_limits():
