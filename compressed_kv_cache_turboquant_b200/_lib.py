@@ -19,7 +19,7 @@ TQ_MAX_TOPK = 64
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m compressed_kv_cache_turboquant_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python compressed_kv_cache_turboquant_b200/build.py` "
         "(this package has no non-CUDA fallback)")
 
 lib = ctypes.CDLL(LIB_PATH)

@@ -1,6 +1,8 @@
 """Compile the CUDA library ``libtq_b200.so`` in-tree for sm_100a.
 
-    python -m compressed_kv_cache_turboquant_b200.build
+    python compressed_kv_cache_turboquant_b200/build.py [-v] [-f]
+
+(run it by path: importing the package loads the library it builds)
 
 nvcc cross-compiles without a GPU.  The shared library exports the C ABI of
 ``include/tq.h`` and links the CUDA runtime statically, so loading it needs no
