@@ -16,6 +16,7 @@ TQ_F32, TQ_BF16 = 0, 1
 TQ_MSE, TQ_PROD = 0, 1
 TQ_MAX_DIM = 4096
 TQ_MAX_TOPK = 64
+TQ_DECODE_STATIC_SCRATCH = 4 * 1024 * 1024
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -47,6 +48,8 @@ SIGNATURES = {
     "tq_attn_decode": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,
                             _p, _p, _sz, _p]),
     "tq_attn_decode_workspace": (_sz, [_p, _i, _i, _i, _i64]),
+    "tq_attn_decode_static": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,
+                                   _p, _p]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_char_p, []),
 }

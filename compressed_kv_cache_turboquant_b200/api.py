@@ -18,6 +18,7 @@ __all__ = [
     "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQError", "Handle", "code_words", "sign_words",
     "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
+    "tq_attn_decode_static",
 ]
 
 
@@ -167,3 +168,15 @@ def tq_attn_decode(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, kv
                                                _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale),
                                                _ptr(out), _ptr(workspace), workspace.numel(),
                                                _stream(stream)))
+
+
+def tq_attn_decode_static(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, kv_stride: int,
+                          kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale: float, out: torch.Tensor,
+                          stream=None) -> None:
+    """tq_attn_decode without a workspace, for callers that may not allocate
+    device memory: the scratch lives in a fixed array inside the library (see
+    include/tq.h for its limit and for the rule that overlapping calls race)."""
+    B, Hq, _ = q.shape
+    check("tq_attn_decode_static", lib.tq_attn_decode_static(
+        hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, kv_stride, _ptr(kcodes), _ptr(ksigns),
+        _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out), _stream(stream)))

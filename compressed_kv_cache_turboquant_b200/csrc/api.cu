@@ -42,7 +42,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // decode attention: context splits per (batch, q-head)
-static int decode_splits(int B, int Hq, int64_t T, int sm_count) {
+int decode_splits(int B, int Hq, int64_t T, int sm_count) {
   // enough CTAs to fill the machine a few times, each split >= 512 tokens
   int64_t want = (int64_t)sm_count * 4 / std::max(1, B * Hq);
   int64_t cap = (T + 511) / 512;

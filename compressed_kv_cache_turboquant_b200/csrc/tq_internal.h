@@ -46,6 +46,9 @@ struct tq_ctx {
 
 namespace tqi {
 
+// number of context splits tq_attn_decode uses for a (B, Hq, T) problem
+int decode_splits(int B, int Hq, int64_t T, int sm_count);
+
 // ---- launchers (kernels_*.cu); all return cudaError_t as int ----
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,

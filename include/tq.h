@@ -243,6 +243,38 @@ TQ_API int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_dtype
                    void* stream);
 TQ_API size_t tq_attn_decode_workspace(tq_handle hk, int B, int Hq, int Hkv, int64_t T);
 
+/*
+ * tq_attn_decode_static -- tq_attn_decode for callers that cannot allocate
+ * device memory.  The paper has no counterpart to this call; it exists for
+ * library users only.
+ * Some callers may not allocate device memory while they run: a plugin whose
+ * host application owns the whole device memory budget through its own pool
+ * and gives the plugin no way to draw from it, or a service that must keep its
+ * device footprint fixed once it has started.  They cannot provide the
+ * workspace tq_attn_decode needs.  This call computes the same result with its
+ * scratch in a fixed array compiled into the library instead, and allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   Arguments and layouts: as tq_attn_decode, without workspace/ws_bytes.
+ *   Limit: a shape whose tq_attn_decode_workspace(...) exceeds
+ *   TQ_DECODE_STATIC_SCRATCH bytes is rejected with TQ_EWORKSPACE.
+ *   The array (TQ_DECODE_STATIC_SCRATCH bytes) is held on every GPU that loads
+ *   the library until the process exits.  The first call on a device looks up
+ *   the array's device address (cudaGetSymbolAddress) with that device
+ *   current; make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents; nothing in it has to start at zero (every scratch value is
+ *   written before it is read within a call).  Calls that overlap on the GPU
+ *   (different streams, or concurrent host threads) race on the array and
+ *   must be serialised by the caller.
+ * Errors: as tq_attn_decode, TQ_EWORKSPACE for shapes beyond the limit.
+ */
+#define TQ_DECODE_STATIC_SCRATCH (4 * 1024 * 1024)
+TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq,
+                                 int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
+                                 const uint32_t* ksigns, const float* knorms, const float* krnorms,
+                                 const uint32_t* vcodes, const float* vnorms, float scale, float* out,
+                                 void* stream);
+
 /* ---------------------------------------------------------------- diagnostics */
 
 /* tq_last_error -- message of the last failing call on this thread ("" if none). */
