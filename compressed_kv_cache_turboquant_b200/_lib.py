@@ -50,6 +50,7 @@ SIGNATURES = {
     "tq_attn_decode_workspace": (_sz, [_p, _i, _i, _i, _i64]),
     "tq_attn_decode_static": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,
                                    _p, _p]),
+    "tq_device_status": (_i, [_p, ctypes.POINTER(_i)]),
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_char_p, []),
 }

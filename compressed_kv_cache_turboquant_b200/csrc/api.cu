@@ -41,6 +41,40 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// round to the nearest bfloat16 (ties to even, via float32); returns the bits
+// and stores the value it represents
+static uint16_t to_bf16(double v, double* represented) {
+  float f = (float)v;
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  const uint16_t b = (uint16_t)(u >> 16);
+  const uint32_t back = (uint32_t)b << 16;
+  float r;
+  std::memcpy(&r, &back, 4);
+  *represented = (double)r;
+  return b;
+}
+
+// Pi = hi + mid + lo in bf16, arranged for the tensor-core kernels (see DevConsts::pi_tc)
+static void split_rotation_bf16(const double* Pi, int d, std::vector<uint16_t>& out) {
+  const int slabs = d / 64;
+  const size_t piece = (size_t)d * d;
+  out.assign(3 * piece, 0);
+  for (int j = 0; j < d; ++j)
+    for (int i = 0; i < d; ++i) {
+      double rem = Pi[(size_t)j * d + i];
+      const int slab = i / 64, c = (i % 64) / 8, e = i % 8;
+      const size_t off = (size_t)slab * d * 64 + (size_t)j * 64 + (size_t)((c ^ (j & 7)) * 8 + e);
+      for (int p = 0; p < 3; ++p) {
+        double rep;
+        out[p * piece + off] = to_bf16(rem, &rep);
+        rem -= rep;
+      }
+    }
+  (void)slabs;
+}
+
 // decode attention: context splits per (batch, q-head)
 int decode_splits(int B, int Hq, int64_t T, int sm_count) {
   // enough CTAs to fill the machine a few times, each split >= 512 tokens
@@ -137,7 +171,11 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   const size_t oPi = take(dd * 4), oPT = take(dd * 4);
   const size_t oS = (variant == TQ_PROD) ? take(dd * 4) : 0;
   const size_t oTT = (variant == TQ_PROD) ? take(dd * 4) : 0;
-  const size_t oC = take(64 * 4), oT = take(64 * 4);
+  const size_t oC = take(64 * 4), oT = take(64 * 4), oStatus = take(256);
+  const bool tc = (d == 64 || d == 128);
+  std::vector<uint16_t> pieces;
+  if (tc) split_rotation_bf16(Pi, d, pieces);
+  const size_t oPiTc = tc ? take(pieces.size() * 2) : 0;
   h->block_bytes = off;
   e = cudaMalloc(&h->block, h->block_bytes);
   if (e != cudaSuccess) {
@@ -149,6 +187,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   h->dev.PiT = (float*)(base + oPT);
   h->dev.centroids = (float*)(base + oC);
   h->dev.thresholds = (float*)(base + oT);
+  h->dev.status = (int*)(base + oStatus);
+  if (tc) h->dev.pi_tc = (uint8_t*)(base + oPiTc);
   if (variant == TQ_PROD) {
     h->dev.S = (float*)(base + oS);
     h->dev.TT = (float*)(base + oTT);
@@ -158,6 +198,9 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess) e = cudaMemcpy(h->dev.centroids, cf.data(), K * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && K > 1)
     e = cudaMemcpy(h->dev.thresholds, tf.data(), (K - 1) * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(h->dev.status, 0, 256);
+  if (e == cudaSuccess && tc)
+    e = cudaMemcpy(h->dev.pi_tc, pieces.data(), pieces.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && variant == TQ_PROD) {
     e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
@@ -179,6 +222,13 @@ extern "C" int tq_destroy(tq_handle h) {
   if (e != cudaSuccess) return cuda_error("tq_destroy", e);
   if (e2 != cudaSuccess) return cuda_error("tq_destroy", e2);
   return clear_error();
+}
+
+extern "C" int tq_device_status(tq_handle h, int* status) {
+  if (!h || !status) return set_error(TQ_EINVAL, "tq_device_status: NULL argument");
+  int e = cudaMemcpy(status, h->dev.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->dev.status, 0, sizeof(int));
+  return e ? cuda_error("tq_device_status", e) : clear_error();
 }
 
 extern "C" int tq_handle_info(tq_handle h, int* d, int* b, int* variant, int* mse_bits) {
@@ -213,7 +263,9 @@ extern "C" int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, in
   int rc = check_quant_args("tq_quant_mse", h, TQ_MSE, x, dtype, N, x_stride, codes, norms, out_stride);
   if (rc) return rc;
   if (N == 0) return clear_error();
-  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream);
+  int e = quant_tc_supported(h, dtype)
+              ? launch_quant_mse_tc(h, x, N, x_stride, codes, norms, out_stride, stream)
+              : launch_quant_simple(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream);
   return e ? cuda_error("tq_quant_mse", e) : clear_error();
 }
 

@@ -1,0 +1,361 @@
+// TurboQuant_mse quantization on the 5th-generation tensor cores (sm_100a).
+//
+// [ttakun, "TurboQuant_mse vs TurboQuant_prod两个变体的精确分工"]: store the norm, rotate,
+// quantize every coordinate on its own against the precomputed Lloyd-Max
+// codebook, [ttakun, "为什么随机旋转是整个算法的底层杠杆"]: the rotation is a plain
+// matrix product followed by branch-free scalar work
+// (ttakun.com/news/45354, "KV缓存52GB瞬间爆内存？TurboQuant随机旋转+标量量化…").
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: 128-vector tiles of x (bf16, 128B-swizzled,
+//               K-major) into a ring of shared-memory stages; the rotation
+//               pieces are bulk-copied into shared memory once
+//   warp 1      TMEM allocation and the single-thread MMA issuer:
+//               Y[128 x d] = X[128 x d] . (Pi_hi + Pi_mid + Pi_lo)^T, three
+//               bf16 passes accumulated in fp32 in TMEM (double-buffered)
+//   warps 2..9  epilogue, one thread per vector (TMEM lane) and half of the
+//               columns per warpgroup: n = ||y|| (= ||x||, Pi orthogonal),
+//               cell of every coordinate against n * t_k, packing, stores
+//
+// Precision: x is exact in bf16; Pi = hi + mid + lo carries ~24 significant
+// bits, so every product is exact in fp32 and y has fp32-level error (far
+// inside the 1e-5/sqrt(d) band the decisions are allowed to differ in).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sm100_common.cuh"
+#include "tq_internal.h"
+
+namespace tqi {
+namespace {
+
+using namespace sm100;
+
+constexpr int kPieces = 3;
+constexpr int kTileM = 128;
+constexpr int kThreads = 320;  // 10 warps
+
+template <int D>
+struct TcShape {
+  static constexpr int kSlabs = D / 64;                      // 128-byte K slabs
+  static constexpr int kSlabBytesX = kTileM * 128;           // one slab of a 128-row x tile
+  static constexpr int kStageBytes = kSlabs * kSlabBytesX;   // one x tile
+  static constexpr int kSlabBytesPi = D * 128;               // one slab of a D-row piece
+  static constexpr int kPieceBytes = kSlabs * kSlabBytesPi;  // = D * D * 2
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kTmemCols = 2 * D;                    // two accumulators
+  static constexpr int kMiscBytes = 4096;  // barriers, TMEM slot, thresholds, norm partials
+  static constexpr int kSmemBytes = kPieces * kPieceBytes + kStages * kStageBytes + kMiscBytes +
+                                    1024 /*alignment*/;
+};
+
+struct TcArgs {
+  const uint8_t* pi_pieces;  // kPieces x [slab][row][128 B swizzled]
+  const float* thresholds;   // [2^bm - 1]
+  int64_t N;
+  int64_t out_stride;
+  uint32_t* codes;
+  float* norms;
+  int* status;
+};
+
+template <int BM>
+__device__ __forceinline__ uint32_t cell_index(float y, const float (&P)[8]) {
+  // P[m] = n * (m-th positive threshold), m = 1 .. 2^(BM-1) - 1 (symmetric codebook)
+  constexpr uint32_t H = 1u << (BM - 1);
+  const float a = fabsf(y);
+  uint32_t m = 0;
+  if constexpr (BM == 2) {
+    m = (a >= P[1]) ? 1u : 0u;
+  } else if constexpr (BM == 3) {
+    const uint32_t m1 = (a >= P[2]) ? 1u : 0u;
+    const float t = m1 ? P[3] : P[1];
+    m = 2u * m1 + ((a >= t) ? 1u : 0u);
+  } else if constexpr (BM == 4) {
+    const uint32_t m2 = (a >= P[4]) ? 1u : 0u;
+    const float t1 = m2 ? P[6] : P[2];
+    const uint32_t m1 = (a >= t1) ? 1u : 0u;
+    const float t2 = m2 ? (m1 ? P[7] : P[5]) : (m1 ? P[3] : P[1]);
+    m = 4u * m2 + 2u * m1 + ((a >= t2) ? 1u : 0u);
+  }
+  // y >= 0 -> upper half H + m; y < 0 -> H - 1 - m (ties on a threshold: upper cell,
+  // up to the exact-equality case that the parity band excuses)
+  const uint32_t base = (y >= 0.f) ? H : H - 1u;
+  return base ^ m;
+}
+
+// pack the 32 coordinates of one group (layout of include/tq.h)
+template <int BM>
+__device__ __forceinline__ void pack_group(const float* v, const float (&P)[8], uint32_t (&w)[BM]) {
+#pragma unroll
+  for (int k = 0; k < BM; ++k) w[k] = 0u;
+  if constexpr (BM == 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[0] |= cell_index<1>(v[i], P) << i;
+  } else if constexpr (BM == 2) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i >> 4] |= cell_index<2>(v[i], P) << (2 * (i & 15));
+  } else if constexpr (BM == 4) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i >> 3] |= cell_index<4>(v[i], P) << (4 * (i & 7));
+  } else {
+    uint32_t X = 0u;
+#pragma unroll
+    for (int i = 0; i < 24; ++i) w[i >> 3] |= cell_index<3>(v[i], P) << (4 * (i & 7));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) X |= cell_index<3>(v[24 + j], P) << (4 * j);
+    w[0] |= (X << 3) & 0x88888888u;
+    w[1] |= (X << 2) & 0x88888888u;
+    w[2] |= (X << 1) & 0x88888888u;
+  }
+}
+
+template <int BM>
+__device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[BM]) {
+  if constexpr (BM == 4) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (BM == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < BM; ++k) dst[k] = w[k];
+  }
+}
+
+template <int D, int BM>
+__global__ void __launch_bounds__(kThreads, 1)
+    quant_mse_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs a) {
+  using S = TcShape<D>;
+  constexpr int W = (D / 32) * BM;  // words per vector
+  constexpr int K = 1 << BM;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* pi_s = smem;
+  uint8_t* x_s = smem + kPieces * S::kPieceBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(x_s + S::kStages * S::kStageBytes);
+  uint64_t* full = bars;                       // [kStages]
+  uint64_t* empty = bars + S::kStages;         // [kStages]
+  uint64_t* acc_full = bars + 2 * S::kStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* pi_bar = acc_empty + 2;
+  uint64_t* done_bar = pi_bar + 1;
+  uint64_t* npart_bar = done_bar + 1;          // [2] norm partials of both halves written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(npart_bar + 2);
+  float* thr_s = reinterpret_cast<float*>(tmem_slot + 4);  // [16]
+  float* npart = thr_s + 16;                               // [2 parity][2 halves][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = (a.N + kTileM - 1) / kTileM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+    }
+    mbar_init(pi_bar, 1);
+    mbar_init(done_bar, 1);
+    mbar_init(&npart_bar[0], 256);
+    mbar_init(&npart_bar[1], 256);
+    fence_mbar_init();
+  }
+  if (threadIdx.x < K - 1) thr_s[threadIdx.x] = a.thresholds[threadIdx.x];
+  if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // rotation pieces, once per CTA
+      mbar_arrive_expect_tx(pi_bar, kPieces * S::kPieceBytes);
+      for (int p = 0; p < kPieces; ++p)
+        bulk_load(pi_s + p * S::kPieceBytes, a.pi_pieces + (size_t)p * S::kPieceBytes, S::kPieceBytes, pi_bar);
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        const int s = i % S::kStages;
+        const uint32_t u = (uint32_t)(i / S::kStages);
+        if (!mbar_wait(&empty[s], (u & 1u) ^ 1u)) {
+          atomicOr(a.status, kStatusTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+        for (int sl = 0; sl < S::kSlabs; ++sl)
+          tma_load_2d(&xmap, &full[s], x_s + s * S::kStageBytes + sl * S::kSlabBytesX, sl * 64,
+                      (int)(tile * kTileM));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(kTileM, D, true);
+      const uint32_t pi_addr = smem_u32(pi_s), x_addr = smem_u32(x_s);
+      bool ok = mbar_wait(pi_bar, 0);
+      int i = 0;
+      for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
+        const int s = i % S::kStages;
+        const uint32_t u = (uint32_t)(i / S::kStages);
+        const int ab = i & 1;
+        const uint32_t ua = (uint32_t)(i >> 1);
+        if (!mbar_wait(&full[s], u & 1u) || !mbar_wait(&acc_empty[ab], (ua & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * D);
+#pragma unroll
+        for (int p = 0; p < kPieces; ++p)
+#pragma unroll
+          for (int sl = 0; sl < S::kSlabs; ++sl)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint64_t ad = sw128_kmajor_desc(x_addr + s * S::kStageBytes + sl * S::kSlabBytesX + k4 * 32);
+              const uint64_t bd = sw128_kmajor_desc(pi_addr + p * S::kPieceBytes + sl * S::kSlabBytesPi + k4 * 32);
+              mma_f16(d_tmem, ad, bd, idesc, (p | sl | k4) != 0 ? 1u : 0u);
+            }
+        mma_commit(&empty[s]);
+        mma_commit(&acc_full[ab]);
+      }
+      if (!ok) atomicOr(a.status, kStatusTimeout);
+      mma_commit(done_bar);  // arrives once everything issued above has completed
+    }
+  } else {
+    // epilogue: 8 warps; warp % 4 selects the TMEM lane quarter, the warpgroup the column half
+    const int ew = warp - 2;
+    const int half = ew >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    constexpr int HC = D / 2;   // columns per half
+    constexpr int GH = HC / 32; // code groups per half
+    float P[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) P[m] = 0.f;
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int ab = i & 1;
+      const uint32_t ua = (uint32_t)(i >> 1);
+      if (!mbar_wait(&acc_full[ab], ua & 1u)) {
+        atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      float v[HC];
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * D + half * HC);
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) tmem_ld32(taddr + c * 32, *reinterpret_cast<float(*)[32]>(&v[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < HC; ++c) ss = fmaf(v[c], v[c], ss);
+      // exchange the two halves' partial sums of squares (bounded wait)
+      float* np = npart + (i & 1) * 256;
+      np[half * 128 + row] = ss;
+      mbar_arrive(&npart_bar[i & 1]);
+      if (!mbar_wait(&npart_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
+        atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+      const float n = sqrtf(np[row] + np[128 + row]);
+#pragma unroll
+      for (int m = 1; m < (1 << (BM - 1)); ++m) P[m] = n * thr_s[(1 << (BM - 1)) - 1 + m];
+      const int64_t vec = tile * kTileM + row;
+      if (vec < a.N) {
+        uint32_t* dst = a.codes + vec * a.out_stride * W + half * GH * BM;
+#pragma unroll
+        for (int g = 0; g < GH; ++g) {
+          uint32_t w[BM];
+          pack_group<BM>(&v[g * 32], P, w);
+          store_words<BM>(dst + g * BM, w);
+        }
+        if (half == 0) a.norms[vec * a.out_stride] = n;
+      }
+    }
+  }
+
+  // teardown: the MMA thread's final commit tells when TMEM is no longer in use
+  __syncthreads();
+  if (warp == 1) {
+    if (!mbar_wait(done_bar, 0) && lane == 0) atomicOr(a.status, kStatusTimeout);
+    __syncwarp();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+template <int D, int BM>
+int launch_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint32_t* codes, float* norms,
+              int64_t out_stride, cudaStream_t stream) {
+  using S = TcShape<D>;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return (int)cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)N};
+  const cuuint64_t gstride[1] = {(cuuint64_t)x_stride * 2};
+  const cuuint32_t box[2] = {64, kTileM};
+  const cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
+  static bool attr_set[5][2] = {};
+  auto kern = quant_mse_tc_kernel<D, BM>;
+  if (!attr_set[BM][D == 128]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    if (e != cudaSuccess) return (int)e;
+    attr_set[BM][D == 128] = true;
+  }
+  TcArgs a{h->dev.pi_tc, h->dev.thresholds, N, out_stride, codes, norms, h->dev.status};
+  const int64_t ntiles = (N + kTileM - 1) / kTileM;
+  const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);
+  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(map, a);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+bool quant_tc_supported(const tq_ctx* h, int dtype) {
+  return h->dev.pi_tc != nullptr && dtype == TQ_BF16 && (h->d == 64 || h->d == 128) && h->variant == TQ_MSE;
+}
+
+int launch_quant_mse_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint32_t* codes,
+                        float* norms, int64_t out_stride, void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  if (h->d == 128) {
+    switch (h->bm) {
+      case 1: return launch_tc<128, 1>(h, x, N, x_stride, codes, norms, out_stride, s);
+      case 2: return launch_tc<128, 2>(h, x, N, x_stride, codes, norms, out_stride, s);
+      case 3: return launch_tc<128, 3>(h, x, N, x_stride, codes, norms, out_stride, s);
+      default: return launch_tc<128, 4>(h, x, N, x_stride, codes, norms, out_stride, s);
+    }
+  }
+  switch (h->bm) {
+    case 1: return launch_tc<64, 1>(h, x, N, x_stride, codes, norms, out_stride, s);
+    case 2: return launch_tc<64, 2>(h, x, N, x_stride, codes, norms, out_stride, s);
+    case 3: return launch_tc<64, 3>(h, x, N, x_stride, codes, norms, out_stride, s);
+    default: return launch_tc<64, 4>(h, x, N, x_stride, codes, norms, out_stride, s);
+  }
+}
+
+}  // namespace tqi

@@ -28,6 +28,11 @@ struct DevConsts {
   uint16_t* T_bf16 = nullptr;   // [pieces][d*d]
   // decode tables
   uint32_t* lut_f16 = nullptr;  // packed fp16 centroid byte tables
+  // rotation split into 3 bf16 pieces (hi, mid, lo) laid out as the tensor-core
+  // kernels hold them in shared memory: [piece][K slab of 64][row j][128 B,
+  // 16-byte chunks XOR-swizzled by row % 8]; only for d in {64, 128}
+  uint8_t* pi_tc = nullptr;
+  int* status = nullptr;        // device status word (bounded waits that expired)
 };
 
 }  // namespace tqi
@@ -50,6 +55,9 @@ namespace tqi {
 int decode_splits(int B, int Hq, int64_t T, int sm_count);
 
 // ---- launchers (kernels_*.cu); all return cudaError_t as int ----
+bool quant_tc_supported(const tq_ctx* h, int dtype);
+int launch_quant_mse_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint32_t* codes,
+                        float* norms, int64_t out_stride, void* stream);
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
                         int64_t out_stride, void* stream);

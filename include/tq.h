@@ -277,6 +277,16 @@ TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int 
 
 /* ---------------------------------------------------------------- diagnostics */
 
+/*
+ * tq_device_status -- read and clear the handle's device status word
+ * (synchronous).  0 = no event.  Bit 0 (TQ_STATUS_TIMEOUT): a tensor-core
+ * kernel gave up a wait on one of its own pipeline barriers after ~2 s and
+ * returned early; its outputs for that call are incomplete.
+ * Errors: TQ_EINVAL, TQ_ECUDA.
+ */
+#define TQ_STATUS_TIMEOUT 1
+TQ_API int tq_device_status(tq_handle h, int* status);
+
 /* tq_last_error -- message of the last failing call on this thread ("" if none). */
 TQ_API const char* tq_last_error(void);
 
