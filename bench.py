@@ -378,7 +378,7 @@ def run_ours(args):
                    "frac_hbm": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9 / hbm} for k, v in ks.items()}
 
     e2e = None
-    if args.workload == "sweep":
+    if args.workload == "sweep" and not args.no_e2e:
         e_ms, h2d, d2h = wl.e2e(max(2, args.steps // 2), 1)
         e_ms = max_over_ranks(e_ms)
         e2e = {"value": units / (e_ms / 1e3), "unit": unit_name, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -462,6 +462,7 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=None)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

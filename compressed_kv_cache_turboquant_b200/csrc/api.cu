@@ -1,5 +1,6 @@
 // C ABI of the TurboQuant hot path: argument checks, handle management and
 // dispatch to the kernels.  The operations are defined in include/tq.h.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -73,6 +74,35 @@ static void split_rotation_bf16(const double* Pi, int d, std::vector<uint16_t>& 
       }
     }
   (void)slabs;
+}
+
+static uint16_t half_bits(double v) {
+  __half h = __double2half(v);
+  uint16_t b;
+  std::memcpy(&b, &h, 2);
+  return b;
+}
+
+static double half_value(uint16_t b) {
+  __half h;
+  std::memcpy(&h, &b, 2);
+  return (double)__half2float(h);
+}
+
+// Pi^T as fp16 pieces (hi, (Pi - hi) * 2^11) in the swizzled K-major layout:
+// B[i][j] = Pi[j][i], row i, K index j
+static void split_rotation_t_f16(const double* Pi, int d, std::vector<uint16_t>& out) {
+  const size_t piece = (size_t)d * d;
+  out.assign(2 * piece, 0);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) {
+      const double v = Pi[(size_t)j * d + i];
+      const int slab = j / 64, c = (j % 64) / 8, e = j % 8;
+      const size_t off = (size_t)slab * d * 64 + (size_t)i * 64 + (size_t)((c ^ (i & 7)) * 8 + e);
+      const uint16_t hi = half_bits(v);
+      out[off] = hi;
+      out[piece + off] = half_bits((v - half_value(hi)) * 2048.0);
+    }
 }
 
 // decode attention: context splits per (batch, q-head)
@@ -176,6 +206,18 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   std::vector<uint16_t> pieces;
   if (tc) split_rotation_bf16(Pi, d, pieces);
   const size_t oPiTc = tc ? take(pieces.size() * 2) : 0;
+  std::vector<uint16_t> tpieces;
+  std::vector<uint32_t> lut(16, 0u);
+  if (tc) {
+    split_rotation_t_f16(Pi, d, tpieces);
+    for (int k = 0; k < K; ++k) {
+      const uint16_t hi = half_bits(h->host_centroids[k]);
+      const uint16_t lo = half_bits((h->host_centroids[k] - half_value(hi)) * 2048.0);
+      lut[k] = (uint32_t)hi | ((uint32_t)lo << 16);
+    }
+  }
+  const size_t oPitF16 = tc ? take(tpieces.size() * 2) : 0;
+  const size_t oLut = take(16 * 4);
   h->block_bytes = off;
   e = cudaMalloc(&h->block, h->block_bytes);
   if (e != cudaSuccess) {
@@ -189,6 +231,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   h->dev.thresholds = (float*)(base + oT);
   h->dev.status = (int*)(base + oStatus);
   if (tc) h->dev.pi_tc = (uint8_t*)(base + oPiTc);
+  if (tc) h->dev.pit_f16 = (uint8_t*)(base + oPitF16);
+  h->dev.lut_dq = (uint32_t*)(base + oLut);
   if (variant == TQ_PROD) {
     h->dev.S = (float*)(base + oS);
     h->dev.TT = (float*)(base + oTT);
@@ -201,6 +245,9 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess) e = cudaMemset(h->dev.status, 0, 256);
   if (e == cudaSuccess && tc)
     e = cudaMemcpy(h->dev.pi_tc, pieces.data(), pieces.size() * 2, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && tc)
+    e = cudaMemcpy(h->dev.pit_f16, tpieces.data(), tpieces.size() * 2, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->dev.lut_dq, lut.data(), 16 * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && variant == TQ_PROD) {
     e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
@@ -293,7 +340,8 @@ extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* n
   TQ_CHECK_ALIGN(norms, "norms");
   TQ_CHECK_ALIGN(out, "out");
   if (N == 0) return clear_error();
-  int e = launch_dequant_simple(h, codes, norms, N, out, out_dtype, stream);
+  int e = dequant_tc_supported(h) ? launch_dequant_tc(h, codes, norms, N, out, out_dtype, stream)
+                                  : launch_dequant_simple(h, codes, norms, N, out, out_dtype, stream);
   return e ? cuda_error("tq_dequant_mse", e) : clear_error();
 }
 

@@ -33,6 +33,10 @@ struct DevConsts {
   // 16-byte chunks XOR-swizzled by row % 8]; only for d in {64, 128}
   uint8_t* pi_tc = nullptr;
   int* status = nullptr;        // device status word (bounded waits that expired)
+  // Pi^T in two fp16 pieces (hi, lo * 2^11), same swizzled K-major layout, and
+  // the centroid table as fp16 pieces (hi | lo * 2^11 << 16), for dequant
+  uint8_t* pit_f16 = nullptr;
+  uint32_t* lut_dq = nullptr;
 };
 
 }  // namespace tqi
@@ -56,6 +60,9 @@ int decode_splits(int B, int Hq, int64_t T, int sm_count);
 
 // ---- launchers (kernels_*.cu); all return cudaError_t as int ----
 bool quant_tc_supported(const tq_ctx* h, int dtype);
+bool dequant_tc_supported(const tq_ctx* h);
+int launch_dequant_tc(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_t N, void* out,
+                      int out_dtype, void* stream);
 int launch_quant_mse_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint32_t* codes,
                         float* norms, int64_t out_stride, void* stream);
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
