@@ -218,6 +218,27 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   }
   const size_t oPitF16 = tc ? take(tpieces.size() * 2) : 0;
   const size_t oLut = take(16 * 4);
+  // fp16 byte tables for register decoding: 8 entries as lo-byte and hi-byte words
+  auto byte_table = [&](const double* c8, uint32_t* t4) {
+    for (int w = 0; w < 2; ++w) {
+      uint32_t lo = 0, hi = 0;
+      for (int k = 0; k < 4; ++k) {
+        const uint16_t hb = half_bits(c8[4 * w + k]);
+        lo |= (uint32_t)(hb & 0xFFu) << (8 * k);
+        hi |= (uint32_t)(hb >> 8) << (8 * k);
+      }
+      t4[w] = lo;
+      t4[2 + w] = hi;
+    }
+  };
+  uint32_t ktab[4] = {0, 0, 0, 0}, vtab[4] = {0, 0, 0, 0};
+  const bool has_ktab = (bm == 3);
+  bool has_vtab = (bm == 4);
+  for (int k = 0; has_vtab && k < 16; ++k)
+    if (h->host_centroids[15 - k] != -h->host_centroids[k]) has_vtab = false;  // needs c[15-i] = -c[i]
+  if (has_ktab) byte_table(h->host_centroids, ktab);
+  if (has_vtab) byte_table(h->host_centroids + 8, vtab);
+  const size_t oTabs = take(8 * 4);
   h->block_bytes = off;
   e = cudaMalloc(&h->block, h->block_bytes);
   if (e != cudaSuccess) {
@@ -233,6 +254,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (tc) h->dev.pi_tc = (uint8_t*)(base + oPiTc);
   if (tc) h->dev.pit_f16 = (uint8_t*)(base + oPitF16);
   h->dev.lut_dq = (uint32_t*)(base + oLut);
+  if (has_ktab) h->dev.ktab = (uint32_t*)(base + oTabs);
+  if (has_vtab) h->dev.vtab = (uint32_t*)(base + oTabs + 16);
   if (variant == TQ_PROD) {
     h->dev.S = (float*)(base + oS);
     h->dev.TT = (float*)(base + oTT);
@@ -248,6 +271,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess && tc)
     e = cudaMemcpy(h->dev.pit_f16, tpieces.data(), tpieces.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(h->dev.lut_dq, lut.data(), 16 * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(base + oTabs, ktab, 16, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(base + oTabs + 16, vtab, 16, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && variant == TQ_PROD) {
     e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
@@ -388,11 +413,47 @@ extern "C" int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint3
   return e ? cuda_error("tq_ip_scores", e) : clear_error();
 }
 
+namespace tqi {
+
+size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t T) {
+  const size_t nq = (size_t)B * Hq;
+  const int sp = std::max(decode_splits(B, Hq, T, hk->sm_count), decode_mma_splits(B, Hkv, T, hk->sm_count));
+  return 2 * align_up(nq * hk->d * 4, 256) + align_up(nq * 2 * hk->d * 2, 256) + align_up(nq * 2 * 4, 256) +
+         align_up(nq * sp * (hk->d + 2) * 4, 256);
+}
+
+// workspace: rotated queries | projected queries (fp32) | fp16 query operands | their scales | partials
+int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                    int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                    const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                    float scale, float* out, void* workspace, void* stream) {
+  const size_t nq = (size_t)B * Hq;
+  char* ws = (char*)workspace;
+  const size_t q32 = align_up(nq * hk->d * 4, 256);
+  float* qrot = (float*)ws;
+  float* qproj = (float*)(ws + q32);
+  void* qfrag = ws + 2 * q32;
+  float* qscale = (float*)(ws + 2 * q32 + align_up(nq * 2 * hk->d * 2, 256));
+  float* partials = (float*)((char*)qscale + align_up(nq * 2 * 4, 256));
+  int e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)nq, qrot, qproj, stream);
+  if (e) return e;
+  if (decode_mma_supported(hk, hv, Hq, Hkv, kv_stride)) {
+    e = launch_qfrag(qrot, qproj, (int64_t)nq, qfrag, qscale, stream);
+    if (e) return e;
+    const int splits = decode_mma_splits(B, Hkv, T, hk->sm_count);
+    return launch_decode_mma(hk, hv, (const uint32_t*)qfrag, qscale, B, Hq, Hkv, T, kv_stride, kcodes, ksigns,
+                             knorms, krnorms, vcodes, vnorms, scale, splits, partials, out, stream);
+  }
+  const int splits = decode_splits(B, Hq, T, hk->sm_count);
+  return launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms,
+                              vcodes, vnorms, scale, splits, partials, out, stream);
+}
+
+}  // namespace tqi
+
 extern "C" size_t tq_attn_decode_workspace(tq_handle hk, int B, int Hq, int Hkv, int64_t T) {
   if (!hk || B < 0 || Hq < 0 || Hkv <= 0 || T < 0) return 0;
-  const int splits = decode_splits(B, Hq, T, hk->sm_count);
-  const size_t q = align_up((size_t)B * Hq * hk->d * 4, 256);
-  return 2 * q + align_up((size_t)B * Hq * splits * (hk->d + 2) * 4, 256);
+  return decode_workspace_bytes(hk, B, Hq, Hkv, T);
 }
 
 extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq,
@@ -420,15 +481,7 @@ extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_d
   const size_t need = tq_attn_decode_workspace(hk, B, Hq, Hkv, T);
   if (!workspace || ws_bytes < need)
     return set_error(TQ_EWORKSPACE, "tq_attn_decode: workspace %zu < %zu bytes", ws_bytes, need);
-  const int splits = decode_splits(B, Hq, T, hk->sm_count);
-  char* ws = (char*)workspace;
-  const size_t qb = align_up((size_t)B * Hq * hk->d * 4, 256);
-  float* qrot = (float*)ws;
-  float* qproj = (float*)(ws + qb);
-  float* partials = (float*)(ws + 2 * qb);
-  int e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)B * Hq, qrot, qproj, stream);
-  if (!e)
-    e = launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms,
-                             krnorms, vcodes, vnorms, scale, splits, partials, out, stream);
+  int e = decode_dispatch(hk, hv, q, q_dtype, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, vcodes,
+                          vnorms, scale, out, workspace, stream);
   return e ? cuda_error("tq_attn_decode", e) : clear_error();
 }

@@ -47,8 +47,6 @@ int scratch_address(void** out) {
   return (int)cudaSuccess;
 }
 
-size_t align256(size_t v) { return (v + 255) / 256 * 256; }
-
 }  // namespace
 }  // namespace tqi
 
@@ -89,19 +87,11 @@ extern "C" int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, 
   if (e != cudaSuccess)
     return set_error(TQ_ECUDA, "tq_attn_decode_static: scratch set-up: %s",
                      cudaGetErrorString((cudaError_t)e));
-  // same partition of the scratch as tq_attn_decode uses for its workspace;
-  // every byte read below is written earlier in the same call, so nothing has
-  // to be cleared between calls
-  const int splits = decode_splits(B, Hq, T, hk->sm_count);
-  const size_t qb = align256((size_t)B * Hq * hk->d * 4);
-  char* base = (char*)ws;
-  float* qrot = (float*)base;
-  float* qproj = (float*)(base + qb);
-  float* partials = (float*)(base + 2 * qb);
-  e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)B * Hq, qrot, qproj, stream);
-  if (!e)
-    e = launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms,
-                             krnorms, vcodes, vnorms, scale, splits, partials, out, stream);
+  // same kernels and the same partition of the scratch as tq_attn_decode uses
+  // for its workspace; every byte read is written earlier in the same call, so
+  // nothing has to be cleared between calls
+  e = decode_dispatch(hk, hv, q, q_dtype, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, vcodes,
+                      vnorms, scale, out, ws, stream);
   if (e)
     return set_error(TQ_ECUDA, "tq_attn_decode_static: %s", cudaGetErrorString((cudaError_t)e));
   return clear_error();

@@ -457,8 +457,13 @@ int launch_decode_simple(const tq_ctx* hk, const tq_ctx* hv, const float* qrot,
   decode_split_simple_kernel<<<dim3(splits, Hq, B), 128, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  decode_merge_kernel<<<B * Hq, 128, hk->d * sizeof(float), s>>>(partials, splits, hk->d,
-                                                                hv->dev.Pi, out);
+  return launch_decode_merge(partials, (int64_t)B * Hq, splits, hv, out, stream);
+}
+
+int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out,
+                        void* stream) {
+  decode_merge_kernel<<<(unsigned)BH, 128, hv->d * sizeof(float), (cudaStream_t)stream>>>(partials, splits, hv->d,
+                                                                                      hv->dev.Pi, out);
   return (int)cudaGetLastError();
 }
 

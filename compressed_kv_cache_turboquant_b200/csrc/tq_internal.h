@@ -37,6 +37,11 @@ struct DevConsts {
   // the centroid table as fp16 pieces (hi | lo * 2^11 << 16), for dequant
   uint8_t* pit_f16 = nullptr;
   uint32_t* lut_dq = nullptr;
+  // fp16 byte tables for register decoding (byte-permute lookups):
+  // ktab (3-bit codebooks): lo bytes of c0..3, c4..7, hi bytes of c0..3, c4..7
+  // vtab (4-bit symmetric codebooks): the same for the upper half c8..c15
+  uint32_t* ktab = nullptr;
+  uint32_t* vtab = nullptr;
 };
 
 }  // namespace tqi
@@ -77,6 +82,21 @@ int launch_scores_simple(const tq_ctx* h, const float* qrot, const float* qproj,
                          const float* rnorms, int64_t N, float* scores, void* stream);
 int launch_topk_simple(const float* scores, int64_t nq, int64_t N, int k, int32_t* top_idx,
                        float* top_val, void* stream);
+int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out,
+                        void* stream);
+bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride);
+int decode_mma_splits(int B, int Hkv, int64_t T, int sm_count);
+int launch_qfrag(const float* qrot, const float* qproj, int64_t nq, void* qfrag, float* qscale, void* stream);
+int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
+                      int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
+                      const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
+                      const float* vnorms, float scale, int splits, float* partials, float* out, void* stream);
+// decode attention through whichever kernel fits; workspace layout owned here
+size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t T);
+int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                    int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                    const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                    float scale, float* out, void* workspace, void* stream);
 int launch_decode_simple(const tq_ctx* hk, const tq_ctx* hv, const float* qrot,
                          const float* qproj, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
                          const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
