@@ -417,9 +417,11 @@ namespace tqi {
 
 size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t T) {
   const size_t nq = (size_t)B * Hq;
-  const int sp = std::max(decode_splits(B, Hq, T, hk->sm_count), decode_mma_splits(B, Hkv, T, hk->sm_count));
+  const size_t simple = nq * decode_splits(B, Hq, T, hk->sm_count) * (hk->d + 2) * 4;
+  const size_t fast = (size_t)decode_mma_grid(B, Hkv, T, hk->sm_count) * decode_mma_max_seg(B, Hkv, T, hk->sm_count) *
+                      4 * (hk->d + 2) * 4;
   return 2 * align_up(nq * hk->d * 4, 256) + align_up(nq * 2 * hk->d * 2, 256) + align_up(nq * 2 * 4, 256) +
-         align_up(nq * sp * (hk->d + 2) * 4, 256);
+         align_up(std::max(simple, fast), 256);
 }
 
 // workspace: rotated queries | projected queries (fp32) | fp16 query operands | their scales | partials
@@ -440,9 +442,8 @@ int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dty
   if (decode_mma_supported(hk, hv, Hq, Hkv, kv_stride)) {
     e = launch_qfrag(qrot, qproj, (int64_t)nq, qfrag, qscale, stream);
     if (e) return e;
-    const int splits = decode_mma_splits(B, Hkv, T, hk->sm_count);
     return launch_decode_mma(hk, hv, (const uint32_t*)qfrag, qscale, B, Hq, Hkv, T, kv_stride, kcodes, ksigns,
-                             knorms, krnorms, vcodes, vnorms, scale, splits, partials, out, stream);
+                             knorms, krnorms, vcodes, vnorms, scale, partials, out, stream);
   }
   const int splits = decode_splits(B, Hq, T, hk->sm_count);
   return launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms,

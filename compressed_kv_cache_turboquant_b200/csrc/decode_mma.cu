@@ -65,13 +65,22 @@ struct DecArgs {
   const float* qscale;     // [B*Hq][2]: 1/s for the two fp16 query copies
   const uint32_t* ktab;    // [4]: K centroid lo bytes c0..3, c4..7, hi bytes c0..3, c4..7
   const uint32_t* vtab;    // [4]: V magnitude table |c|[8..15], lo and hi bytes
-  int B, Hq, Hkv, splits;
-  int64_t T, kv_stride, per_split;
+  int B, Hq, Hkv;
+  int64_t T, kv_stride;
+  int64_t nblk;            // 64-token blocks per (batch, kv-head)
+  int64_t total;           // B * Hkv * nblk
+  int max_seg;             // partial slots per CTA
   float scale_log2;        // logit scale * log2(e)
   float qjl_coef;          // sqrt(pi/2) / d
-  float* partials;         // [B][Hq][splits][d + 2]
+  float* partials;         // [CTA][max_seg][4 heads][d + 2]: acc[d], m (natural log), l
   int* status;
 };
+
+// CTA i of G owns the global blocks [i*total/G, (i+1)*total/G); a global block
+// gb is block gb % nblk of (batch, kv-head) gb / nblk
+__host__ __device__ __forceinline__ int64_t cta_first_block(int64_t i, int64_t total, int64_t G) {
+  return i * total / G;
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) { return __byte_perm(a, b, s); }
 
@@ -127,41 +136,40 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
   uint8_t* stages = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
-  __half* pbuf = reinterpret_cast<__half*>(empty + kStages);             // [kCons][4 heads][16 tokens]
-  float* mrg = reinterpret_cast<float*>(pbuf + kCons * 64);               // [kCons][4][2 + D]
+  uint64_t* pub = empty + kStages;                                        // consumers published their state
+  __half* pbuf = reinterpret_cast<__half*>(pub + 2);                     // [kCons][4 heads][16 tokens]
+  float* mrg = reinterpret_cast<float*>(pbuf + kCons * 64);               // [2][kCons][4][2 + D]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int bh = blockIdx.y;  // b * Hkv + h
-  const int b = bh / a.Hkv, h = bh % a.Hkv;
-  const int64_t t_begin = (int64_t)split * a.per_split;
-  const int64_t t_end = min(a.T, t_begin + a.per_split);
-  const int64_t row0 = (int64_t)bh * a.kv_stride;
-  const int64_t nblk = (t_end > t_begin) ? (t_end - t_begin + kBlk - 1) / kBlk : 0;
+  const int64_t G = gridDim.x;
+  const int64_t gb_lo = cta_first_block(blockIdx.x, a.total, G);
+  const int64_t gb_hi = cta_first_block(blockIdx.x + 1, a.total, G);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCons);
     }
+    mbar_init(pub, 32 * kCons);
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t i = 0; i < nblk; ++i) {
+      for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i) {
         const int s = (int)(i % kStages);
         const uint32_t u = (uint32_t)(i / kStages);
         if (!mbar_wait(&empty[s], (u & 1u) ^ 1u)) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }
-        const int64_t t0 = t_begin + i * kBlk;
-        const int n = (int)min((int64_t)kBlk, t_end - t0);
+        const int64_t bh = gb / a.nblk;
+        const int64_t t0 = (gb % a.nblk) * kBlk;
+        const int n = (int)min((int64_t)kBlk, a.T - t0);
         const int n4 = n & ~3;  // norms are copied in whole 16-byte units
         uint8_t* st = stages + s * kStageBytes;
-        const int64_t r = row0 + t0;
+        const int64_t r = bh * a.kv_stride + t0;
         mbar_arrive_expect_tx(&full[s], (uint32_t)(n * (kKW + kSW + kVW) * 4 + 3 * n4 * 4));
         bulk_load(st + kOffK, a.kcodes + r * kKW, n * kKW * 4, &full[s]);
         bulk_load(st + kOffS, a.ksigns + r * kSW, n * kSW * 4, &full[s]);
@@ -175,45 +183,103 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
     }
   } else {
     const int cw = warp - 1;           // consumer index
+    const int ct = threadIdx.x - 32;   // consumer thread 0..127
     const int g = lane >> 2, c = lane & 3;
     const int cp = c & 1;              // heads 2cp, 2cp+1 handled by this lane
-    // tables
+    const int group = a.Hq / a.Hkv;    // 4
     uint32_t kt[4], vt[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) kt[i] = a.ktab[i], vt[i] = a.vtab[i];
-    // B fragments of the queries: mse columns 0-3 (q' of head g), QJL columns 4-7 (q'' of head g-4)
-    const int hq0 = h * (a.Hq / a.Hkv);
     uint32_t bm[8][2], bq[8][2];
-    {
-      const int qh = g & 3;
-      const uint32_t* qf = a.qfrag + (int64_t)((int64_t)b * a.Hq + hq0 + qh) * 2 * 64;
-#pragma unroll
-      for (int kb = 0; kb < 8; ++kb) {
-        const uint2 vm = *reinterpret_cast<const uint2*>(qf + (32 * c + 4 * kb) / 2);
-        const uint2 vq = *reinterpret_cast<const uint2*>(qf + 64 + (32 * c + 4 * kb) / 2);
-        bm[kb][0] = (g < 4) ? vm.x : 0u;
-        bm[kb][1] = (g < 4) ? vm.y : 0u;
-        bq[kb][0] = (g >= 4) ? vq.x : 0u;
-        bq[kb][1] = (g >= 4) ? vq.y : 0u;
-      }
-    }
     float inv_s1[2], inv_s2[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int64_t qi = (int64_t)b * a.Hq + hq0 + 2 * cp + j;
-      inv_s1[j] = a.qscale[2 * qi];
-      inv_s2[j] = a.qscale[2 * qi + 1];
-    }
-    float m_run[2] = {-FLT_MAX, -FLT_MAX}, l_run[2] = {0.f, 0.f};
+    float m_run[2], l_run[2];
     float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
     __half* pb = pbuf + cw * 64;
-
+    int64_t cur_bh = -1;
+    int seg = -1;
     bool ok = true;
-    for (int64_t i = 0; i < nblk; ++i) {
+
+    // publish this warp's state, combine the four warps, write one partial
+    auto flush = [&](int sg, int64_t bhv) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
+      }
+      float* mb = mrg + (sg & 1) * kCons * 4 * (2 + D);
+      float* mw = mb + cw * 4 * (2 + D);
+      if (c < 2) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float* mh = mw + (2 * c + j) * (2 + D);
+          if (g == 0) mh[0] = m_run[j], mh[1] = l_run[j];
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            mh[2 + 16 * g + 2 * mt] = acc[mt][j];
+            mh[2 + 16 * g + 2 * mt + 1] = acc[mt][2 + j];
+          }
+        }
+      }
+      mbar_arrive(pub);
+      if (!mbar_wait(pub, (uint32_t)(sg & 1))) {
+        ok = false;
+        return;
+      }
+      float* dst = a.partials + ((int64_t)blockIdx.x * a.max_seg + sg) * 4 * (D + 2);
+      for (int idx = ct; idx < 4 * (2 + D); idx += 32 * kCons) {
+        const int hd = idx / (2 + D), k = idx % (2 + D);
+        float M = -FLT_MAX;
+#pragma unroll
+        for (int w = 0; w < kCons; ++w) M = fmaxf(M, mb[(w * 4 + hd) * (2 + D)]);
+        if (k == 0) {
+          dst[hd * (D + 2) + D] = M / kLog2e;  // natural-log units for the merge
+        } else {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kCons; ++w) {
+            const float* mh = mb + (w * 4 + hd) * (2 + D);
+            v += mh[k] * exp2f(mh[0] - M);
+          }
+          if (k == 1) dst[hd * (D + 2) + D + 1] = v;
+          else dst[hd * (D + 2) + k - 2] = v;
+        }
+      }
+      (void)bhv;
+    };
+
+    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i) {
+      const int64_t bh = gb / a.nblk;
+      if (bh != cur_bh) {
+        if (seg >= 0) flush(seg, cur_bh);
+        if (!ok) break;
+        ++seg;
+        cur_bh = bh;
+        // queries of this (batch, kv-head): mse columns 0-3 (q' of head g), QJL columns 4-7 (q'' of head g-4)
+        const int64_t b = bh / a.Hkv, hh = bh % a.Hkv;
+        const int64_t q0 = b * a.Hq + hh * group;
+        const uint32_t* qf = a.qfrag + (q0 + (g & 3)) * 2 * 64;
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) {
+          const uint2 vm = *reinterpret_cast<const uint2*>(qf + 16 * c + 2 * kb);
+          const uint2 vq = *reinterpret_cast<const uint2*>(qf + 64 + 16 * c + 2 * kb);
+          bm[kb][0] = (g < 4) ? vm.x : 0u;
+          bm[kb][1] = (g < 4) ? vm.y : 0u;
+          bq[kb][0] = (g >= 4) ? vq.x : 0u;
+          bq[kb][1] = (g >= 4) ? vq.y : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          inv_s1[j] = a.qscale[2 * (q0 + 2 * cp + j)];
+          inv_s2[j] = a.qscale[2 * (q0 + 2 * cp + j) + 1];
+          m_run[j] = -FLT_MAX;
+          l_run[j] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+      }
       const int s = (int)(i % kStages);
       const uint32_t u = (uint32_t)(i / kStages);
       if (!mbar_wait(&full[s], u & 1u)) {
@@ -221,9 +287,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
         break;
       }
       const uint8_t* st = stages + s * kStageBytes;
-      const int64_t t0 = t_begin + i * kBlk;
-      const int n = (int)min((int64_t)kBlk, t_end - t0);
+      const int64_t t0 = (gb % a.nblk) * kBlk;
+      const int n = (int)min((int64_t)kBlk, a.T - t0);
       const int n4 = n & ~3;
+      const int64_t row0 = bh * a.kv_stride + t0;
       const int tb = cw * 16;  // this warp's 16 tokens within the block
       // ---------------- logits: keys g and g+8 of the sub-block
       float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -268,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
           kr[r] = reinterpret_cast<const float*>(st + kOffR)[tok];
           vn[r] = reinterpret_cast<const float*>(st + kOffVN)[tok];
         } else if (tok < n) {
-          const int64_t gi = row0 + t0 + tok;
+          const int64_t gi = row0 + tok;
           kn[r] = a.knorms[gi];
           kr[r] = a.krnorms[gi];
           vn[r] = a.vnorms[gi];
@@ -345,50 +412,65 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
+    if (ok && seg >= 0) flush(seg, cur_bh);
     if (!ok) atomicOr(a.status, kStatusTimeout);
-    // warp totals of the softmax sums (over the 8 lanes with the same c)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
-      l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
-      l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
-    }
-    // publish this warp's state: mrg[cw][head][0] = m, [1] = l, [2 + coord] = acc
-    float* mw = mrg + cw * 4 * (2 + D);
-    if (c < 2) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float* mh = mw + (2 * c + j) * (2 + D);
-        if (g == 0) mh[0] = m_run[j], mh[1] = l_run[j];
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          mh[2 + 16 * g + 2 * mt] = acc[mt][j];
-          mh[2 + 16 * g + 2 * mt + 1] = acc[mt][2 + j];
-        }
-      }
-    }
   }
   __syncthreads();
-  // merge the 4 consumer warps and write one partial per head
-  for (int idx = threadIdx.x; idx < 4 * (2 + D); idx += blockDim.x) {
-    const int hd = idx / (2 + D), k = idx % (2 + D);
+}
+
+// Combine the partials of every CTA that covered a (batch, kv-head) and rotate
+// back once: out = Pi_V^T (sum_s acc_s e^(m_s - M)) / (sum_s l_s e^(m_s - M)).
+// One CTA per (batch, q-head).
+__global__ void __launch_bounds__(128) decode_merge_persistent_kernel(const float* partials, int64_t G, int max_seg,
+                                                                      int64_t nblk, int64_t total, int Hq, int Hkv,
+                                                                      const float* PiV, float* out) {
+  __shared__ float orot[D];
+  __shared__ float ML[2];
+  __shared__ int64_t range[2];
+  const int64_t bq = blockIdx.x;
+  const int64_t b = bq / Hq, hq = bq % Hq;
+  const int group = Hq / Hkv;
+  const int64_t bh = b * Hkv + hq / group;
+  const int hd = (int)(hq % group);
+  const int64_t lo = bh * nblk, hi = lo + nblk;
+  if (threadIdx.x == 0) {
+    // first CTA whose block range meets [lo, hi)
+    int64_t i = lo * G / total;
+    while (i > 0 && cta_first_block(i, total, G) > lo) --i;
+    while (i < G && cta_first_block(i + 1, total, G) <= lo) ++i;
+    int64_t i1 = i;
     float M = -FLT_MAX;
-    for (int w = 0; w < kCons; ++w) M = fmaxf(M, mrg[(w * 4 + hd) * (2 + D)]);
-    float v = 0.f;
-    if (k == 0) {
-      v = M;
-    } else {
-      for (int w = 0; w < kCons; ++w) {
-        const float* mh = mrg + (w * 4 + hd) * (2 + D);
-        v += mh[k] * exp2f(mh[0] - M);
-      }
+    for (; i1 < G && cta_first_block(i1, total, G) < hi; ++i1) {
+      const int64_t sg = bh - cta_first_block(i1, total, G) / nblk;
+      M = fmaxf(M, partials[((i1 * max_seg + sg) * 4 + hd) * (D + 2) + D]);
     }
-    const int hq = h * (a.Hq / a.Hkv) + hd;
-    float* out = a.partials + (((int64_t)b * a.Hq + hq) * a.splits + split) * (D + 2);
-    // partial layout: acc[0..d), m, l  -- m in natural-log units for the merge kernel
-    if (k == 0) out[D] = M / kLog2e;
-    else if (k == 1) out[D + 1] = v;
-    else out[k - 2] = v;
+    float L = 0.f;
+    for (int64_t k = i; k < i1; ++k) {
+      const int64_t sg = bh - cta_first_block(k, total, G) / nblk;
+      const float* p = partials + ((k * max_seg + sg) * 4 + hd) * (D + 2);
+      L += p[D + 1] * __expf(p[D] - M);
+    }
+    range[0] = i;
+    range[1] = i1;
+    ML[0] = M;
+    ML[1] = L;
+  }
+  __syncthreads();
+  const float M = ML[0], invL = 1.f / ML[1];
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+    float v = 0.f;
+    for (int64_t k = range[0]; k < range[1]; ++k) {
+      const int64_t sg = bh - cta_first_block(k, total, G) / nblk;
+      const float* p = partials + ((k * max_seg + sg) * 4 + hd) * (D + 2);
+      v += p[j] * __expf(p[D] - M);
+    }
+    orot[j] = v * invL;
+  }
+  __syncthreads();
+  for (int i2 = threadIdx.x; i2 < D; i2 += blockDim.x) {
+    float v = 0.f;
+    for (int j = 0; j < D; ++j) v = fmaf(PiV[(int64_t)j * D + i2], orot[j], v);
+    out[bq * D + i2] = v;
   }
 }
 
@@ -399,19 +481,25 @@ bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, i
          hk->dev.ktab != nullptr && hv->dev.vtab != nullptr;
 }
 
-int decode_mma_splits(int B, int Hkv, int64_t T, int sm_count) {
-  const int64_t bh = (int64_t)B * Hkv;
-  int64_t s = (2 * (int64_t)sm_count + bh - 1) / bh;
-  const int64_t cap = (T + 255) / 256;
-  s = s < 1 ? 1 : s;
-  s = s > cap ? cap : s;
-  return (int)(s > 1024 ? 1024 : s);
+// grid of the persistent kernel (2 CTAs per SM) and the partial slots each CTA needs
+int decode_mma_grid(int B, int Hkv, int64_t T, int sm_count) {
+  const int64_t total = (int64_t)B * Hkv * ((T + kBlk - 1) / kBlk);
+  const int64_t g = 2 * (int64_t)sm_count;
+  return (int)(total < g ? total : g);
+}
+
+int decode_mma_max_seg(int B, int Hkv, int64_t T, int sm_count) {
+  const int64_t nblk = (T + kBlk - 1) / kBlk;
+  const int64_t total = (int64_t)B * Hkv * nblk;
+  const int64_t G = decode_mma_grid(B, Hkv, T, sm_count);
+  const int64_t per = (total + G - 1) / G;
+  return (int)((per + nblk - 1) / nblk + 1);
 }
 
 int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
                       int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
-                      const float* vnorms, float scale, int splits, float* partials, float* out, void* stream) {
+                      const float* vnorms, float scale, float* partials, float* out, void* stream) {
   DecArgs a;
   a.kcodes = kcodes;
   a.ksigns = ksigns;
@@ -426,18 +514,17 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
-  a.splits = splits;
   a.T = T;
   a.kv_stride = kv_stride;
-  // split boundaries on whole 64-token blocks
-  int64_t per = (T + splits - 1) / splits;
-  per = (per + kBlk - 1) / kBlk * kBlk;
-  a.per_split = per;
+  a.nblk = (T + kBlk - 1) / kBlk;
+  a.total = (int64_t)B * Hkv * a.nblk;
+  a.max_seg = decode_mma_max_seg(B, Hkv, T, hk->sm_count);
   a.scale_log2 = scale * kLog2e;
   a.qjl_coef = 1.2533141373155003f / 128.0f;
   a.partials = partials;
   a.status = hk->dev.status;
-  const int smem = kStages * kStageBytes + 2 * kStages * 8 + kCons * 64 * 2 + kCons * 4 * (2 + D) * 4;
+  const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
+  const int smem = kStages * kStageBytes + (2 * kStages + 2) * 8 + kCons * 64 * 2 + 2 * kCons * 4 * (2 + D) * 4;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -445,10 +532,12 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
     attr = true;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  decode_mma_kernel<<<dim3(splits, B * Hkv), kThreads, smem, s>>>(a);
+  decode_mma_kernel<<<G, kThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  return launch_decode_merge(partials, B * Hq, splits, hv, out, stream);
+  decode_merge_persistent_kernel<<<B * Hq, 128, 0, s>>>(partials, G, a.max_seg, a.nblk, a.total, Hq, Hkv,
+                                                        hv->dev.Pi, out);
+  return (int)cudaGetLastError();
 }
 
 }  // namespace tqi

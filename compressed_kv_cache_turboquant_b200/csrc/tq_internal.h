@@ -85,12 +85,13 @@ int launch_topk_simple(const float* scores, int64_t nq, int64_t N, int k, int32_
 int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out,
                         void* stream);
 bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride);
-int decode_mma_splits(int B, int Hkv, int64_t T, int sm_count);
+int decode_mma_grid(int B, int Hkv, int64_t T, int sm_count);
+int decode_mma_max_seg(int B, int Hkv, int64_t T, int sm_count);
 int launch_qfrag(const float* qrot, const float* qproj, int64_t nq, void* qfrag, float* qscale, void* stream);
 int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
                       int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
-                      const float* vnorms, float scale, int splits, float* partials, float* out, void* stream);
+                      const float* vnorms, float scale, float* partials, float* out, void* stream);
 // decode attention through whichever kernel fits; workspace layout owned here
 size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t T);
 int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,

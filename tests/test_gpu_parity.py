@@ -256,3 +256,16 @@ def test_decode_small_ragged():
 def test_decode_cfg4_full_size_sampled():
     """B = 8, Hq = 32, Hkv = 8, d = 128, T = 131072: full launch, sampled slices."""
     _decode_case(B=8, Hq=32, Hkv=8, T=131072, d=128, sample=[(0, 0), (7, 7), (3, 5)], seed=0)
+
+
+def test_decode_one_kv_head_long_context():
+    """A single (batch, kv-head): every CTA of the persistent grid works on it and the
+    merge combines hundreds of partials."""
+    _decode_case(B=1, Hq=4, Hkv=1, T=70001, d=128, sample=[(0, 0)], seed=2)
+
+
+def test_decode_fallback_shapes():
+    """Shapes the register-decode kernel does not take (odd cache stride, 2 q-heads per
+    kv-head) go through the general kernel and must agree just the same."""
+    _decode_case(B=1, Hq=4, Hkv=1, T=777, d=128, sample=[(0, 0)], seed=3, stride_extra=3)
+    _decode_case(B=2, Hq=4, Hkv=2, T=500, d=128, sample=[(0, 1), (1, 0)], seed=4)
