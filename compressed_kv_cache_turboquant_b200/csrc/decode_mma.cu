@@ -19,10 +19,10 @@
 //   the four warps' states merge in shared memory; partial (max, sum, acc[d])
 //   per head goes to the workspace; the merge kernel combines the splits and
 //   rotates back once.
-// Decoding is register-only: 3-bit key indices and 4-bit value indices become
-// fp16 through byte-permute lookups in 8-entry byte tables (the value
-// codebook's symmetry c[15-i] = -c[i] keeps its table at 8 entries); QJL bits
-// become +-1.0 with one shift and one logic op per pair.
+// Decoding: every byte of key or value codes holds two indices and is turned
+// into an fp16 pair by one lookup in a 256-entry table in shared memory (one
+// table replica per lane, so the 32 lookups of a warp never share a bank); QJL
+// bits become +-1.0 with one shift and one logic op per pair.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -37,22 +37,35 @@ namespace {
 using namespace sm100;
 
 constexpr int D = 128;
-constexpr int kBlk = 64;       // tokens per stage
-constexpr int kStages = 8;
-constexpr int kCons = 4;       // consumer warps
+constexpr int kBlk = 128;      // tokens per stage (16 per consumer warp)
+constexpr int kStages = 4;
+constexpr int kCons = 8;       // consumer warps
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kKW = 12;        // K code words per token (3 bits x 128 / 32)
 constexpr int kSW = 4;         // sign words
 constexpr int kVW = 16;        // V code words (4 bits)
 // stage layout (bytes)
 constexpr int kOffK = 0;
-constexpr int kOffS = kOffK + kBlk * kKW * 4;   // 3072
-constexpr int kOffV = kOffS + kBlk * kSW * 4;   // 4096
-constexpr int kOffN = kOffV + kBlk * kVW * 4;   // 8192
+constexpr int kOffS = kOffK + kBlk * kKW * 4;
+constexpr int kOffV = kOffS + kBlk * kSW * 4;
+constexpr int kOffN = kOffV + kBlk * kVW * 4;
 constexpr int kOffR = kOffN + kBlk * 4;
 constexpr int kOffVN = kOffR + kBlk * 4;
-constexpr int kStageBytes = kOffVN + kBlk * 4;  // 8960
+constexpr int kStageBytes = kOffVN + kBlk * 4;  // 17920
+// Decode tables in shared memory, 256 rows of 256 bytes each, indexed by one
+// byte of codes (two indices, or eight sign bits):
+//   KV table, row B: [K entry, one 4-byte copy per lane][V entry, one per lane]
+//     K entry = fp16 pair (cK[B & 7], cK[(B >> 4) & 7])   (3-bit codes; bits 3, 7 ignored)
+//     V entry = fp16 pair (cV[B & 15], cV[B >> 4])         (4-bit codes)
+//   sign table, row B: 16 copies of 16 bytes = four fp16 pairs (s0,s1)..(s6,s7),
+//     s_i = +1.0 if bit i of B is set, else -1.0
+// With a copy per lane (per 16-byte lane group for the sign rows) the lookups
+// of a warp never meet in a bank, and the address of a lookup is one byte
+// permute: (code byte) << 8 | (lane offset).
+constexpr int kTabBytes = 256 * 256;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 4.0f;        // rescale only when a logit passes the running max by 2^4
+constexpr float kPScale = 0.0625f;   // fp16 weights p * ||v|| / 16 stay below ||v||
 
 struct DecArgs {
   const uint32_t* kcodes;
@@ -61,13 +74,13 @@ struct DecArgs {
   const float* krnorms;
   const uint32_t* vcodes;
   const float* vnorms;
-  const uint32_t* qfrag;   // [B*Hq][2][128] fp16 pairs: rotated (natural order), projected (QJL order)
+  const uint32_t* qfrag;   // [B*Hq][2][128] fp16: rotated and projected queries, coordinate order
   const float* qscale;     // [B*Hq][2]: 1/s for the two fp16 query copies
-  const uint32_t* ktab;    // [4]: K centroid lo bytes c0..3, c4..7, hi bytes c0..3, c4..7
-  const uint32_t* vtab;    // [4]: V magnitude table |c|[8..15], lo and hi bytes
+  const uint32_t* klut;    // [16]: fp16 of the key codebook c0..c7 in the low halves
+  const uint32_t* vlut;    // [16]: fp16 of the value codebook c0..c15 in the low halves
   int B, Hq, Hkv;
   int64_t T, kv_stride;
-  int64_t nblk;            // 64-token blocks per (batch, kv-head)
+  int64_t nblk;            // token blocks per (batch, kv-head)
   int64_t total;           // B * Hkv * nblk
   int max_seg;             // partial slots per CTA
   float scale_log2;        // logit scale * log2(e)
@@ -93,52 +106,57 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 8 coordinates whose 3-bit indices sit in the nibbles of `sel` (bit 3 clear)
-// -> 4 fp16 pairs (coords 0-1, 2-3, 4-5, 6-7) from the 8-entry byte tables
-__device__ __forceinline__ void lut8(uint32_t sel, uint32_t tl0, uint32_t tl1, uint32_t th0, uint32_t th1,
-                                     uint32_t* out) {
-  const uint32_t s1 = sel >> 16;
-  const uint32_t la = prmt(tl0, tl1, sel), ha = prmt(th0, th1, sel);
-  const uint32_t lb = prmt(tl0, tl1, s1), hb = prmt(th0, th1, s1);
-  out[0] = prmt(la, ha, 0x5140);
-  out[1] = prmt(la, ha, 0x7362);
-  out[2] = prmt(lb, hb, 0x5140);
-  out[3] = prmt(lb, hb, 0x7362);
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// the 4 bytes of a code word -> 4 fp16 pairs; `lane_off` holds this lane's
+// column offset in byte 0, `tab` the table's shared-memory address
+__device__ __forceinline__ void lookup4(uint32_t w, uint32_t tab, uint32_t lane_off, uint32_t* out) {
+  out[0] = lds32(tab + prmt(w, lane_off, 0x5504));
+  out[1] = lds32(tab + prmt(w, lane_off, 0x5514));
+  out[2] = lds32(tab + prmt(w, lane_off, 0x5524));
+  out[3] = lds32(tab + prmt(w, lane_off, 0x5534));
 }
 
 // one 3-bit group of 32 coordinates (words w0..w2, layout of tq.h) -> 16 fp16 pairs in coordinate order
-__device__ __forceinline__ void decode_k3(uint32_t w0, uint32_t w1, uint32_t w2, const uint32_t (&t)[4],
+__device__ __forceinline__ void decode_k3(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t tab, uint32_t lane_off,
                                           uint32_t (&h)[16]) {
+  // coordinates 24..31 live in the fourth bit of every nibble of w0..w2
   const uint32_t s3 = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
-  lut8(w0 & 0x77777777u, t[0], t[1], t[2], t[3], h + 0);
-  lut8(w1 & 0x77777777u, t[0], t[1], t[2], t[3], h + 4);
-  lut8(w2 & 0x77777777u, t[0], t[1], t[2], t[3], h + 8);
-  lut8(s3, t[0], t[1], t[2], t[3], h + 12);
+  lookup4(w0, tab, lane_off, h + 0);
+  lookup4(w1, tab, lane_off, h + 4);
+  lookup4(w2, tab, lane_off, h + 8);
+  lookup4(s3, tab, lane_off, h + 12);
 }
 
-// 8 coordinates of 4-bit value indices (one word) -> 4 fp16 pairs in coordinate order.
-// c[i] = +T[i-8] for i >= 8, -T[7-i] for i < 8 (symmetric codebook), T = |c| of the upper half.
-__device__ __forceinline__ void decode_v4(uint32_t w, const uint32_t (&t)[4], uint32_t* out) {
-  const uint32_t neg = (~w >> 3) & 0x11111111u;        // 1 where the index is in the lower half
-  const uint32_t mag = (w ^ (neg * 7u)) & 0x77777777u;  // magnitude index m
-  const uint32_t sg = neg << 2;                         // selector 4 -> byte 0x80, 0 -> 0x00
-  const uint32_t m1 = mag >> 16, g1 = sg >> 16;
-  const uint32_t la = prmt(t[0], t[1], mag), ha = prmt(t[2], t[3], mag) ^ prmt(0u, 0x80u, sg);
-  const uint32_t lb = prmt(t[0], t[1], m1), hb = prmt(t[2], t[3], m1) ^ prmt(0u, 0x80u, g1);
-  out[0] = prmt(la, ha, 0x5140);
-  out[1] = prmt(la, ha, 0x7362);
-  out[2] = prmt(lb, hb, 0x5140);
-  out[3] = prmt(lb, hb, 0x7362);
+// 32 QJL sign bits -> 16 fp16 pairs (+-1.0) in coordinate order
+__device__ __forceinline__ void decode_signs(uint32_t w, uint32_t tab, uint32_t lane_off, uint32_t (&h)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = lds128(tab + prmt(w, lane_off, 0x5504 | (i << 4)));
+    h[4 * i + 0] = v.x, h[4 * i + 1] = v.y, h[4 * i + 2] = v.z, h[4 * i + 3] = v.w;
+  }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* kvtab = smem + kStages * kStageBytes;
+  uint8_t* sgtab = kvtab + kTabBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sgtab + kTabBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* pub = empty + kStages;                                        // consumers published their state
+  uint64_t* pub = empty + kStages;                                        // consumer sync at segment ends
   __half* pbuf = reinterpret_cast<__half*>(pub + 2);                     // [kCons][4 heads][16 tokens]
-  float* mrg = reinterpret_cast<float*>(pbuf + kCons * 64);               // [2][kCons][4][2 + D]
+  float* mrg = reinterpret_cast<float*>(pbuf + kCons * 64);               // [kCons][4][2 + D]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t G = gridDim.x;
@@ -152,6 +170,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
     }
     mbar_init(pub, 32 * kCons);
     fence_mbar_init();
+  }
+  // tables
+  {
+    uint32_t* kv = reinterpret_cast<uint32_t*>(kvtab);
+    for (int w = threadIdx.x; w < kTabBytes / 4; w += blockDim.x) {
+      const uint32_t row = (uint32_t)w >> 6, col = (uint32_t)w & 63u;
+      kv[w] = (col < 32) ? ((a.klut[row & 7u] & 0xFFFFu) | (a.klut[(row >> 4) & 7u] << 16))
+                         : ((a.vlut[row & 15u] & 0xFFFFu) | (a.vlut[row >> 4] << 16));
+    }
+    uint32_t* sg = reinterpret_cast<uint32_t*>(sgtab);
+    for (int w = threadIdx.x; w < kTabBytes / 4; w += blockDim.x) {
+      const uint32_t row = (uint32_t)w >> 6, pair = (uint32_t)w & 3u;
+      const uint32_t lo = ((row >> (2 * pair)) & 1u) ? 0x3C00u : 0xBC00u;
+      const uint32_t hi = ((row >> (2 * pair + 1)) & 1u) ? 0x3C00u : 0xBC00u;
+      sg[w] = lo | (hi << 16);
+    }
   }
   __syncthreads();
 
@@ -183,37 +217,36 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
     }
   } else {
     const int cw = warp - 1;           // consumer index
-    const int ct = threadIdx.x - 32;   // consumer thread 0..127
+    const int ct = threadIdx.x - 32;   // consumer thread 0..255
     const int g = lane >> 2, c = lane & 3;
     const int cp = c & 1;              // heads 2cp, 2cp+1 handled by this lane
     const int group = a.Hq / a.Hkv;    // 4
-    uint32_t kt[4], vt[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) kt[i] = a.ktab[i], vt[i] = a.vtab[i];
+    const uint32_t kvt = smem_u32(kvtab), sgt = smem_u32(sgtab);
+    const uint32_t k_off = (uint32_t)lane * 4u, v_off = 128u + (uint32_t)lane * 4u;
+    const uint32_t s_off = (uint32_t)(lane & 15) * 16u;
     uint32_t bm[8][2], bq[8][2];
     float inv_s1[2], inv_s2[2];
-    float m_run[2], l_run[2];
+    float m_ref[2], l_run[2];
     float acc[8][4];
     __half* pb = pbuf + cw * 64;
     int64_t cur_bh = -1;
     int seg = -1;
     bool ok = true;
 
-    // publish this warp's state, combine the four warps, write one partial
-    auto flush = [&](int sg, int64_t bhv) {
+    // publish this warp's state, combine the eight warps, write one partial
+    auto flush = [&](int sg) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
         l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
         l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
       }
-      float* mb = mrg + (sg & 1) * kCons * 4 * (2 + D);
-      float* mw = mb + cw * 4 * (2 + D);
+      float* mw = mrg + cw * 4 * (2 + D);
       if (c < 2) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           float* mh = mw + (2 * c + j) * (2 + D);
-          if (g == 0) mh[0] = m_run[j], mh[1] = l_run[j];
+          if (g == 0) mh[0] = m_ref[j], mh[1] = l_run[j];
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             mh[2 + 16 * g + 2 * mt] = acc[mt][j];
@@ -222,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
         }
       }
       mbar_arrive(pub);
-      if (!mbar_wait(pub, (uint32_t)(sg & 1))) {
+      if (!mbar_wait(pub, 0u)) {
         ok = false;
         return;
       }
@@ -231,27 +264,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
         const int hd = idx / (2 + D), k = idx % (2 + D);
         float M = -FLT_MAX;
 #pragma unroll
-        for (int w = 0; w < kCons; ++w) M = fmaxf(M, mb[(w * 4 + hd) * (2 + D)]);
+        for (int w = 0; w < kCons; ++w) M = fmaxf(M, mrg[(w * 4 + hd) * (2 + D)]);
         if (k == 0) {
           dst[hd * (D + 2) + D] = M / kLog2e;  // natural-log units for the merge
         } else {
           float v = 0.f;
 #pragma unroll
           for (int w = 0; w < kCons; ++w) {
-            const float* mh = mb + (w * 4 + hd) * (2 + D);
+            const float* mh = mrg + (w * 4 + hd) * (2 + D);
             v += mh[k] * exp2f(mh[0] - M);
           }
           if (k == 1) dst[hd * (D + 2) + D + 1] = v;
           else dst[hd * (D + 2) + k - 2] = v;
         }
       }
-      (void)bhv;
+      // second phase: everyone has read the merge buffer before it is written again
+      mbar_arrive(pub);
+      if (!mbar_wait(pub, 1u)) ok = false;
     };
 
     for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i) {
       const int64_t bh = gb / a.nblk;
       if (bh != cur_bh) {
-        if (seg >= 0) flush(seg, cur_bh);
+        if (seg >= 0) flush(seg);
         if (!ok) break;
         ++seg;
         cur_bh = bh;
@@ -271,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           inv_s1[j] = a.qscale[2 * (q0 + 2 * cp + j)];
-          inv_s2[j] = a.qscale[2 * (q0 + 2 * cp + j) + 1];
-          m_run[j] = -FLT_MAX;
+          inv_s2[j] = a.qscale[2 * (q0 + 2 * cp + j) + 1] * a.qjl_coef;
+          m_ref[j] = -FLT_MAX;
           l_run[j] = 0.f;
         }
 #pragma unroll
@@ -289,95 +324,104 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
       const uint8_t* st = stages + s * kStageBytes;
       const int64_t t0 = (gb % a.nblk) * kBlk;
       const int n = (int)min((int64_t)kBlk, a.T - t0);
-      const int n4 = n & ~3;
-      const int64_t row0 = bh * a.kv_stride + t0;
       const int tb = cw * 16;  // this warp's 16 tokens within the block
       // ---------------- logits: keys g and g+8 of the sub-block
       float sc[4] = {0.f, 0.f, 0.f, 0.f};
       {
-        uint32_t hk0[16], hk1[16], sg0, sg1;
+        uint32_t h0[16], h1[16];
         const uint32_t* kc0 = reinterpret_cast<const uint32_t*>(st + kOffK) + (tb + g) * kKW + 3 * c;
         const uint32_t* kc1 = kc0 + 8 * kKW;
-        decode_k3(kc0[0], kc0[1], kc0[2], kt, hk0);
-        decode_k3(kc1[0], kc1[1], kc1[2], kt, hk1);
+        decode_k3(kc0[0], kc0[1], kc0[2], kvt, k_off, h0);
+        decode_k3(kc1[0], kc1[1], kc1[2], kvt, k_off, h1);
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb)
+          mma16816(sc, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bm[kb][0], bm[kb][1]);
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(st + kOffS);
-        sg0 = sw[(tb + g) * kSW + c];
-        sg1 = sw[(tb + g + 8) * kSW + c];
+        decode_signs(sw[(tb + g) * kSW + c], sgt, s_off, h0);
+        decode_signs(sw[(tb + g + 8) * kSW + c], sgt, s_off, h1);
 #pragma unroll
-        for (int kb = 0; kb < 8; ++kb) mma16816(sc, hk0[2 * kb], hk1[2 * kb], hk0[2 * kb + 1], hk1[2 * kb + 1],
-                                                 bm[kb][0], bm[kb][1]);
-        const uint32_t one = 0x3C003C00u;
-#pragma unroll
-        for (int kb = 0; kb < 8; ++kb) {
-          // sign pairs (coords m, m+16) for m = 2kb and 2kb+1; bit set -> +1.0
-          const uint32_t a0 = (~(sg0 << (15 - 2 * kb)) & 0x80008000u) | one;
-          const uint32_t a1 = (~(sg1 << (15 - 2 * kb)) & 0x80008000u) | one;
-          const uint32_t a2 = (~(sg0 << (14 - 2 * kb)) & 0x80008000u) | one;
-          const uint32_t a3 = (~(sg1 << (14 - 2 * kb)) & 0x80008000u) | one;
-          mma16816(sc, a0, a1, a2, a3, bq[kb][0], bq[kb][1]);
-        }
+        for (int kb = 0; kb < 8; ++kb)
+          mma16816(sc, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bq[kb][0], bq[kb][1]);
       }
-      // exchange: lanes c and c^2 hold the mse and QJL dots of the same heads
+      // lanes c and c^2 hold the mse and QJL dots of the same heads
       float ot[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) ot[e] = __shfl_xor_sync(0xffffffffu, sc[e], 2);
       const float* mse = (c < 2) ? sc : ot;
       const float* qjl = (c < 2) ? ot : sc;
-      // norms of keys g and g+8 (tail tokens past the copied multiple of 4 come from global memory)
+      // norms of keys g and g+8; a partial last block reads its tail from global memory
       float kn[2], kr[2], vn[2];
-      bool valid[2];
+      if (n == kBlk) {
+        const float* N0 = reinterpret_cast<const float*>(st + kOffN);
+        const float* R0 = reinterpret_cast<const float*>(st + kOffR);
+        const float* V0 = reinterpret_cast<const float*>(st + kOffVN);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          kn[r] = N0[tb + g + 8 * r];
+          kr[r] = R0[tb + g + 8 * r];
+          vn[r] = V0[tb + g + 8 * r];
+        }
+      } else {
+        const int n4 = n & ~3;
+        const int64_t row0 = bh * a.kv_stride + t0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int tok = tb + g + 8 * r;
+          if (tok < n4) {
+            kn[r] = reinterpret_cast<const float*>(st + kOffN)[tok];
+            kr[r] = reinterpret_cast<const float*>(st + kOffR)[tok];
+            vn[r] = reinterpret_cast<const float*>(st + kOffVN)[tok];
+          } else if (tok < n) {
+            kn[r] = a.knorms[row0 + tok];
+            kr[r] = a.krnorms[row0 + tok];
+            vn[r] = a.vnorms[row0 + tok];
+          } else {
+            kn[r] = kr[r] = vn[r] = 0.f;
+          }
+        }
+      }
+      // logits in base 2: [token r][head j]; tokens past the context end are -inf
+      float lg[2][2];
+      bool grow = false;
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int tok = tb + g + 8 * r;
-        valid[r] = tok < n;
-        if (tok < n4) {
-          kn[r] = reinterpret_cast<const float*>(st + kOffN)[tok];
-          kr[r] = reinterpret_cast<const float*>(st + kOffR)[tok];
-          vn[r] = reinterpret_cast<const float*>(st + kOffVN)[tok];
-        } else if (tok < n) {
-          const int64_t gi = row0 + tok;
-          kn[r] = a.knorms[gi];
-          kr[r] = a.krnorms[gi];
-          vn[r] = a.vnorms[gi];
-        } else {
-          kn[r] = kr[r] = vn[r] = 0.f;
-        }
-      }
-      // logits (base 2): [token r][head j]
-      float lg[2][2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
+        const bool valid = (tb + g + 8 * r) < n;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const float est = kn[r] * mse[2 * r + j] * inv_s1[j] + kr[r] * a.qjl_coef * qjl[2 * r + j] * inv_s2[j];
-          lg[r][j] = valid[r] ? est * a.scale_log2 : -FLT_MAX;
-        }
-      // online softmax per head over the 16 tokens
-      float alpha[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float mx = fmaxf(lg[0][j], lg[1][j]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mn = fmaxf(m_run[j], mx);
-        alpha[j] = exp2f(m_run[j] - mn);
-        m_run[j] = mn;
-        const float p0 = valid[0] ? exp2f(lg[0][j] - mn) : 0.f;
-        const float p1 = valid[1] ? exp2f(lg[1][j] - mn) : 0.f;
-        l_run[j] = l_run[j] * alpha[j] + p0 + p1;
-        // weights carry the value norms
-        if (c < 2) {
-          pb[(2 * cp + j) * 16 + g] = __float2half_rn(p0 * vn[0]);
-          pb[(2 * cp + j) * 16 + g + 8] = __float2half_rn(p1 * vn[1]);
+          const float est = fmaf(kn[r] * inv_s1[j], mse[2 * r + j], kr[r] * inv_s2[j] * qjl[2 * r + j]);
+          lg[r][j] = valid ? est * a.scale_log2 : -FLT_MAX;
+          grow |= lg[r][j] > m_ref[j] + kLazy;
         }
       }
+      // lazy rescale: the reference max moves only when some logit passes it by kLazy
+      if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        acc[mt][0] *= alpha[0];
-        acc[mt][1] *= alpha[1];
-        acc[mt][2] *= alpha[0];
-        acc[mt][3] *= alpha[1];
+        for (int j = 0; j < 2; ++j) {
+          float mx = fmaxf(lg[0][j], lg[1][j]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float mn = fmaxf(m_ref[j], mx);
+          const float alpha = exp2f(m_ref[j] - mn);
+          m_ref[j] = mn;
+          l_run[j] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            acc[mt][j] *= alpha;
+            acc[mt][2 + j] *= alpha;
+          }
+        }
+      }
+      const bool v0 = (tb + g) < n, v1 = (tb + g + 8) < n;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float p0 = v0 ? exp2f(lg[0][j] - m_ref[j]) : 0.f;
+        const float p1 = v1 ? exp2f(lg[1][j] - m_ref[j]) : 0.f;
+        l_run[j] += (p0 + p1) * kPScale;
+        if (c < 2) {
+          pb[(2 * cp + j) * 16 + g] = __float2half_rn(p0 * vn[0] * kPScale);
+          pb[(2 * cp + j) * 16 + g + 8] = __float2half_rn(p1 * vn[1] * kPScale);
+        }
       }
       __syncwarp();
       uint32_t pw0 = 0u, pw1 = 0u;
@@ -393,14 +437,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
         const uint2 wb = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 1) * kVW + 2 * g);
         const uint2 wc = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 8) * kVW + 2 * g);
         const uint2 wd = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 9) * kVW + 2 * g);
-        decode_v4(wa.x, vt, xa);
-        decode_v4(wa.y, vt, xa + 4);
-        decode_v4(wb.x, vt, xb);
-        decode_v4(wb.y, vt, xb + 4);
-        decode_v4(wc.x, vt, xc);
-        decode_v4(wc.y, vt, xc + 4);
-        decode_v4(wd.x, vt, xd);
-        decode_v4(wd.y, vt, xd + 4);
+        lookup4(wa.x, kvt, v_off, xa);
+        lookup4(wa.y, kvt, v_off, xa + 4);
+        lookup4(wb.x, kvt, v_off, xb);
+        lookup4(wb.y, kvt, v_off, xb + 4);
+        lookup4(wc.x, kvt, v_off, xc);
+        lookup4(wc.y, kvt, v_off, xc + 4);
+        lookup4(wd.x, kvt, v_off, xd);
+        lookup4(wd.y, kvt, v_off, xd + 4);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           // rows (coords 16g + 2mt, 16g + 2mt + 1), token pairs (2c, 2c+1) and (2c+8, 2c+9)
@@ -412,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(DecArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (ok && seg >= 0) flush(seg, cur_bh);
+    if (ok && seg >= 0) flush(seg);
     if (!ok) atomicOr(a.status, kStatusTimeout);
   }
   __syncthreads();
@@ -478,13 +522,13 @@ __global__ void __launch_bounds__(128) decode_merge_persistent_kernel(const floa
 
 bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride) {
   return hk->d == 128 && hv->d == 128 && hk->bm == 3 && hv->bm == 4 && Hq == 4 * Hkv && (kv_stride % 4) == 0 &&
-         hk->dev.ktab != nullptr && hv->dev.vtab != nullptr;
+         hk->dev.lut_dq != nullptr && hv->dev.lut_dq != nullptr;
 }
 
 // grid of the persistent kernel (2 CTAs per SM) and the partial slots each CTA needs
 int decode_mma_grid(int B, int Hkv, int64_t T, int sm_count) {
   const int64_t total = (int64_t)B * Hkv * ((T + kBlk - 1) / kBlk);
-  const int64_t g = 2 * (int64_t)sm_count;
+  const int64_t g = (int64_t)sm_count;  // one CTA per SM
   return (int)(total < g ? total : g);
 }
 
@@ -509,8 +553,8 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.vnorms = vnorms;
   a.qfrag = qfrag;
   a.qscale = qscale;
-  a.ktab = hk->dev.ktab;
-  a.vtab = hv->dev.vtab;
+  a.klut = hk->dev.lut_dq;
+  a.vlut = hv->dev.lut_dq;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -524,7 +568,8 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.partials = partials;
   a.status = hk->dev.status;
   const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
-  const int smem = kStages * kStageBytes + (2 * kStages + 2) * 8 + kCons * 64 * 2 + 2 * kCons * 4 * (2 + D) * 4;
+  const int smem = kStages * kStageBytes + 2 * kTabBytes + (2 * kStages + 2) * 8 + kCons * 64 * 2 +
+                   kCons * 4 * (2 + D) * 4;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -546,11 +591,8 @@ namespace tqi {
 namespace {
 
 // Rotated / projected queries (fp32, from query_prep) -> scaled fp16 MMA B
-// operands.  Per query: s = 2^(14 - ceil(log2 max|v|)) so the largest entry
-// lands in (2^13, 2^14]; 1/s is kept to undo it.  The rotated copy stays in
-// coordinate order; the projected copy is permuted within each group of 32 so
-// that position 4kb + e holds coordinate 2kb, 2kb+16, 2kb+1, 2kb+17 (e = 0..3),
-// the order in which the decode kernel pairs QJL sign bits.
+// operands, both in coordinate order.  Per query copy: s = 2^(14 - ceil(log2
+// max|v|)) so the largest entry lands in (2^13, 2^14]; 1/s is kept to undo it.
 __global__ void qfrag_kernel(const float* qrot, const float* qproj, int64_t nq, __half* qfrag, float* qscale) {
   const int64_t qi = blockIdx.x;
   if (qi >= nq) return;
@@ -566,13 +608,7 @@ __global__ void qfrag_kernel(const float* qrot, const float* qproj, int64_t nq, 
     int e = 0;
     if (mx > 0.f) (void)frexpf(mx, &e);  // mx in [2^(e-1), 2^e)
     const float s = (mx > 0.f) ? ldexpf(1.f, 14 - e) : 1.f;
-    int coord = t;
-    if (which) {
-      const int grp = t >> 5, pp = t & 31, kb = pp >> 2, el = pp & 3;
-      const int off = (el == 0) ? 2 * kb : (el == 1) ? 2 * kb + 16 : (el == 2) ? 2 * kb + 1 : 2 * kb + 17;
-      coord = 32 * grp + off;
-    }
-    qfrag[qi * 2 * D + which * D + t] = __float2half_rn(src[coord] * s);
+    qfrag[qi * 2 * D + which * D + t] = __float2half_rn(src[t] * s);
     if (t == 0) qscale[2 * qi + which] = 1.f / s;
     __syncthreads();
   }
