@@ -18,7 +18,7 @@ __all__ = [
     "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQError", "Handle", "code_words", "sign_words",
     "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
-    "tq_attn_decode_static",
+    "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
 ]
 
 
@@ -180,3 +180,44 @@ def tq_attn_decode_static(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: 
     check("tq_attn_decode_static", lib.tq_attn_decode_static(
         hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, kv_stride, _ptr(kcodes), _ptr(ksigns),
         _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out), _stream(stream)))
+
+
+def tq_device_status(h: Handle) -> int:
+    v = ctypes.c_int(0)
+    check("tq_device_status", lib.tq_device_status(h.ptr, ctypes.byref(v)))
+    return v.value
+
+
+def tq_quant_gather(h: Handle, x: torch.Tensor, channels: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
+                    signs=None, rnorms=None, out_stride: int = 1, stream=None) -> None:
+    """Quantize x[:, channels] (one channel group of a split cache)."""
+    check("tq_quant_gather", lib.tq_quant_gather(h.ptr, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1],
+                                                 _ptr(channels), _ptr(codes), _ptr(signs), _ptr(norms),
+                                                 _ptr(rnorms), out_stride, _stream(stream)))
+
+
+def _ptr_array(items):
+    arr = (ctypes.c_void_p * len(items))()
+    for i, t in enumerate(items):
+        arr[i] = _ptr(t)
+    return arr
+
+
+def tq_attn_logits_workspace(handles, B: int, Hq: int) -> int:
+    hs = (ctypes.c_void_p * len(handles))(*[h.ptr for h in handles])
+    return int(lib.tq_attn_logits_workspace(hs, len(handles), B, Hq))
+
+
+def tq_attn_logits(handles, channels, q: torch.Tensor, Hkv: int, T: int, kv_stride: int, kcodes, ksigns, knorms,
+                   krnorms, scale: float, logits: torch.Tensor, workspace=None, stream=None) -> None:
+    """Logits [B][Hq][T] over a key cache of one or two channel groups (lists
+    of per-group tensors); q is [B][Hq][dq]."""
+    B, Hq, dq = q.shape
+    hs = (ctypes.c_void_p * len(handles))(*[h.ptr for h in handles])
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_attn_logits_workspace(handles, B, Hq)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_attn_logits", lib.tq_attn_logits(hs, len(handles), _ptr(channels), _ptr(q), _dtype_code(q), dq, B, Hq,
+                                               Hkv, T, kv_stride, _ptr_array(kcodes), _ptr_array(ksigns),
+                                               _ptr_array(knorms), _ptr_array(krnorms), float(scale), _ptr(logits),
+                                               _ptr(workspace), workspace.numel(), _stream(stream)))

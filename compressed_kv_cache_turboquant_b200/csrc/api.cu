@@ -486,3 +486,92 @@ extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_d
                           vnorms, scale, out, workspace, stream);
   return e ? cuda_error("tq_attn_decode", e) : clear_error();
 }
+
+extern "C" int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                               const int32_t* channels, uint32_t* codes, uint32_t* signs, float* norms,
+                               float* rnorms, int64_t out_stride, void* stream) {
+  if (!h) return set_error(TQ_EINVAL, "tq_quant_gather: NULL handle");
+  if (N < 0) return set_error(TQ_EINVAL, "tq_quant_gather: N < 0");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return set_error(TQ_EUNSUPPORTED, "tq_quant_gather: dtype %d", dtype);
+  if (x_stride < 1 || out_stride < 1) return set_error(TQ_EINVAL, "tq_quant_gather: stride < 1");
+  const bool prod = h->variant == TQ_PROD;
+  if (N > 0 && (!x || !channels || !codes || !norms || (prod && (!signs || !rnorms))))
+    return set_error(TQ_EINVAL, "tq_quant_gather: NULL pointer");
+  // appends point at one token slot of a cache: element alignment is enough here
+  for (const void* p : {(const void*)x, (const void*)channels, (const void*)codes, (const void*)signs,
+                        (const void*)norms, (const void*)rnorms})
+    if (reinterpret_cast<uintptr_t>(p) & 3u)
+      return set_error(TQ_EALIGN, "tq_quant_gather: a device pointer is not 4-byte aligned");
+  if (N == 0) return clear_error();
+  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, prod ? signs : nullptr, norms, prod ? rnorms : nullptr,
+                              out_stride, stream, channels);
+  return e ? cuda_error("tq_quant_gather", e) : clear_error();
+}
+
+extern "C" size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, int Hq) {
+  if (!hk || ngroups < 1 || ngroups > 2 || B < 0 || Hq < 0) return 0;
+  size_t bytes = 0;
+  for (int g = 0; g < ngroups; ++g) {
+    if (!hk[g]) return 0;
+    bytes += 2 * align_up((size_t)B * Hq * hk[g]->d * 4, 256);
+  }
+  return bytes;
+}
+
+extern "C" int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* channels, const void* q, int q_dtype,
+                              int dq, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
+                              const uint32_t* const* kcodes, const uint32_t* const* ksigns,
+                              const float* const* knorms, const float* const* krnorms, float scale, float* logits,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!hk || ngroups < 1 || ngroups > 2) return set_error(TQ_EINVAL, "tq_attn_logits: need 1 or 2 groups");
+  int dsum = 0;
+  for (int g = 0; g < ngroups; ++g) {
+    if (!hk[g] || hk[g]->variant != TQ_PROD) return set_error(TQ_EINVAL, "tq_attn_logits: need TQ_PROD handles");
+    dsum += hk[g]->d;
+  }
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16)
+    return set_error(TQ_EUNSUPPORTED, "tq_attn_logits: q_dtype %d", q_dtype);
+  if (B < 0 || Hq < 0 || Hkv <= 0 || Hq != 4 * Hkv || T < 0 || kv_stride < T)
+    return set_error(TQ_EUNSUPPORTED, "tq_attn_logits: need Hq = 4 Hkv and kv_stride >= T");
+  if (!channels && (ngroups != 1 || dq != hk[0]->d))
+    return set_error(TQ_EINVAL, "tq_attn_logits: channels may be NULL only for one group with dq = d");
+  if (channels && dq < 1) return set_error(TQ_EINVAL, "tq_attn_logits: dq < 1");
+  (void)dsum;
+  if (!std::isfinite(scale)) return set_error(TQ_EINVAL, "tq_attn_logits: scale is not finite");
+  if (!logits_supported(hk, ngroups))
+    return set_error(TQ_EUNSUPPORTED, "tq_attn_logits: groups must be d = 64 (two groups) or 64/128 (one), mse bits 1..3");
+  if (B == 0 || Hq == 0 || T == 0) return clear_error();
+  if (!q || !logits || !kcodes || !ksigns || !knorms || !krnorms)
+    return set_error(TQ_EINVAL, "tq_attn_logits: NULL pointer");
+  for (int g = 0; g < ngroups; ++g) {
+    if (!kcodes[g] || !ksigns[g] || !knorms[g] || !krnorms[g]) return set_error(TQ_EINVAL, "tq_attn_logits: NULL pointer");
+    for (const void* p : {(const void*)kcodes[g], (const void*)ksigns[g], (const void*)knorms[g],
+                          (const void*)krnorms[g]})
+      TQ_CHECK_ALIGN(p, "a device pointer");
+  }
+  for (const void* p : {(const void*)q, (const void*)logits, (const void*)channels, (const void*)workspace})
+    TQ_CHECK_ALIGN(p, "a device pointer");
+  const size_t need = tq_attn_logits_workspace(hk, ngroups, B, Hq);
+  if (!workspace || ws_bytes < need)
+    return set_error(TQ_EWORKSPACE, "tq_attn_logits: workspace %zu < %zu bytes", ws_bytes, need);
+  const float* qr[2] = {nullptr, nullptr};
+  const float* qp[2] = {nullptr, nullptr};
+  char* ws = (char*)workspace;
+  int off = 0;
+  int e = 0;
+  for (int g = 0; g < ngroups && !e; ++g) {
+    const size_t qb = align_up((size_t)B * Hq * hk[g]->d * 4, 256);
+    float* r = (float*)ws;
+    float* p = (float*)(ws + qb);
+    ws += 2 * qb;
+    e = launch_query_prep_gather(hk[g], q, q_dtype, (int64_t)B * Hq, dq, channels ? channels + off : nullptr, r, p,
+                                 stream);
+    qr[g] = r;
+    qp[g] = p;
+    off += hk[g]->d;
+  }
+  if (!e)
+    e = launch_logits(hk, ngroups, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale, logits,
+                      stream);
+  return e ? cuda_error("tq_attn_logits", e) : clear_error();
+}

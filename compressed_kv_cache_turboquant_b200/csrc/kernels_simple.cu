@@ -94,6 +94,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 
 struct QuantArgs {
   const void* x;
+  const int32_t* channels;  // optional: coordinate i reads x[channels[i]]
   int64_t N, x_stride, out_stride;
   int d, bm, prod;
   const float* PiT;  // [i][j] = Pi[j][i]
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(128) quant_simple_kernel(QuantArgs a) {
   for (int64_t v = blockIdx.x; v < a.N; v += gridDim.x) {
     float ss = 0.f;
     for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      float e = load_elem(x, v * a.x_stride + i);
+      float e = load_elem(x, v * a.x_stride + (a.channels ? a.channels[i] : i));
       xs[i] = e;
       ss += e * e;
     }
@@ -388,8 +389,8 @@ int grid_for(int64_t n, int cap) { return (int)((n < cap) ? (n > 0 ? n : 1) : ca
 
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
-                        int64_t out_stride, void* stream) {
-  QuantArgs a{x, N, x_stride, out_stride, h->d, h->bm, h->variant == TQ_PROD, h->dev.PiT,
+                        int64_t out_stride, void* stream, const int32_t* channels) {
+  QuantArgs a{x, channels, N, x_stride, out_stride, h->d, h->bm, h->variant == TQ_PROD, h->dev.PiT,
               h->dev.TT, h->dev.centroids, h->dev.thresholds, codes, signs, norms, rnorms};
   const size_t smem = 3 * (size_t)h->d * sizeof(float) + h->d;
   const int grid = grid_for(N, h->sm_count * 16);

@@ -72,7 +72,14 @@ int launch_quant_mse_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_str
                         float* norms, int64_t out_stride, void* stream);
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
-                        int64_t out_stride, void* stream);
+                        int64_t out_stride, void* stream, const int32_t* channels = nullptr);
+int launch_query_prep_gather(const tq_ctx* h, const void* q, int q_dtype, int64_t nq, int dq,
+                             const int32_t* channels, float* qrot, float* qproj, void* stream);
+bool logits_supported(const tq_ctx* const* hk, int ngroups);
+int launch_logits(const tq_ctx* const* hk, int ngroups, const float* const* qrot, const float* const* qproj, int B,
+                  int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* const* kcodes,
+                  const uint32_t* const* ksigns, const float* const* knorms, const float* const* krnorms,
+                  float scale, float* logits, void* stream);
 int launch_dequant_simple(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_t N,
                           void* out, int out_dtype, void* stream);
 int launch_query_prep(const tq_ctx* h, const float* q, int q_dtype, int64_t nq, float* qrot,

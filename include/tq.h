@@ -275,6 +275,54 @@ TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int 
                                  const uint32_t* vcodes, const float* vnorms, float scale, float* out,
                                  void* stream);
 
+/* ---------------------------------------------------------------- channel groups */
+
+/*
+ * tq_quant_gather -- quantize rows restricted to a list of channels:
+ * vector i is (x_i[channels[0]], ..., x_i[channels[d-1]]), then exactly
+ * tq_quant_mse / tq_quant_prod with the handle's variant.  Used to append a
+ * token to a key cache whose channels are split into groups that are quantized
+ * as separate instances (outlier channels at more bits, the rest at fewer:
+ * [tq.net, "TurboQuant 最近的进展和外溢影响"]; 3.5 bits per channel and quantizing
+ * each token as it arrives: [ttakun, "为什么TurboQuant把…"] / [ttakun, "新旧量化方案深度权衡矩阵"]).
+ *   channels   dev in, [d] int32 channel indices into a row of x (x_stride wide)
+ *   signs, rnorms  ignored (may be NULL) for TQ_MSE handles
+ *   other arguments as tq_quant_prod, except that pointers need only be
+ *   4-byte aligned (so codes/signs/norms may point at one token slot of a cache)
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                           const int32_t* channels, uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
+                           int64_t out_stride, void* stream);
+
+/*
+ * tq_attn_logits -- attention logits over a TurboQuant_prod key cache whose
+ * channels may be split into groups (the pages' outlier channels kept at
+ * higher precision, [tq.net, "TurboQuant 最近的进展和外溢影响"]; logits over a
+ * compressed cache, [tmdm, "实测数据"]).  For batch b, query head j
+ * (kv-head h = j / 4, grouped-query attention with 4 query heads per kv-head):
+ *   logits[b][j][t] = scale * sum_g est_g(q_bj[channels_g], k_{b,h,t,g})
+ * with est_g the TurboQuant_prod estimator of group g's handle.
+ *   hk         host array [ngroups] of TQ_PROD handles (1 group: d 64 or 128;
+ *              2 groups: d = 64 each), mse bits 1..3
+ *   channels   dev [sum d_g] int32: group g's channels of the query rows, at
+ *              offset sum_{g'<g} d_g'; NULL allowed for one group with dq = d
+ *   q          dev [B][Hq][dq] of q_dtype (TQ_F32 or TQ_BF16)
+ *   Hq         must be 4 * Hkv
+ *   kcodes, ksigns, knorms, krnorms   host arrays [ngroups] of dev pointers,
+ *              each group's cache laid out as in tq_attn_decode (row
+ *              (b*Hkv + h)*kv_stride + t)
+ *   logits     dev out, [B][Hq][T] float32
+ *   workspace  dev scratch of at least tq_attn_logits_workspace(...) bytes
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
+ */
+TQ_API int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* channels, const void* q, int q_dtype,
+                          int dq, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
+                          const uint32_t* const* kcodes, const uint32_t* const* ksigns,
+                          const float* const* knorms, const float* const* krnorms, float scale, float* logits,
+                          void* workspace, size_t ws_bytes, void* stream);
+TQ_API size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, int Hq);
+
 /* ---------------------------------------------------------------- diagnostics */
 
 /*

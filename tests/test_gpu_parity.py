@@ -269,3 +269,101 @@ def test_decode_fallback_shapes():
     kv-head) go through the general kernel and must agree just the same."""
     _decode_case(B=1, Hq=4, Hkv=1, T=777, d=128, sample=[(0, 0)], seed=3, stride_extra=3)
     _decode_case(B=2, Hq=4, Hkv=2, T=500, d=128, sample=[(0, 1), (1, 0)], seed=4)
+
+
+# ------------------------------------------------------------------ channel groups (3.5-bit streaming cache)
+
+def _split_instances(d=128, n_hi=64, seed=0):
+    scales = synth.lognormal_channel_scales(d, 1.0, seed, 30)
+    hi, lo = oq.channel_split(scales, n_hi)
+    ia = Instance(64, 4, tq.TQ_PROD, seed=seed, sub=(0,))
+    ib = Instance(64, 3, tq.TQ_PROD, seed=seed, sub=(1,))
+    channels = torch.tensor(np.concatenate([hi, lo]).astype(np.int32), device=DEV)
+    return scales, hi, lo, ia, ib, channels
+
+
+def _split_keys(T, h, scales, seed):
+    z = synth.rng(seed, synth.DATA, 40, h).standard_normal((T, len(scales)))
+    return bf16_exact(z * scales[None, :])
+
+
+def test_streaming_append_gathers_channel_groups():
+    """Tokens arrive one at a time for 8 kv-heads; each group of channels is
+    quantized into its own cache slot t (out_stride = cache capacity)."""
+    Hkv, cap, steps = 8, 40, 5
+    scales, hi, lo, ia, ib, channels = _split_instances()
+    keys = [_split_keys(steps, h, scales, 7) for h in range(Hkv)]
+    caches = {}
+    for inst, name, off in ((ia, "a", 0), (ib, "b", 64)):
+        caches[name] = inst.alloc_outputs(Hkv * cap)
+    for t in range(steps):
+        x = to_device(np.stack([keys[h][t] for h in range(Hkv)]), torch.bfloat16)  # [Hkv][128]
+        for inst, name, off in ((ia, "a", 0), (ib, "b", 64)):
+            c = caches[name]
+            sl = slice(t, None)
+            tq.tq_quant_gather(inst.h, x, channels[off:off + 64], c["codes"][sl], c["norms"][sl],
+                               signs=c["signs"][sl], rnorms=c["rnorms"][sl], out_stride=cap)
+    torch.cuda.synchronize()
+    for inst, name, chans in ((ia, "a", hi), (ib, "b", lo)):
+        c = caches[name]
+        rows = np.array([h * cap + t for h in range(Hkv) for t in range(steps)])
+        x64 = np.stack([keys[h][t][chans] for h in range(Hkv) for t in range(steps)])
+        sub = {k: v[torch.tensor(rows, device=DEV)] for k, v in c.items()}
+        _check_quant(inst, x64, sub)
+
+
+def _logits_case(B, Hq, Hkv, T, sample, seed=0):
+    scales, hi, lo, ia, ib, channels = _split_instances(seed=seed)
+    rows = B * Hkv * T
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    cache = {}
+    for inst, name in ((ia, "a"), (ib, "b")):
+        cache[name] = dict(
+            codes=torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, inst.h.words), dtype=torch.int32, device=DEV, generator=g),
+            signs=torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, 2), dtype=torch.int32, device=DEV, generator=g),
+            norms=torch.rand(rows, device=DEV, generator=g) + 1,
+            rnorms=torch.rand(rows, device=DEV, generator=g) * 0.3)
+    q64 = bf16_exact(synth.decode_queries(B, Hq, 128, seed=seed))
+    refs = {}
+    for (b, h) in sample:
+        k64 = _split_keys(T, b * Hkv + h, scales, seed)
+        r0 = (b * Hkv + h) * T
+        st = {}
+        for inst, name, chans in ((ia, "a", hi), (ib, "b", lo)):
+            s_ = inst.oracle_quant(k64[:, chans])
+            c = cache[name]
+            c["codes"][r0:r0 + T] = upload_words(oq.pack_codes_vec(s_["idx"], inst.bm))
+            c["signs"][r0:r0 + T] = upload_words(oq.pack_signs(s_["signs"]))
+            c["norms"][r0:r0 + T] = torch.tensor(s_["norms"], device=DEV)
+            c["rnorms"][r0:r0 + T] = torch.tensor(s_["rnorms"], device=DEV)
+            st[name] = s_
+        refs[(b, h)] = (st, k64)
+    q = to_device(q64, torch.bfloat16)
+    logits = torch.empty((B, Hq, T), dtype=torch.float32, device=DEV)
+    scale = 1.0 / math.sqrt(128)
+    tq.tq_attn_logits([ia.h, ib.h], channels, q, Hkv, T, T, [cache["a"]["codes"], cache["b"]["codes"]],
+                      [cache["a"]["signs"], cache["b"]["signs"]], [cache["a"]["norms"], cache["b"]["norms"]],
+                      [cache["a"]["rnorms"], cache["b"]["rnorms"]], scale, logits)
+    torch.cuda.synchronize()
+    got = logits.cpu().numpy()
+    for (b, h), (st, k64) in refs.items():
+        for j in range(4):
+            qv = q64[b, 4 * h + j]
+            ref = np.zeros(T)
+            for inst, name, chans in ((ia, "a", hi), (ib, "b", lo)):
+                s_ = st[name]
+                ref += oq.prod_estimate(qv[chans], s_["idx"], s_["norms"], s_["signs"], s_["rnorms"], inst.Pi_o,
+                                        inst.S, inst.c_o, inst.b)[0]
+            ref *= scale
+            tol = scale * 1e-4 * np.linalg.norm(qv) * np.linalg.norm(k64, axis=1)
+            err = np.abs(got[b, 4 * h + j] - ref)
+            assert np.all(err <= tol), (b, h, j, float(np.max(err / tol)))
+
+
+def test_split_group_logits_small_ragged():
+    _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 0), (1, 1)], seed=1)
+
+
+def test_split_group_logits_full_context_sampled():
+    """Batch 1, 32 q-heads / 8 kv-heads, context 2^20: the full launch, one kv-head checked."""
+    _logits_case(B=1, Hq=32, Hkv=8, T=1 << 20, sample=[(0, 5)], seed=0)
