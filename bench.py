@@ -301,6 +301,74 @@ class Decode:
         return self.B * self.Hkv * self.T
 
 
+class Stream:
+    """Config: batch 1, 32 q-heads / 8 kv-heads, d = 128, context 2^20; keys split
+    into the 64 largest-scale channels at prod 4 bits and 64 at prod 3 bits
+    (3.5 bits per channel).  One step = append one token for every kv-head
+    (per-token quantization of both channel groups) + full-context logits."""
+
+    def __init__(self, tq, torch, rank, dev, T=1 << 20):
+        from_np = lambda a: torch.tensor(a, device=dev)
+        self.tq, self.torch, self.dev = tq, torch, dev
+        self.Hq, self.Hkv, self.T = 32, 8, T
+        scales = synth.lognormal_channel_scales(D, 1.0, 0, 30)
+        order = np.argsort(-scales, kind="stable")
+        hi, lo = np.sort(order[:64]), np.sort(order[64:])
+        self.channels = from_np(np.concatenate([hi, lo]).astype(np.int32))
+        self.h = []
+        for grp, b in ((0, 4), (1, 3)):
+            P = tq.tq_make_rotation(synth.gaussian_matrix(64, 64, 0, synth.ROT_K, grp))
+            S = synth.gaussian_matrix(64, 64, 0, synth.QJL_K, grp)
+            self.h.append(tq.tq_create(64, b, tq.TQ_PROD, P, S))
+        rows = self.Hkv * T
+        self.cache = []
+        for h in self.h:
+            self.cache.append(dict(codes=torch.empty((rows, h.words), dtype=torch.int32, device=dev),
+                                   signs=torch.empty((rows, 2), dtype=torch.int32, device=dev),
+                                   norms=torch.empty(rows, dtype=torch.float32, device=dev),
+                                   rnorms=torch.empty(rows, dtype=torch.float32, device=dev)))
+        g = torch.Generator(device=dev).manual_seed(3000 + rank)
+        sc = torch.tensor(scales, dtype=torch.float32, device=dev)
+        for hh in range(self.Hkv):
+            x = (torch.randn((T, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+            sl = slice(hh * T, (hh + 1) * T)
+            for k, (h, c) in enumerate(zip(self.h, self.cache)):
+                tq.tq_quant_gather(h, x, self.channels[64 * k:64 * (k + 1)], c["codes"][sl], c["norms"][sl],
+                                   signs=c["signs"][sl], rnorms=c["rnorms"][sl])
+        self.token = (torch.randn((self.Hkv, D), generator=g, device=dev) * sc).to(torch.bfloat16)
+        sq = torch.tensor(synth.lognormal_channel_scales(D, 1.0, 0, 20), dtype=torch.float32, device=dev)
+        self.q = (torch.randn((1, self.Hq, D), generator=g, device=dev) * sq).to(torch.bfloat16)
+        self.logits = torch.empty((1, self.Hq, T), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, tq.tq_attn_logits_workspace(self.h, 1, self.Hq)), dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.app, self.lgt = [], []
+
+    def step(self, record=False):
+        tq, torch = self.tq, self.torch
+        E = lambda: torch.cuda.Event(enable_timing=True)
+        if record:
+            e0, e1, e2 = E(), E(), E()
+            e0.record(self.stream)
+        t = self.T - 1  # slot of the arriving token
+        for k, (h, c) in enumerate(zip(self.h, self.cache)):
+            tq.tq_quant_gather(h, self.token, self.channels[64 * k:64 * (k + 1)], c["codes"][t:], c["norms"][t:],
+                               signs=c["signs"][t:], rnorms=c["rnorms"][t:], out_stride=self.T)
+        if record:
+            e1.record(self.stream)
+        tq.tq_attn_logits(self.h, self.channels, self.q, self.Hkv, self.T, self.T,
+                          [c["codes"] for c in self.cache], [c["signs"] for c in self.cache],
+                          [c["norms"] for c in self.cache], [c["rnorms"] for c in self.cache],
+                          1.0 / math.sqrt(D), self.logits, self.ws)
+        if record:
+            e2.record(self.stream)
+            self.app.append((e0, e1))
+            self.lgt.append((e1, e2))
+
+    def bytes_logits(self):
+        # per token per kv-head: group A 24 B codes + 8 B signs + 8 B norms, group B 16 + 8 + 8, logits 4 x 4 B
+        return self.Hkv * self.T * (40 + 32 + 16)
+
+
 # ----------------------------------------------------------------- driver
 
 def run_ours(args):
@@ -410,6 +478,25 @@ def run_ours(args):
                             "ms_per_step": dms, "GBps": gbs, "frac_hbm": gbs / hbm,
                             "bytes_per_step": dl.bytes_per_step(),
                             "config": "B=8, Hq=32, Hkv=8, d=128, T=131072, K prod 4b, V mse 4b"}
+
+    if args.workload == "sweep" and not args.no_decode:
+        torch.cuda.empty_cache()
+        sw = Stream(tq, torch, rank, dev)
+        for _ in range(args.warmup):
+            sw.step()
+        barrier()
+        for _ in range(args.steps):
+            sw.step(record=True)
+        torch.cuda.synchronize()
+        app = max_over_ranks(sum(a.elapsed_time(b) for a, b in sw.app) / len(sw.app))
+        lg = max_over_ranks(sum(a.elapsed_time(b) for a, b in sw.lgt) / len(sw.lgt))
+        gbs = sw.bytes_logits() / (lg / 1e3) / 1e9
+        result["stream"] = {"logits_value": sw.Hkv * sw.T * world / (lg / 1e3), "unit": "keys/s",
+                            "logits_ms": lg, "GBps": gbs, "frac_hbm": gbs / hbm,
+                            "bytes_per_logits_call": sw.bytes_logits(),
+                            "append_us_per_token": app * 1e3,
+                            "config": "B=1, Hq=32, Hkv=8, d=128 split 64 ch @ prod 4b + 64 ch @ prod 3b, T=2^20"}
+        del sw
 
     if rank == 0 and world == 1 and not args.no_cpu:
         if args.workload == "sweep":
