@@ -89,6 +89,32 @@ static double half_value(uint16_t b) {
   return (double)__half2float(h);
 }
 
+// A common scale alpha in [1, 2) (20 fractional bits) for which every scaled
+// centroid alpha c[k] is closest to an fp16 value, relative to its size.  With
+// the scale divided out again in fp32, the fp16 table carries the codebook to
+// about 2e-5 relative for 8 levels and 1e-6 or better for 4 or fewer, instead
+// of the 2^-11 of a plain fp16 rounding.
+static void scaled_half_codebook(tq_ctx* h) {
+  const int K = 1 << h->bm;
+  double mags[8];
+  int nm = 0;
+  for (int k = K / 2; k < K && nm < 8; ++k) mags[nm++] = std::fabs(h->host_centroids[k]);
+  double best = 1e300, best_a = 1.0;
+  for (int i = 0; i < (1 << 20); ++i) {
+    const double a = 1.0 + std::ldexp((double)i, -20);
+    double e = 0.0;
+    for (int m = 0; m < nm && e < best; ++m) {
+      const double v = a * mags[m];
+      if (v == 0.0) continue;
+      e = std::fmax(e, std::fabs(half_value(half_bits(v)) - v) / v);
+    }
+    if (e < best) best = e, best_a = a;
+  }
+  for (int k = 0; k < K; ++k) h->sc_tab[k] = half_bits(best_a * h->host_centroids[k]);
+  h->sc_inv_alpha = (float)(1.0 / best_a);
+  h->sc_rel_err = best;
+}
+
 // Pi^T as fp16 pieces (hi, (Pi - hi) * 2^11) in the swizzled K-major layout:
 // B[i][j] = Pi[j][i], row i, K index j
 static void split_rotation_t_f16(const double* Pi, int d, std::vector<uint16_t>& out) {
@@ -158,6 +184,7 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
       return rc;
     }
   }
+  if (bm <= 3) scaled_half_codebook(h);
   int e = cudaGetDevice(&h->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
   if (e != cudaSuccess) {
@@ -375,7 +402,8 @@ extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* n
 extern "C" size_t tq_ip_scores_workspace(tq_handle h, int64_t nq, int64_t N, int topk) {
   if (!h || nq < 0 || N < 0) return 0;
   size_t bytes = align_up((size_t)nq * h->d * 4, 256) * 2;
-  if (topk > 0) bytes += align_up((size_t)nq * N * 4, 256);
+  if (topk > 0 && !scores_tc_supported(h, topk)) bytes += align_up((size_t)nq * N * 4, 256);
+  if (scores_tc_supported(h, topk)) bytes = std::max(bytes, scores_tc_workspace(h, nq, N, topk));
   return bytes;
 }
 
@@ -402,6 +430,11 @@ extern "C" int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint3
   const size_t need = tq_ip_scores_workspace(h, nq, N, topk);
   if (!workspace || ws_bytes < need)
     return set_error(TQ_EWORKSPACE, "tq_ip_scores: workspace %zu < %zu bytes", ws_bytes, need);
+  if (scores_tc_supported(h, topk)) {
+    int e = launch_scores_tc(h, q, nq, codes, signs, norms, rnorms, N, scores, topk, top_idx, top_val, workspace,
+                             stream);
+    return e ? cuda_error("tq_ip_scores", e) : clear_error();
+  }
   char* ws = (char*)workspace;
   float* qrot = (float*)ws;
   float* qproj = (float*)(ws + align_up((size_t)nq * h->d * 4, 256));

@@ -56,6 +56,12 @@ struct tq_ctx {
   // host copies (float64) kept for diagnostics
   double host_centroids[16] = {0};
   double host_thresholds[15] = {0};
+  // fp16 codebook for the tensor-core scorer: sc_tab[k] = fp16(alpha c[k]) with
+  // one fp32 scale alpha in [1, 2) chosen so the scaled centroids are as close
+  // to fp16 values as possible; products are divided by alpha in fp32
+  uint16_t sc_tab[16] = {0};
+  float sc_inv_alpha = 1.f;
+  double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 
 namespace tqi {
@@ -75,6 +81,11 @@ int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, in
                         int64_t out_stride, void* stream, const int32_t* channels = nullptr);
 int launch_query_prep_gather(const tq_ctx* h, const void* q, int q_dtype, int64_t nq, int dq,
                              const int32_t* channels, float* qrot, float* qproj, void* stream);
+bool scores_tc_supported(const tq_ctx* h, int topk);
+size_t scores_tc_workspace(const tq_ctx* h, int64_t nq, int64_t N, int topk);
+int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t* codes, const uint32_t* signs,
+                     const float* norms, const float* rnorms, int64_t N, float* scores, int topk, int32_t* top_idx,
+                     float* top_val, void* workspace, void* stream);
 bool logits_supported(const tq_ctx* const* hk, int ngroups);
 int launch_logits(const tq_ctx* const* hk, int ngroups, const float* const* qrot, const float* const* qproj, int B,
                   int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* const* kcodes,

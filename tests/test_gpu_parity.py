@@ -367,3 +367,49 @@ def test_split_group_logits_small_ragged():
 def test_split_group_logits_full_context_sampled():
     """Batch 1, 32 q-heads / 8 kv-heads, context 2^20: the full launch, one kv-head checked."""
     _logits_case(B=1, Hq=32, Hkv=8, T=1 << 20, sample=[(0, 5)], seed=0)
+
+
+# ------------------------------------------------------------------ nearest-neighbour search (scores + top-k)
+
+def _search_case(d, b, N, nq, sample, seed=0, with_scores=False, k=10):
+    inst = Instance(d, b, tq.TQ_PROD, seed=seed)
+    x64 = synth.unit_rows(N, d, seed)
+    q64 = synth.unit_rows(nq, d, seed, stream=synth.QUERY)
+    st = inst.oracle_quant(x64)
+    codes = upload_words(oq.pack_codes_vec(st["idx"], inst.bm))
+    signs = upload_words(oq.pack_signs(st["signs"]))
+    norms = torch.tensor(st["norms"], device=DEV)
+    rnorms = torch.tensor(st["rnorms"], device=DEV)
+    q = to_device(q64, torch.float32)
+    ti = torch.empty((nq, k), dtype=torch.int32, device=DEV)
+    tv = torch.empty((nq, k), dtype=torch.float32, device=DEV)
+    scores = torch.empty((nq, N), dtype=torch.float32, device=DEV) if with_scores else None
+    tq.tq_ip_scores(inst.h, q, codes, signs, norms, rnorms, scores=scores, topk=k, top_idx=ti, top_val=tv)
+    torch.cuda.synchronize()
+    ti, tv = ti.cpu().numpy(), tv.cpu().numpy()
+    xh = oq.dequant_mse(st["idx"], st["norms"], inst.Pi_o, inst.c_o)
+    Sx = np.where(st["signs"], 1.0, -1.0)
+    coef = st["rnorms"].astype(np.float64) * math.sqrt(math.pi / 2) / d
+    for r in sample:
+        ref = xh @ q64[r] + coef * (Sx @ (inst.S @ q64[r]))
+        tol = 1e-4 * np.linalg.norm(q64[r]) * np.linalg.norm(x64, axis=1)
+        assert np.all(np.abs(tv[r] - ref[ti[r]]) <= tol[ti[r]]), r
+        assert np.all(np.diff(tv[r]) <= 0) and len(set(ti[r].tolist())) == k
+        rest = np.ones(N, bool)
+        rest[ti[r]] = False
+        assert np.max(ref[rest]) <= tv[r, -1] + 2 * np.max(tol), r
+        if with_scores:
+            err = np.abs(scores[r].cpu().numpy() - ref)
+            assert np.all(err <= tol), (r, float(np.max(err / tol)))
+    return inst
+
+
+def test_search_d200_full_size_sampled():
+    """10^6 unit database vectors (the GloVe shape, d = 200), 10^4 queries, prod 4 bits,
+    top-10 for all queries in one call; 8 queries checked against the exact estimator."""
+    _search_case(200, 4, 1_000_000, 10_000, sample=[0, 1, 777, 4095, 5000, 8191, 9998, 9999])
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_search_d1536_scores_and_topk(b):
+    _search_case(1536, b, 3000, 200, sample=list(range(0, 200, 17)), seed=b, with_scores=True)
