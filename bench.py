@@ -369,6 +369,64 @@ class Stream:
         return self.Hkv * self.T * (40 + 32 + 16)
 
 
+class Search:
+    """Config: N = 10^6 unit-norm fp32 database vectors (Gaussian, normalised),
+    10^4 unit queries, TurboQuant_prod at b total bits, d = 200 or 1536.  One
+    step = quantize the database, then score every (query, vector) pair with a
+    fused top-10 (the full score matrix is not written)."""
+
+    def __init__(self, tq, torch, rank, dev, d=200, b=4, N=10 ** 6, nq=10 ** 4, topk=10):
+        self.tq, self.torch, self.dev = tq, torch, dev
+        self.d, self.b, self.N, self.nq, self.topk = d, b, N, nq, topk
+        P = tq.tq_make_rotation(synth.gaussian_matrix(d, d, 0, synth.ROT_K))
+        S = synth.gaussian_matrix(d, d, 0, synth.QJL_K)
+        self.h = tq.tq_create(d, b, tq.TQ_PROD, P, S)
+        g = torch.Generator(device=dev).manual_seed(4000 + rank)
+        x = torch.randn((N, d), generator=g, device=dev)
+        self.x = x / x.norm(dim=1, keepdim=True)
+        q = torch.randn((nq, d), generator=g, device=dev)
+        self.q = q / q.norm(dim=1, keepdim=True)
+        self.codes = torch.empty((N, self.h.words), dtype=torch.int32, device=dev)
+        self.signs = torch.empty((N, tq.sign_words(d)), dtype=torch.int32, device=dev)
+        self.norms = torch.empty(N, dtype=torch.float32, device=dev)
+        self.rnorms = torch.empty(N, dtype=torch.float32, device=dev)
+        self.ti = torch.empty((nq, topk), dtype=torch.int32, device=dev)
+        self.tv = torch.empty((nq, topk), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, tq.tq_ip_scores_workspace(self.h, nq, N, topk)), dtype=torch.uint8,
+                              device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.quant, self.score = [], []
+
+    def step(self, record=False):
+        tq, torch = self.tq, self.torch
+        E = lambda: torch.cuda.Event(enable_timing=True)
+        if record:
+            e0, e1, e2 = E(), E(), E()
+            e0.record(self.stream)
+        tq.tq_quant_prod(self.h, self.x, self.codes, self.signs, self.norms, self.rnorms)
+        if record:
+            e1.record(self.stream)
+        tq.tq_ip_scores(self.h, self.q, self.codes, self.signs, self.norms, self.rnorms, topk=self.topk,
+                        top_idx=self.ti, top_val=self.tv, workspace=self.ws)
+        if record:
+            e2.record(self.stream)
+            self.quant.append((e0, e1))
+            self.score.append((e1, e2))
+
+    def summary(self, hbm, tc_peak):
+        qms = sum(a.elapsed_time(b) for a, b in self.quant) / len(self.quant)
+        sms = sum(a.elapsed_time(b) for a, b in self.score) / len(self.score)
+        d = self.d
+        q_flop = 2 * 2 * d * d * self.N            # two d x d contractions per vector (rotation, QJL)
+        s_flop = 4 * d * self.N * self.nq          # 2d MACs per pair (codebook part + sign part)
+        return {"quantize_vectors_per_s": self.N / (qms / 1e3), "quantize_ms": qms,
+                "quantize_TFLOPs": q_flop / (qms / 1e3) / 1e12,
+                "score_pairs_per_s": self.N * self.nq / (sms / 1e3), "score_ms": sms,
+                "score_TFLOPs": s_flop / (sms / 1e3) / 1e12,
+                "score_frac_tensor": s_flop / (sms / 1e3) / 1e12 / tc_peak,
+                "config": f"N={self.N} unit fp32, d={d}, nq={self.nq}, prod b={self.b}, fused top-{self.topk}"}
+
+
 # ----------------------------------------------------------------- driver
 
 def run_ours(args):
@@ -498,6 +556,18 @@ def run_ours(args):
                             "config": "B=1, Hq=32, Hkv=8, d=128 split 64 ch @ prod 4b + 64 ch @ prod 3b, T=2^20"}
         del sw
 
+    if args.workload == "sweep" and not args.no_search:
+        torch.cuda.empty_cache()
+        sr = Search(tq, torch, rank, dev, d=args.search_d)
+        for _ in range(args.warmup):
+            sr.step()
+        barrier()
+        for _ in range(max(1, args.steps // 2)):
+            sr.step(record=True)
+        torch.cuda.synchronize()
+        result["search"] = sr.summary(hbm, bf16)
+        del sr
+
     if rank == 0 and world == 1 and not args.no_cpu:
         if args.workload == "sweep":
             rate, dt = oracle_sweep_rate(args.cpu_sample)
@@ -550,6 +620,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-search", action="store_true")
+    ap.add_argument("--search-d", type=int, default=200)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

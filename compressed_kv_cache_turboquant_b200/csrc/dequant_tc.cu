@@ -15,7 +15,11 @@
 //          fp16 pieces up in a 16-entry table and writes them into the
 //          128B-swizzled K-major A tiles (double-buffered)
 //   5..8   epilogue: one thread per vector reads both accumulators from TMEM,
-//          combines, scales by n and stores fp32 or bf16
+//          combines and scales by n; each warp stages its 32 rows x 128 B
+//          column chunk in 128B-swizzled shared memory (two buffers) and
+//          writes it with one TMA tensor store, so global writes are whole
+//          128-byte lines instead of 32 scattered 16-byte pieces per store
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -40,7 +44,9 @@ struct DqShape {
   static constexpr int kStages = 2;
   static constexpr int kTmemCols = (4 * D <= 256) ? 256 : 512;  // 2 buffers x 2 accumulators
   static constexpr int kMiscBytes = 1024;
-  static constexpr int kSmemBytes = 2 * kBBytes + kStages * 2 * kABytes + kMiscBytes + 1024;
+  static constexpr int kStageOut = 32 * 128;  // one warp's output chunk: 32 rows x 128 B
+  static constexpr int kOutBytes = 4 * 2 * kStageOut;
+  static constexpr int kSmemBytes = 2 * kBBytes + kStages * 2 * kABytes + kOutBytes + kMiscBytes + 1024;
 };
 
 struct DqArgs {
@@ -49,20 +55,20 @@ struct DqArgs {
   int64_t N;
   const uint8_t* pit_f16;  // 2 pieces x [slab][row i][128 B swizzled] of Pi^T (B[i][j] = Pi[j][i])
   const uint32_t* lut;     // [16]: fp16 hi | fp16 lo' << 16 of c_k
-  void* out;
   int out_bf16;
   int* status;
 };
 
 template <int D, int BM>
-__global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_constant__ CUtensorMap omap, DqArgs a) {
   using S = DqShape<D>;
   constexpr int W = (D / 32) * BM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* b_s = smem;                      // [2 pieces][kBBytes]
   uint8_t* a_s = smem + 2 * S::kBBytes;     // [stage][2 pieces][kABytes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + S::kStages * 2 * S::kABytes);
+  uint8_t* o_s = a_s + S::kStages * 2 * S::kABytes;  // [4 warps][2][kStageOut], 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_s + S::kOutBytes);
   uint64_t* a_full = bars;              // [2]  decoders -> MMA (count 128)
   uint64_t* a_empty = bars + 2;         // [2]  MMA commit -> decoders
   uint64_t* acc_full = bars + 4;        // [2]  MMA commit -> epilogue
@@ -130,21 +136,14 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
       mma_commit(done_bar);
     }
   } else if (warp <= 4) {
-    // decoders: thread r of the 128 decodes vector r of the tile
+    // decoders: thread r of the 128 decodes vector r of the tile; the codes of
+    // the next tile are loaded while this one is decoded
     const int r = threadIdx.x - 32;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-      const int s = i & 1;
-      const uint32_t u = (uint32_t)(i >> 1);
-      if (!mbar_wait(&a_empty[s], (u & 1u) ^ 1u)) {
-        atomicOr(a.status, kStatusTimeout);
-        break;
-      }
+    auto load_codes = [&](int64_t tile, uint32_t (&w)[W]) {
       const int64_t vec = tile * kTileM + r;
-      uint32_t w[W];
-      if (vec < a.N) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.codes + vec * W);
+      if (tile < ntiles && vec < a.N) {
         if constexpr (W % 4 == 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.codes + vec * W);
 #pragma unroll
           for (int q = 0; q < W / 4; ++q) {
             const uint4 t = src[q];
@@ -157,6 +156,21 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
       } else {
 #pragma unroll
         for (int q = 0; q < W; ++q) w[q] = 0u;
+      }
+    };
+    uint32_t w_next[W];
+    load_codes(blockIdx.x, w_next);
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int s = i & 1;
+      const uint32_t u = (uint32_t)(i >> 1);
+      uint32_t w[W];
+#pragma unroll
+      for (int q = 0; q < W; ++q) w[q] = w_next[q];
+      load_codes(tile + gridDim.x, w_next);
+      if (!mbar_wait(&a_empty[s], (u & 1u) ^ 1u)) {
+        atomicOr(a.status, kStatusTimeout);
+        break;
       }
       uint8_t* hi_tile = a_s + s * 2 * S::kABytes;
       uint8_t* lo_tile = hi_tile + S::kABytes;
@@ -202,58 +216,69 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
     // epilogue: warp % 4 selects the TMEM lane quarter
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    uint8_t* stage = o_s + quarter * 2 * S::kStageOut;
+    constexpr int kCols = 32;  // fp32 columns per 128-byte chunk (bf16: 64)
+    int nst = 0;
     int i = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
+      const int64_t vec = tile * kTileM + r;
+      const int64_t row0 = tile * kTileM + quarter * 32;
+      const float n = (vec < a.N) ? a.norms[vec] : 0.f;  // issued before the wait
       if (!mbar_wait(&acc_full[s], u & 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      const int64_t vec = tile * kTileM + r;
-      const float n = (vec < a.N) ? a.norms[vec] : 0.f;
       const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 2 * D);
+      const int nchunks = a.out_bf16 ? D / 64 : D / 32;
+      for (int c = 0; c < nchunks; ++c, ++nst) {
+        uint8_t* buf = stage + (nst & 1) * S::kStageOut;
+        // the store issued from this buffer two chunks ago must have read it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint32_t pk[32];
+        if (a.out_bf16) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float v0[32], v1[32];
-        tmem_ld32(t0 + c * 32, v0);
-        tmem_ld32(t0 + D + c * 32, v1);
-        tmem_wait_ld();
-        if (vec < a.N) {
-          if (a.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + vec * D + c * 32);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            float v0[32], v1[32];
+            tmem_ld32(t0 + c * 64 + hlf * 32, v0);
+            tmem_ld32(t0 + D + c * 64 + hlf * 32, v1);
+            tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = 8 * q + 2 * e;
-                const float y0 = n * fmaf(v1[j], 4.8828125e-4f, v0[j]);
-                const float y1 = n * fmaf(v1[j + 1], 4.8828125e-4f, v0[j + 1]);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-                pk[e] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              dst[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + vec * D + c * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 o;
-              o.x = n * fmaf(v1[4 * q + 0], 4.8828125e-4f, v0[4 * q + 0]);
-              o.y = n * fmaf(v1[4 * q + 1], 4.8828125e-4f, v0[4 * q + 1]);
-              o.z = n * fmaf(v1[4 * q + 2], 4.8828125e-4f, v0[4 * q + 2]);
-              o.w = n * fmaf(v1[4 * q + 3], 4.8828125e-4f, v0[4 * q + 3]);
-              dst[q] = o;
+            for (int e = 0; e < 16; ++e) {
+              const float y0 = n * fmaf(v1[2 * e], 4.8828125e-4f, v0[2 * e]);
+              const float y1 = n * fmaf(v1[2 * e + 1], 4.8828125e-4f, v0[2 * e + 1]);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+              pk[16 * hlf + e] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
+        } else {
+          float v0[32], v1[32];
+          tmem_ld32(t0 + c * kCols, v0);
+          tmem_ld32(t0 + D + c * kCols, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
+        }
+        // row `lane` of the 128B-swizzled box: 16-byte unit j lands at j ^ (lane & 7)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < a.N) {
+          tma_store_2d(&omap, buf, c * (a.out_bf16 ? 64 : kCols), (int)row0);
+          bulk_commit();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[s]);
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -268,6 +293,19 @@ template <int D, int BM>
 int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_t N, void* out, int out_bf16,
               cudaStream_t stream) {
   using S = DqShape<D>;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return (int)cudaErrorNotSupported;
+  // output as a [N][D] tensor, boxes of 32 rows x 128 bytes
+  CUtensorMap omap;
+  const int esz = out_bf16 ? 2 : 4;
+  const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)N};
+  const cuuint64_t gstride[1] = {(cuuint64_t)D * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&omap, out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, gdim, gstride,
+          box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return (int)cudaErrorInvalidValue;
   auto kern = dequant_tc_kernel<D, BM>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -275,10 +313,10 @@ int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out, out_bf16, h->dev.status};
+  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, h->dev.status};
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);
-  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(a);
+  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(omap, a);
   return (int)cudaGetLastError();
 }
 

@@ -491,21 +491,6 @@ __global__ void topk_merge_kernel(const float* cand_val, const int32_t* cand_idx
   for (int j = 0; j < K; ++j) top_val[q * K + j] = bv[j], top_idx[q * K + j] = bi[j];
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn2() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
 
 }  // namespace
 
@@ -570,7 +555,7 @@ int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t
   if (e) return e;
   qcat_kernel<<<(unsigned)p.nq_pad, 128, 0, s>>>(qrot, qproj, nq, p.nq_pad, h->d, p.d_pad, prod ? 1 : 0, qcat, inv_s);
   if ((e = (int)cudaGetLastError())) return e;
-  EncodeTiledFn enc = encode_fn2();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return (int)cudaErrorNotSupported;
   CUtensorMap map;
   const cuuint64_t gdim[2] = {(cuuint64_t)p.kdim, (cuuint64_t)p.nq_pad};
