@@ -429,31 +429,58 @@ class Search:
 
 # ----------------------------------------------------------------- driver
 
+class Ranks:
+    """One process per GPU, ranks from the torchrun environment.  The path has
+    no exchange step: the only collectives are the barrier around the timed
+    region and the max-over-ranks reduction of its duration."""
+
+    def __init__(self, backend: str = "nccl", device: str | None = None, timeout_s: int = 300):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self.cuda = device is not None and device.startswith("cuda")
+        if self.world > 1 and not dist.is_initialized():
+            from datetime import timedelta
+            kw = {"device_id": torch.device(device)} if self.cuda else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+        if self.cuda:
+            self.torch.cuda.synchronize()
+
+    def close(self):
+        if self.world > 1 and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     import compressed_kv_cache_turboquant_b200 as tq
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = f"cuda:{local}"
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device(dev))
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    max_over_ranks, barrier = ranks.max, ranks.barrier
 
     hbm, bf16, peak_kind = peaks()
     wl_cls = Sweep if args.workload == "sweep" else Decode
@@ -471,7 +498,7 @@ def run_ours(args):
     barrier()
     ms = max_over_ranks(s.elapsed_time(e) / args.steps)
     units = wl.units_per_step() * world
-    value = units / (ms / 1e3)
+    value = job_rate(wl.units_per_step(), world, ms)
 
     if args.workload == "sweep":
         ks = wl.kernel_stats()
@@ -579,8 +606,7 @@ def run_ours(args):
                                   "sample": sample}
     if rank == 0:
         print(json.dumps(result), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def run_reference(args):
