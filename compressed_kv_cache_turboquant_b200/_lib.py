@@ -43,6 +43,8 @@ SIGNATURES = {
     "tq_quant_mse": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _i64, _p]),
     "tq_dequant_mse": (_i, [_p, _p, _p, _i64, _p, _i, _p]),
     "tq_quant_prod": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _i64, _p]),
+    "tq_quant_prod_ws": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _i64, _p, _sz, _p]),
+    "tq_quant_prod_workspace": (_sz, [_p, _i64]),
     "tq_ip_scores": (_i, [_p, _p, _i64, _p, _p, _p, _p, _i64, _p, _i, _p, _p, _p, _sz, _p]),
     "tq_ip_scores_workspace": (_sz, [_p, _i64, _i64, _i]),
     "tq_attn_decode": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,

@@ -17,6 +17,7 @@ from ._lib import (TQ_BF16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQError, check
 __all__ = [
     "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQError", "Handle", "code_words", "sign_words",
     "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
+    "tq_quant_prod_workspace",
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
     "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
 ]
@@ -127,12 +128,24 @@ def tq_dequant_mse(h: Handle, codes: torch.Tensor, norms: torch.Tensor, out: tor
                                                _dtype_code(out), _stream(stream)))
 
 
+def tq_quant_prod_workspace(h: Handle, N: int) -> int:
+    return int(lib.tq_quant_prod_workspace(h.ptr, N))
+
+
 def tq_quant_prod(h: Handle, x: torch.Tensor, codes: torch.Tensor, signs: torch.Tensor,
-                  norms: torch.Tensor, rnorms: torch.Tensor, out_stride: int = 1, stream=None) -> None:
+                  norms: torch.Tensor, rnorms: torch.Tensor, out_stride: int = 1, workspace=None,
+                  stream=None) -> None:
+    """TurboQuant_prod quantization (tq_quant_prod_ws; the workspace, needed only
+    above d = 256, is allocated here when none is passed)."""
     N = x.shape[0]
-    check("tq_quant_prod", lib.tq_quant_prod(h.ptr, _ptr(x), _dtype_code(x), N, x.shape[1], _ptr(codes),
-                                             _ptr(signs), _ptr(norms), _ptr(rnorms), out_stride,
-                                             _stream(stream)))
+    if workspace is None:
+        nbytes = tq_quant_prod_workspace(h, N)
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    check("tq_quant_prod_ws", lib.tq_quant_prod_ws(h.ptr, _ptr(x), _dtype_code(x), N, x.shape[1], _ptr(codes),
+                                                   _ptr(signs), _ptr(norms), _ptr(rnorms), out_stride,
+                                                   _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                                   _stream(stream)))
 
 
 def tq_ip_scores_workspace(h: Handle, nq: int, N: int, topk: int = 0) -> int:

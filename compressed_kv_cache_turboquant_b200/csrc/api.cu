@@ -3,6 +3,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -195,6 +196,7 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   // host staging of every constant (float32), then one upload
   const size_t dd = (size_t)d * d;
   std::vector<float> Pf(dd), PTf(dd), Sf, TTf;
+  std::vector<double> Td;
   for (int j = 0; j < d; ++j)
     for (int i = 0; i < d; ++i) {
       Pf[(size_t)j * d + i] = (float)Pi[(size_t)j * d + i];
@@ -205,14 +207,36 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
     TTf.resize(dd);
     for (size_t k = 0; k < dd; ++k) Sf[k] = (float)S[k];
     // T = S Pi^T in float64: T[j][i] = sum_k S[j][k] Pi[i][k]; stored as TT[i][j]
-    std::vector<double> row(d);
+    Td.resize(dd);
     for (int j = 0; j < d; ++j)
       for (int i = 0; i < d; ++i) {
         double acc = 0.0;
         const double* s = S + (size_t)j * d;
         const double* p = Pi + (size_t)i * d;
         for (int k = 0; k < d; ++k) acc += s[k] * p[k];
+        Td[(size_t)j * d + i] = acc;
         TTf[(size_t)i * d + j] = (float)acc;
+      }
+  }
+  // general-d quantizer pieces (hi, lo * 2^11) of Pi and of [S | T]
+  const int dp = (d + 127) / 128 * 128;
+  h->gen_d_pad = dp;
+  std::vector<uint16_t> gpi((size_t)2 * dp * dp, 0), gst;
+  auto split_into = [&](double v, uint16_t* hi, uint16_t* lo) {
+    const uint16_t hb = half_bits(v);
+    *hi = hb;
+    *lo = half_bits((v - half_value(hb)) * 2048.0);
+  };
+  for (int n = 0; n < d; ++n)
+    for (int k = 0; k < d; ++k)
+      split_into(Pi[(size_t)n * d + k], &gpi[(size_t)n * dp + k], &gpi[((size_t)dp + n) * dp + k]);
+  if (variant == TQ_PROD) {
+    const size_t w2 = (size_t)2 * dp;
+    gst.assign(2 * (size_t)dp * w2, 0);
+    for (int n = 0; n < d; ++n)
+      for (int k = 0; k < d; ++k) {
+        split_into(S[(size_t)n * d + k], &gst[(size_t)n * w2 + k], &gst[((size_t)dp + n) * w2 + k]);
+        split_into(Td[(size_t)n * d + k], &gst[(size_t)n * w2 + dp + k], &gst[((size_t)dp + n) * w2 + dp + k]);
       }
   }
   std::vector<float> cf(K), tf(K);
@@ -266,6 +290,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (has_ktab) byte_table(h->host_centroids, ktab);
   if (has_vtab) byte_table(h->host_centroids + 8, vtab);
   const size_t oTabs = take(8 * 4);
+  const size_t oGenPi = take(gpi.size() * 2);
+  const size_t oGenSt = gst.empty() ? 0 : take(gst.size() * 2);
   h->block_bytes = off;
   e = cudaMalloc(&h->block, h->block_bytes);
   if (e != cudaSuccess) {
@@ -281,6 +307,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (tc) h->dev.pi_tc = (uint8_t*)(base + oPiTc);
   if (tc) h->dev.pit_f16 = (uint8_t*)(base + oPitF16);
   h->dev.lut_dq = (uint32_t*)(base + oLut);
+  h->dev.gen_pi = (uint16_t*)(base + oGenPi);
+  if (!gst.empty()) h->dev.gen_st = (uint16_t*)(base + oGenSt);
   if (has_ktab) h->dev.ktab = (uint32_t*)(base + oTabs);
   if (has_vtab) h->dev.vtab = (uint32_t*)(base + oTabs + 16);
   if (variant == TQ_PROD) {
@@ -300,6 +328,9 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess) e = cudaMemcpy(h->dev.lut_dq, lut.data(), 16 * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(base + oTabs, ktab, 16, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(base + oTabs + 16, vtab, 16, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->dev.gen_pi, gpi.data(), gpi.size() * 2, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !gst.empty())
+    e = cudaMemcpy(h->dev.gen_st, gst.data(), gst.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && variant == TQ_PROD) {
     e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
@@ -364,21 +395,55 @@ extern "C" int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, in
   if (N == 0) return clear_error();
   int e = quant_tc_supported(h, dtype)
               ? launch_quant_mse_tc(h, x, N, x_stride, codes, norms, out_stride, stream)
+          : quant_gen_supported(h)
+              ? launch_quant_gen(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, nullptr, 0,
+                                 stream)
               : launch_quant_simple(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream);
   return e ? cuda_error("tq_quant_mse", e) : clear_error();
+}
+
+static int quant_prod_impl(const char* fn, tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                           uint32_t* codes, uint32_t* signs, float* norms, float* rnorms, int64_t out_stride,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_quant_args(fn, h, TQ_PROD, x, dtype, N, x_stride, codes, norms, out_stride);
+  if (rc) return rc;
+  if (N > 0 && (!signs || !rnorms)) return set_error(TQ_EINVAL, "%s: NULL pointer", fn);
+  TQ_CHECK_ALIGN(signs, "signs");
+  TQ_CHECK_ALIGN(rnorms, "rnorms");
+  TQ_CHECK_ALIGN(workspace, "workspace");
+  if (N == 0) return clear_error();
+  const bool need_ws = quant_gen_supported(h) && quant_gen_needs_workspace(h);
+  if (need_ws && workspace && ws_bytes < (size_t)128 * quant_gen_workspace_rows_bytes(h))
+    return set_error(TQ_EWORKSPACE, "%s: workspace of %zu bytes is below the %zu-byte minimum", fn, ws_bytes,
+                     (size_t)128 * quant_gen_workspace_rows_bytes(h));
+  // tensor cores unless this d needs the residual workspace and none was given
+  const bool gen = quant_gen_supported(h) && (!need_ws || workspace);
+  int e = gen ? launch_quant_gen(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, workspace,
+                                 ws_bytes, stream)
+              : launch_quant_simple(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream);
+  return e ? cuda_error(fn, e) : clear_error();
 }
 
 extern "C" int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                              uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
                              int64_t out_stride, void* stream) {
-  int rc = check_quant_args("tq_quant_prod", h, TQ_PROD, x, dtype, N, x_stride, codes, norms, out_stride);
-  if (rc) return rc;
-  if (N > 0 && (!signs || !rnorms)) return set_error(TQ_EINVAL, "tq_quant_prod: NULL pointer");
-  TQ_CHECK_ALIGN(signs, "signs");
-  TQ_CHECK_ALIGN(rnorms, "rnorms");
-  if (N == 0) return clear_error();
-  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream);
-  return e ? cuda_error("tq_quant_prod", e) : clear_error();
+  return quant_prod_impl("tq_quant_prod", h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride,
+                         nullptr, 0, stream);
+}
+
+extern "C" int tq_quant_prod_ws(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                                uint32_t* codes, uint32_t* signs, float* norms, float* rnorms, int64_t out_stride,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return quant_prod_impl("tq_quant_prod_ws", h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride,
+                         workspace, ws_bytes, stream);
+}
+
+extern "C" size_t tq_quant_prod_workspace(tq_handle h, int64_t N) {
+  if (!h || N <= 0 || h->variant != TQ_PROD || !quant_gen_supported(h) || !quant_gen_needs_workspace(h)) return 0;
+  // whole 128-row tiles, at most four per SM per launch
+  const int64_t cap = (int64_t)4 * h->sm_count * 128;
+  const int64_t rows = std::min((N + 127) / 128 * 128, cap);
+  return (size_t)rows * quant_gen_workspace_rows_bytes(h);
 }
 
 extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* norms, int64_t N,

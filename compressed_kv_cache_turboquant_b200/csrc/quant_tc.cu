@@ -23,6 +23,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
+
 #include "sm100_common.cuh"
 #include "tq_internal.h"
 
@@ -263,7 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float n = sqrtf(np[row] + np[128 + row]);
 #pragma unroll
-      for (int m = 1; m < (1 << (BM - 1)); ++m) P[m] = n * thr_s[(1 << (BM - 1)) - 1 + m];
+      // a zero vector has y = 0, which lies below every positive threshold
+      for (int m = 1; m < (1 << (BM - 1)); ++m) P[m] = n > 0.f ? n * thr_s[(1 << (BM - 1)) - 1 + m] : INFINITY;
       const int64_t vec = tile * kTileM + row;
       if (vec < a.N) {
         uint32_t* dst = a.codes + vec * a.out_stride * W + half * GH * BM;

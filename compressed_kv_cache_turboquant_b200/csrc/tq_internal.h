@@ -42,6 +42,12 @@ struct DevConsts {
   // vtab (4-bit symmetric codebooks): the same for the upper half c8..c15
   uint32_t* ktab = nullptr;
   uint32_t* vtab = nullptr;
+  // general-d quantizer operands, fp16 row-major, d_pad = d rounded up to 128,
+  // zero padded: gen_pi = [hi; lo * 2^11] of Pi as [2 d_pad][d_pad] (row = output
+  // coordinate, column = input coordinate); gen_st (prod) = [hi; lo * 2^11] of
+  // [S | T] as [2 d_pad][2 d_pad]
+  uint16_t* gen_pi = nullptr;
+  uint16_t* gen_st = nullptr;
 };
 
 }  // namespace tqi
@@ -61,6 +67,7 @@ struct tq_ctx {
   // to fp16 values as possible; products are divided by alpha in fp32
   uint16_t sc_tab[16] = {0};
   float sc_inv_alpha = 1.f;
+  int gen_d_pad = 0;
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 
@@ -81,6 +88,12 @@ int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, in
                         int64_t out_stride, void* stream, const int32_t* channels = nullptr);
 int launch_query_prep_gather(const tq_ctx* h, const void* q, int q_dtype, int64_t nq, int dq,
                              const int32_t* channels, float* qrot, float* qproj, void* stream);
+bool quant_gen_supported(const tq_ctx* h);
+bool quant_gen_needs_workspace(const tq_ctx* h);
+size_t quant_gen_workspace_rows_bytes(const tq_ctx* h);
+int launch_quant_gen(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
+                     uint32_t* signs, float* norms, float* rnorms, int64_t out_stride, void* workspace,
+                     size_t ws_bytes, void* stream);
 bool scores_tc_supported(const tq_ctx* h, int topk);
 size_t scores_tc_workspace(const tq_ctx* h, int64_t nq, int64_t N, int topk);
 int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t* codes, const uint32_t* signs,

@@ -191,6 +191,27 @@ TQ_API int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, int64
                   void* stream);
 
 /*
+ * tq_quant_prod_ws -- tq_quant_prod with a caller workspace (same outputs,
+ * same passages).  For dimensions above 256 the tensor-core path computes the
+ * QJL projection from the stored residual u = y - c[idx] (two fp16 pieces per
+ * coordinate, 4 d_pad bytes per vector, d_pad = d rounded up to 128) so that
+ * its fp32 sums stay of size ||u|| rather than ||x||; the workspace holds those
+ * rows for up to ws_bytes / (4 d_pad) vectors (whole multiples of 128) at a
+ * time and the call walks the batch in such chunks.  tq_quant_prod without a
+ * workspace runs those dimensions on the CUDA cores instead.
+ *   workspace, ws_bytes   dev scratch; tq_quant_prod_workspace(h, N) bytes run
+ *            the batch in the fewest launches; any size of at least 512 d_pad
+ *            bytes (128 vectors) is accepted; ignored (may be NULL) for d <= 256
+ * Errors: as tq_quant_prod, plus TQ_EWORKSPACE (a non-NULL workspace below the
+ * minimum).
+ */
+TQ_API int tq_quant_prod_ws(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
+                     uint32_t* codes, uint32_t* signs, float* norms, float* rnorms, int64_t out_stride,
+                     void* workspace, size_t ws_bytes, void* stream);
+/* Suggested workspace bytes for tq_quant_prod_ws (0 when none is used). */
+TQ_API size_t tq_quant_prod_workspace(tq_handle h, int64_t N);
+
+/*
  * tq_ip_scores -- estimated inner products of nq queries with N quantized vectors
  * ([tmdm, "双剑合璧", ✦ QJL]: the unbiased estimator corrects the quantization error
  * while the score is computed; [admirer, "內存價格能下來嗎？": nearest-neighbour search).

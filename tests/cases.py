@@ -90,14 +90,22 @@ def compare_codes(gpu_words: np.ndarray, idx: np.ndarray, y_unit: np.ndarray, th
     return rows_exact, int(excused.sum())
 
 
-def compare_signs(gpu_words: np.ndarray, bits: np.ndarray, Sr: np.ndarray, rn: np.ndarray, rows: np.ndarray):
-    """QJL sign bits on rows whose mse codes match; a bit is excused where
-    |(S r)_j| <= 1e-5 ||r||."""
-    excused = np.abs(Sr) <= 1e-5 * np.asarray(rn, dtype=np.float64)[:, None]
+def compare_signs(gpu_words: np.ndarray, bits: np.ndarray, Sr: np.ndarray, n: np.ndarray, rows: np.ndarray,
+                  check_fraction: bool = True):
+    """QJL sign bits on rows whose mse codes match, bit-exact except where the
+    projected residual lies within 1e-5 of zero in the unit frame of x:
+    |(S r)_j| <= 1e-5 ||x||.  (The code band is 1e-5/sqrt(d) on y = Pi x/||x||;
+    with S's rows normalised to unit length, (S r)_j / (sqrt(d) ||x||) is the
+    same kind of coordinate, so its band is 1e-5/sqrt(d) on that value.)  At
+    most 1e-4 of the compared bits may fall in the band."""
+    excused = np.abs(Sr) <= 1e-5 * np.asarray(n, dtype=np.float64)[:, None]
+    if check_fraction and excused[rows].size >= 200000:
+        assert excused[rows].sum() <= 1e-4 * excused[rows].size, f"{excused[rows].sum()} excused sign bits"
     mask = oq.pack_codes_vec(excused.astype(np.int64), 1)
     expect = oq.pack_codes_vec(bits.astype(np.int64), 1)
-    diff = ((gpu_words ^ expect) & ~mask)[rows]
-    bad = np.argwhere(diff != 0)
+    diff = (gpu_words ^ expect) & ~mask
+    diff[~np.asarray(rows)] = 0
+    bad = np.argwhere(diff != 0)  # (row, word) in the caller's numbering
     assert len(bad) == 0, f"{len(bad)} sign words differ, first at {bad[:5]}"
 
 

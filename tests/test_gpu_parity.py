@@ -3,7 +3,8 @@
 Codes: bit-exact except coordinates whose oracle rotated value lies within
 1e-5/sqrt(d) of a decision threshold (at most 1e-4 of all coordinates).
 QJL signs: bit-exact on vectors whose mse codes match, except |(S r)_j| <=
-1e-5 ||r||.  Reconstructions: relative L2 <= 1e-5.  Scores: |delta| <=
+1e-5 ||x|| (the same 1e-5/sqrt(d) band in the unit frame of x, with S's rows
+normalised to unit length).  Reconstructions: relative L2 <= 1e-5.  Scores: |delta| <=
 1e-4 ||q|| ||k|| against the oracle estimator on the same (oracle) codes.
 """
 import math
@@ -34,7 +35,7 @@ def _check_quant(inst: Instance, x64: np.ndarray, out: dict, rows=None):
     norms = out["norms"].cpu().numpy()[rows]
     assert np.max(rel_err(norms, ref["norms"])) <= NORM_RTOL
     if inst.prod:
-        compare_signs(words_u32(out["signs"])[rows], ref["signs"], ref["Sr"], ref["rnorms"], exact)
+        compare_signs(words_u32(out["signs"])[rows], ref["signs"], ref["Sr"], ref["norms"], exact)
         rn = out["rnorms"].cpu().numpy()[rows]
         assert np.max(rel_err(rn[exact], ref["rnorms"][exact])) <= NORM_RTOL
     return ref, exact
@@ -107,6 +108,67 @@ def test_zero_vectors_strides_and_slots():
     # untouched slots stay zero
     other = out["codes"].view(N, slots, -1)[:, 1:]
     assert int(other.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("d", [64, 128, 200])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("variant,b", [(tq.TQ_MSE, 3), (tq.TQ_PROD, 4)])
+def test_zero_vectors_every_path(d, dtype, variant, b):
+    """Zero rows among ordinary ones: y := 0 takes the cell above the middle
+    threshold, x_hat = 0, every QJL bit set, rn = 0 (every quantizer path)."""
+    N = 300
+    inst = Instance(d, b, variant, seed=11)
+    x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=11)
+    zero = [0, 1, 150, 299]
+    x64[zero] = 0.0
+    if dtype == torch.bfloat16:
+        x64 = bf16_exact(x64)
+    out = inst.alloc_outputs(N)
+    inst.gpu_quant(to_device(x64, dtype), out)
+    torch.cuda.synchronize()
+    _check_quant(inst, x64, out)
+    assert np.all(out["norms"].cpu().numpy()[zero] == 0)
+
+
+def test_prod_many_row_tiles_per_cta():
+    """40000 fp32 vectors at d = 200: several 128-vector tiles per persistent CTA."""
+    d, N = 200, 40000
+    inst = Instance(d, 3, tq.TQ_PROD, seed=21)
+    x64 = synth.scaled_gaussian_rows(N, d, 0.5, seed=21)
+    out = inst.alloc_outputs(N)
+    inst.gpu_quant(to_device(x64, torch.float32), out)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([synth.rng(21, 1).choice(N, 2000, replace=False), np.arange(N - 130, N)]))
+    _check_quant(inst, x64, out, rows)
+
+
+def test_prod_d1536_workspace_chunks_and_no_workspace():
+    """d = 1536: a workspace of exactly 128 rows walks 300 vectors in three
+    chunks and gives the same words as one launch; without a workspace the C
+    call runs the CUDA-core path; both match the oracle."""
+    from compressed_kv_cache_turboquant_b200._lib import lib
+    from compressed_kv_cache_turboquant_b200.api import _ptr
+    d, N = 1536, 300
+    inst = Instance(d, 3, tq.TQ_PROD, seed=4)
+    x64 = synth.unit_rows(N, d, 4)
+    x = to_device(x64, torch.float32)
+    full, small, none = inst.alloc_outputs(N), inst.alloc_outputs(N), inst.alloc_outputs(N)
+    inst.gpu_quant(x, full)
+    row_bytes = tq.tq_quant_prod_workspace(inst.h, 1) // 128
+    ws = torch.empty(128 * row_bytes, dtype=torch.uint8, device=DEV)
+    tq.tq_quant_prod(inst.h, x, small["codes"], small["signs"], small["norms"], small["rnorms"], workspace=ws)
+    rc = lib.tq_quant_prod(inst.h.ptr, _ptr(x), tq.TQ_F32, N, d, _ptr(none["codes"]), _ptr(none["signs"]),
+                           _ptr(none["norms"]), _ptr(none["rnorms"]), 1, None)
+    assert rc == 0
+    torch.cuda.synchronize()
+    for k in full:
+        assert torch.equal(full[k], small[k]), k
+    _check_quant(inst, x64, full)
+    _check_quant(inst, x64, none)
+    # a workspace below one 128-row tile is refused
+    with pytest.raises(tq.TQError):
+        tq.tq_quant_prod(inst.h, x, small["codes"], small["signs"], small["norms"], small["rnorms"],
+                         workspace=ws[: 127 * row_bytes])
 
 
 def test_fp32_d1536_prod_sampled():
