@@ -14,9 +14,11 @@
 // 128 queries x TN keys is therefore a GEMM with fp32 accumulators in TMEM, one
 // for the codebook part and (TurboQuant_prod) one for the sign part, and the
 // per-key factors n / alpha and rn sqrt(pi/2)/d are applied in fp32 in the
-// epilogue.  The query side is split as q s = hi + lo (two fp16 pieces, s a
-// power of two per query) and both pieces multiply the same decoded key chunk,
-// so the products carry the query to about 2^-22.
+// epilogue.  The query side of the codebook part is split as q' s = hi + lo
+// (two fp16 pieces, s a power of two per query) and both pieces multiply the
+// same decoded key chunk, so those products carry the query to about 2^-22;
+// the sign part (a term of size ~||r|| ||q|| / sqrt(d)) takes q'' s in one fp16
+// piece, whose rounding stays below 2e-5 of the score bound.
 //
 // Persistent CTAs walk (query tile, key tile) work items in query-tile-major
 // order; the epilogue keeps a running top-k per query (k <= 16) and writes
@@ -24,8 +26,11 @@
 // of the CTAs that covered a query tile.
 //   warp 0      TMA producer of query chunks [128 x 64] fp16 (hi and lo)
 //   warp 1      TMEM allocation and the MMA issuer
-//   warps 2-5   decoders: TN / 128 keys per thread per 64-coordinate chunk
-//   warps 6-9   epilogue: one thread per query row
+//   warps 2-9   decoders: 256 threads, one (key, 32-coordinate group) pair
+//               each (prod: 128 keys x 2 groups; mse: 256 keys x both groups);
+//               each thread stages its own packed words for the chunks ahead in
+//               a shared-memory ring with 4-byte asynchronous copies
+//   warps 10-13 epilogue: one thread per query row
 // Tiles: TurboQuant_mse 128 x 256 with one accumulator, TurboQuant_prod
 // 128 x 128 with two; either way two accumulator sets (512 TMEM columns) let the
 // epilogue of one tile overlap the MMAs of the next.
@@ -47,7 +52,7 @@ constexpr int kTM = 128;          // queries per tile
 constexpr int kAStages = 4;
 constexpr int kABytes = kTM * 128;  // one 64-wide fp16 chunk of the query tile
 constexpr int kTabBytes = 32768;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kKMax = 16;          // largest fused top-k
 // per-key factor buffers: the decoders start item j only after the MMA issuer
 // has released all but kBStages chunks of item j-1, and the issuer is at most
@@ -59,9 +64,14 @@ template <bool PROD>
 struct Tile {
   static constexpr int TN = PROD ? 128 : 256;       // keys per tile
   static constexpr int KPT = TN / 128;              // keys per decoder thread
-  static constexpr int BStages = PROD ? 4 : 2;
+  static constexpr int BStages = PROD ? 3 : 2;
   static constexpr int BBytes = TN * 128;           // one 64-wide fp16 chunk of the key tile
-  static constexpr int Smem = kAStages * kABytes + BStages * BBytes + 2 * kTabBytes + kMkBufs * TN * 8 + 512 + 1024;
+  static constexpr int Tabs = PROD ? 2 : 1;         // codebook table (+ sign table)
+  static constexpr int Ring = PROD ? 8 : 4;         // staged chunks ahead per decoder thread
+  static constexpr int RingWords = 8;               // words staged per key per chunk (4 per group)
+  static constexpr int RingBytes = Ring * TN * RingWords * 4;
+  static constexpr int Smem = kAStages * kABytes + BStages * BBytes + Tabs * kTabBytes + kMkBufs * TN * 8 +
+                              RingBytes + 512 + 1024;
 };
 
 struct ScArgs {
@@ -90,70 +100,68 @@ __device__ __forceinline__ uint32_t ctab_at(const ScArgs& a, uint32_t k) {
   return (a.ctab[k >> 1] >> (16 * (k & 1u))) & 0xFFFFu;
 }
 
-// 64 coordinates of one key (two groups of 32) -> 32 fp16 pairs (coordinate
-// order) of the scaled codebook
-__device__ __forceinline__ void decode_mse64(const uint32_t* w /*2*bm words*/, int bm, bool g1_valid,
-                                             const uint8_t* tab, int lane, uint32_t (&h)[32]) {
+// one group of 32 coordinates (BM words) -> 16 fp16 pairs (coordinate order)
+// of the scaled codebook, by byte-indexed lookups in per-lane table copies
+template <int BM>
+__device__ __forceinline__ void decode_mse32(const uint32_t* p, const uint8_t* tab, int lane, uint32_t (&o)[16]) {
+  if constexpr (BM == 3) {
+    const uint32_t s3 = ((p[0] >> 3) & 0x11111111u) | ((p[1] >> 2) & 0x22222222u) | ((p[2] >> 1) & 0x44444444u);
+    const uint32_t ws[4] = {p[0], p[1], p[2], s3};
 #pragma unroll
-  for (int gg = 0; gg < 2; ++gg) {
-    if (gg == 1 && !g1_valid) {
+    for (int q = 0; q < 4; ++q)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) h[16 + i] = 0u;
-      break;
-    }
-    const uint32_t* p = w + gg * bm;
-    uint32_t* o = h + 16 * gg;
-    if (bm == 3) {
-      const uint32_t s3 = ((p[0] >> 3) & 0x11111111u) | ((p[1] >> 2) & 0x22222222u) | ((p[2] >> 1) & 0x44444444u);
-      const uint32_t ws[4] = {p[0], p[1], p[2], s3};
+      for (int i = 0; i < 4; ++i)
+        o[4 * q + i] = *reinterpret_cast<const uint32_t*>(tab + ((ws[q] >> (8 * i)) & 0xFFu) * 128 + lane * 4);
+  } else if constexpr (BM == 2) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          o[4 * q + i] = *reinterpret_cast<const uint32_t*>(tab + ((ws[q] >> (8 * i)) & 0xFFu) * 128 + lane * 4);
-    } else if (bm == 2) {
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint2 v = *reinterpret_cast<const uint2*>(tab + ((p[k] >> (8 * i)) & 0xFFu) * 128 + (lane & 15) * 8);
-          o[8 * k + 2 * i] = v.x;
-          o[8 * k + 2 * i + 1] = v.y;
-        }
-    } else {
+    for (int k = 0; k < 2; ++k)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4*>(tab + ((p[0] >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
-        o[4 * i + 0] = v.x;
-        o[4 * i + 1] = v.y;
-        o[4 * i + 2] = v.z;
-        o[4 * i + 3] = v.w;
+        const uint2 v = *reinterpret_cast<const uint2*>(tab + ((p[k] >> (8 * i)) & 0xFFu) * 128 + (lane & 15) * 8);
+        o[8 * k + 2 * i] = v.x;
+        o[8 * k + 2 * i + 1] = v.y;
       }
-    }
-  }
-}
-
-// 64 sign bits -> 32 fp16 pairs of +-1
-__device__ __forceinline__ void decode_sign64(const uint32_t* s /*2 words*/, bool g1_valid, const uint8_t* tab,
-                                              int lane, uint32_t (&h)[32]) {
-#pragma unroll
-  for (int gg = 0; gg < 2; ++gg) {
+  } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      if (gg == 1 && !g1_valid) {
-        h[16 * gg + 4 * i + 0] = h[16 * gg + 4 * i + 1] = h[16 * gg + 4 * i + 2] = h[16 * gg + 4 * i + 3] = 0u;
-        continue;
-      }
-      const uint4 v = *reinterpret_cast<const uint4*>(tab + ((s[gg] >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
-      h[16 * gg + 4 * i + 0] = v.x;
-      h[16 * gg + 4 * i + 1] = v.y;
-      h[16 * gg + 4 * i + 2] = v.z;
-      h[16 * gg + 4 * i + 3] = v.w;
+      const uint4 v = *reinterpret_cast<const uint4*>(tab + ((p[0] >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
+      o[4 * i + 0] = v.x;
+      o[4 * i + 1] = v.y;
+      o[4 * i + 2] = v.z;
+      o[4 * i + 3] = v.w;
     }
   }
 }
 
-template <bool PROD>
+// 32 sign bits -> 16 fp16 pairs of +-1
+__device__ __forceinline__ void decode_sign32(uint32_t sw, const uint8_t* tab, int lane, uint32_t (&o)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(tab + ((sw >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
+    o[4 * i + 0] = v.x;
+    o[4 * i + 1] = v.y;
+    o[4 * i + 2] = v.z;
+    o[4 * i + 3] = v.w;
+  }
+}
+
+// Insert (s, key) into the descending top-K list (bv, bi) of one query row
+// (s > bv[K-1] on entry); an equal score stays behind the earlier, lower key.
+// Rare after the first keys, so kept out of line: the unrolled epilogue only
+// compares against the returned new k-th value.
+__device__ __noinline__ float topk_insert(float* bv, int32_t* bi, int K, float s, int32_t key) {
+  int j = K - 1;
+  while (j > 0 && bv[j - 1] < s) {
+    bv[j] = bv[j - 1];
+    bi[j] = bi[j - 1];
+    --j;
+  }
+  bv[j] = s;
+  bi[j] = key;
+  return bv[K - 1];
+}
+
+template <bool PROD, int BM>
 __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ CUtensorMap qmap, ScArgs a) {
   using T = Tile<PROD>;
   constexpr int TN = T::TN, KPT = T::KPT, kBStages = T::BStages, kBBytes = T::BBytes;
@@ -162,11 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
   uint8_t* a_s = smem;                                  // [kAStages][kABytes]
   uint8_t* b_s = a_s + kAStages * kABytes;              // [kBStages][kBBytes]
   uint8_t* mtab = b_s + kBStages * kBBytes;             // codebook table (layout by bm)
-  uint8_t* stab = mtab + kTabBytes;                     // sign table
+  uint8_t* stab = mtab + kTabBytes;                     // sign table (prod)
   // per-key factors of each work item: n / alpha (negative = no key) and rn sqrt(pi/2)/d
-  float* mk_s = reinterpret_cast<float*>(stab + kTabBytes);  // [kMkBufs][TN]
-  float* qk_s = mk_s + kMkBufs * TN;                         // [kMkBufs][TN]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qk_s + kMkBufs * TN);
+  float* mk_s = reinterpret_cast<float*>(mtab + T::Tabs * kTabBytes);  // [kMkBufs][TN]
+  float* qk_s = mk_s + kMkBufs * TN;                                   // [kMkBufs][TN]
+  uint32_t* ring_s = reinterpret_cast<uint32_t*>(qk_s + kMkBufs * TN); // [Ring][TN][RingWords]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_s + T::Ring * TN * T::RingWords);
   uint64_t* a_full = bars;                 // [kAStages]
   uint64_t* a_empty = a_full + kAStages;   // [kAStages]
   uint64_t* b_full = a_empty + kAStages;   // [kBStages] count 128
@@ -184,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAStages; ++s) mbar_init(&a_full[s], 1), mbar_init(&a_empty[s], 1);
-    for (int s = 0; s < kBStages; ++s) mbar_init(&b_full[s], 128), mbar_init(&b_empty[s], 1);
+    for (int s = 0; s < kBStages; ++s) mbar_init(&b_full[s], 256), mbar_init(&b_empty[s], 1);
     for (int s = 0; s < 2; ++s) mbar_init(&acc_full[s], 1), mbar_init(&acc_empty[s], 128);
     mbar_init(done_bar, 1);
     fence_mbar_init();
@@ -193,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
   for (int w = threadIdx.x; w < kTabBytes / 4; w += blockDim.x) {
     const uint32_t row = (uint32_t)w >> 5, col = (uint32_t)w & 31u;
     uint32_t v;
-    if (a.bm == 3) {
+    if (BM == 3) {
       v = ctab_at(a, row & 7u) | (ctab_at(a, (row >> 4) & 7u) << 16);
-    } else if (a.bm == 2) {  // 16 copies of 2 pairs (4 two-bit codes)
+    } else if (BM == 2) {  // 16 copies of 2 pairs (4 two-bit codes)
       const uint32_t pr = col & 1u, i0 = (row >> (4 * pr)) & 3u, i1 = (row >> (4 * pr + 2)) & 3u;
       v = ctab_at(a, i0) | (ctab_at(a, i1) << 16);
     } else {  // 8 copies of 4 pairs (8 one-bit codes)
@@ -203,9 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
       v = ctab_at(a, i0) | (ctab_at(a, i1) << 16);
     }
     reinterpret_cast<uint32_t*>(mtab)[w] = v;
-    const uint32_t pr = col & 3u;
-    const uint32_t lo = ((row >> (2 * pr)) & 1u) ? 0x3C00u : 0xBC00u, hi = ((row >> (2 * pr + 1)) & 1u) ? 0x3C00u : 0xBC00u;
-    reinterpret_cast<uint32_t*>(stab)[w] = lo | (hi << 16);
+    if (PROD) {
+      const uint32_t pr = col & 3u;
+      const uint32_t lo = ((row >> (2 * pr)) & 1u) ? 0x3C00u : 0xBC00u;
+      const uint32_t hi = ((row >> (2 * pr + 1)) & 1u) ? 0x3C00u : 0xBC00u;
+      reinterpret_cast<uint32_t*>(stab)[w] = lo | (hi << 16);
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -215,21 +227,24 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
 
   if (warp == 0) {
     if (lane == 0) {
-      // per key chunk kc: the hi query chunk kc, then the lo chunk nkc + kc
+      // per key chunk kc: the hi query chunk kc, then (codebook part) the lo chunk nkc + kc
       int64_t ch = 0;
-      for (int64_t it = it_lo; it < it_hi; ++it) {
+      bool ok = true;
+      for (int64_t it = it_lo; ok && it < it_hi; ++it) {
         const int64_t qt = it / a.kt_count;
-        for (int kc = 0; kc < 2 * nkc; ++kc, ++ch) {
-          const int s = (int)(ch % kAStages);
-          const uint32_t u = (uint32_t)(ch / kAStages);
-          if (!mbar_wait(&a_empty[s], (u & 1u) ^ 1u)) {
-            atomicOr(a.status, kStatusTimeout);
-            it = it_hi;
-            break;
+        for (int kc = 0; ok && kc < nkc; ++kc) {
+          for (int piece = 0; piece < (kc < nkc_m ? 2 : 1); ++piece, ++ch) {
+            const int s = (int)(ch % kAStages);
+            const uint32_t u = (uint32_t)(ch / kAStages);
+            if (!mbar_wait(&a_empty[s], (u & 1u) ^ 1u)) {
+              atomicOr(a.status, kStatusTimeout);
+              ok = false;
+              break;
+            }
+            const int col = piece ? nkc + kc : kc;
+            mbar_arrive_expect_tx(&a_full[s], kABytes);
+            tma_load_2d(&qmap, &a_full[s], a_s + s * kABytes, col * 64, (int)(qt * kTM));
           }
-          const int col = (kc >> 1) + (kc & 1) * nkc;
-          mbar_arrive_expect_tx(&a_full[s], kABytes);
-          tma_load_2d(&qmap, &a_full[s], a_s + s * kABytes, col * 64, (int)(qt * kTM));
         }
       }
     }
@@ -257,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
           const bool qpart = PROD && kc >= nkc_m;
           const uint32_t d_tmem = tmem_base + (uint32_t)(ab * 256) + (qpart ? 128u : 0u);
           const int kfirst = qpart ? nkc_m : 0;
-          for (int piece = 0; piece < 2; ++piece, ++cha) {
+          for (int piece = 0; piece < (kc < nkc_m ? 2 : 1); ++piece, ++cha) {
             const int sa = (int)(cha % kAStages);
             if (!mbar_wait(&a_full[sa], (uint32_t)((cha / kAStages) & 1))) {
               ok = false;
@@ -280,65 +295,99 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
       if (!ok) atomicOr(a.status, kStatusTimeout);
       mma_commit(done_bar);
     }
-  } else if (warp < 6) {
-    // decoders: keys r + 128 e of the tile
-    const int r = threadIdx.x - 64;
+  } else if (warp < 10) {
+    // decoders.  Thread t takes key row kr of the tile and, for prod, group hf
+    // of each 64-coordinate chunk (mse: both groups).  The words of flattened
+    // chunk c (item it_lo + c / nkc, key chunk c % nkc) land in ring slot
+    // c % Ring, row kr, words 4 j .. 4 j + 3 for group j; word 3 (7) of a tile's
+    // first chunk carries n (rn).  Each thread copies what it decodes, Ring - 1
+    // chunks ahead, so a wait for its own copy groups is the only sync needed.
+    const int t = threadIdx.x - 64;
+    constexpr int R = T::Ring, RW = T::RingWords;
+    constexpr int NG = PROD ? 1 : 2;          // groups per thread per chunk
+    const int kr = PROD ? (t & 127) : t;      // key row in the tile
+    const int hf = PROD ? (t >> 7) : 0;       // first group (within the chunk)
+    const int64_t nch = (it_hi - it_lo) * nkc;
+    auto issue = [&](int64_t c) {
+      if (c < nch) {
+        const int64_t kt = (it_lo + c / nkc) % a.kt_count;
+        const int kc = (int)(c % nkc);
+        const bool qpart = PROD && kc >= nkc_m;
+        const int g0 = 2 * (qpart ? kc - nkc_m : kc);
+        const int64_t key = kt * TN + kr;
+        if (key < a.N) {
+          uint32_t* dst = ring_s + ((size_t)(c % R) * TN + kr) * RW;
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            const int gj = hf + j;  // group within the chunk
+            const int g = g0 + gj;
+            if (g >= a.G) break;
+            if (!qpart) {
+              const uint32_t* src = a.codes + key * a.W + g * BM;
+#pragma unroll
+              for (int q = 0; q < BM; ++q) cp_async4(dst + 4 * gj + q, src + q);
+            } else {
+              cp_async4(dst + 4 * gj, a.signs + key * a.G + g);
+            }
+          }
+          if (kc == 0) {
+            if (hf == 0) cp_async4(dst + 3, a.norms + key);
+            else cp_async4(dst + 7, a.rnorms + key);
+          }
+        }
+      }
+      cp_async_commit();  // one group per chunk, empty or not
+    };
+    for (int64_t c = 0; c < R - 1; ++c) issue(c);
     int64_t ch = 0;
     int i = 0;
     bool ok = true;
     for (int64_t it = it_lo; ok && it < it_hi; ++it, ++i) {
       const int64_t kt = it % a.kt_count;
+      const bool valid = kt * TN + kr < a.N;
       float* mk = mk_s + (i % kMkBufs) * TN;
       float* qk = qk_s + (i % kMkBufs) * TN;
-      int64_t key[KPT];
-      bool valid[KPT];
-#pragma unroll
-      for (int e = 0; e < KPT; ++e) {
-        key[e] = kt * TN + r + 128 * e;
-        valid[e] = key[e] < a.N;
-        mk[r + 128 * e] = valid[e] ? a.norms[key[e]] * a.inv_alpha : -1.f;
-        if (PROD) qk[r + 128 * e] = valid[e] ? a.rnorms[key[e]] * a.qjl_coef : 0.f;
-      }
       for (int kc = 0; kc < nkc; ++kc, ++ch) {
+        issue(ch + R - 1);
+        cp_async_wait<R - 1>();  // this thread's copies of chunk ch have landed
+        const uint32_t* slot = ring_s + ((size_t)(ch % R) * TN + kr) * RW;
+        if (kc == 0) {
+          if (hf == 0) mk[kr] = valid ? __uint_as_float(slot[3]) * a.inv_alpha : -1.f;
+          else qk[kr] = valid ? __uint_as_float(slot[7]) * a.qjl_coef : 0.f;
+        }
         const int sb = (int)(ch % kBStages);
         if (!mbar_wait(&b_empty[sb], (uint32_t)(((ch / kBStages) & 1) ^ 1))) {
           ok = false;
           break;
         }
-        uint8_t* bt = b_s + sb * kBBytes;
+        uint8_t* brow = b_s + sb * kBBytes + kr * 128;
         const bool qpart = PROD && kc >= nkc_m;
-        const int c64 = qpart ? kc - nkc_m : kc;  // 64-coordinate chunk index
-        const int g0 = 2 * c64;                   // first code group of the chunk
+        const int g0 = 2 * (qpart ? kc - nkc_m : kc);
 #pragma unroll
-        for (int e = 0; e < KPT; ++e) {
-          const int row = r + 128 * e;
-          uint32_t h[32];
-          if (!valid[e] || g0 >= a.G) {
+        for (int j = 0; j < NG; ++j) {
+          const int gj = hf + j;
+          uint32_t o[16];
+          if (!valid || g0 + gj >= a.G) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) h[q] = 0u;
+            for (int q = 0; q < 16; ++q) o[q] = 0u;
           } else if (!qpart) {
-            uint32_t w[6] = {0u, 0u, 0u, 0u, 0u, 0u};
-            const uint32_t* src = a.codes + key[e] * a.W + g0 * a.bm;
-            const int nw = ((g0 + 1 < a.G) ? 2 : 1) * a.bm;
-            for (int q = 0; q < nw; ++q) w[q] = src[q];
-            decode_mse64(w, a.bm, g0 + 1 < a.G, mtab, lane, h);
+            const uint4 w = *reinterpret_cast<const uint4*>(slot + 4 * gj);
+            const uint32_t p[3] = {w.x, w.y, w.z};
+            decode_mse32<BM>(p, mtab, lane, o);
           } else {
-            uint32_t sw[2];
-            const uint32_t* src = a.signs + key[e] * a.G + g0;
-            sw[0] = src[0];
-            sw[1] = (g0 + 1 < a.G) ? src[1] : 0u;
-            decode_sign64(sw, g0 + 1 < a.G, stab, lane, h);
+            decode_sign32(slot[4 * gj], stab, lane, o);
           }
-          // row of the K-major 128B-swizzled tile: 8 chunks of 16 bytes
+          // 16-byte units 4 gj .. 4 gj + 3 of the key's row, 128B-swizzled
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8)
-            *reinterpret_cast<uint4*>(bt + row * 128 + ((c8 ^ (row & 7)) * 16)) =
-                make_uint4(h[4 * c8], h[4 * c8 + 1], h[4 * c8 + 2], h[4 * c8 + 3]);
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(brow + (((4 * gj + u) ^ (kr & 7)) * 16)) =
+                make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        fence_async_smem();
         mbar_arrive(&b_full[sb]);
       }
     }
+    cp_async_wait<0>();  // no copy may still be writing when the block exits
     if (!ok) atomicOr(a.status, kStatusTimeout);
   } else {
     // epilogue: thread = query row of the tile
@@ -347,15 +396,14 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     float bv[kKMax];
     int32_t bi[kKMax];
     const int K = a.topk;
+    float kth = -FLT_MAX;  // bv[K - 1], kept in a register
     int64_t cur_qt = -1;
     int seg = -1;
     int i = 0;
     auto flush = [&]() {
       if (seg < 0 || K == 0) return;
       const int64_t base = (((int64_t)blockIdx.x * a.max_seg + seg) * kTM + row) * K;
-#pragma unroll
-      for (int j = 0; j < kKMax; ++j)
-        if (j < K) a.cand_val[base + j] = bv[j], a.cand_idx[base + j] = bi[j];
+      for (int j = 0; j < K; ++j) a.cand_val[base + j] = bv[j], a.cand_idx[base + j] = bi[j];
     };
     for (int64_t it = it_lo; it < it_hi; ++it, ++i) {
       const int64_t qt = it / a.kt_count, kt = it % a.kt_count;
@@ -363,8 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         flush();
         ++seg;
         cur_qt = qt;
-#pragma unroll
         for (int j = 0; j < kKMax; ++j) bv[j] = -FLT_MAX, bi[j] = INT32_MAX;
+        kth = -FLT_MAX;
       }
       const int ab = i & 1;
       if (!mbar_wait(&acc_full[ab], (uint32_t)((i >> 1) & 1))) {
@@ -381,28 +429,48 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         float v[32], vq[32];
         tmem_ld32(t0 + c * 32, v);
         if (PROD) tmem_ld32(t0 + 128 + c * 32, vq);
+        // per-key factors of the 32 columns (same for every row: broadcast reads)
+        float mv[32], qv[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mk + c * 32 + 4 * u);
+          mv[4 * u] = m4.x, mv[4 * u + 1] = m4.y, mv[4 * u + 2] = m4.z, mv[4 * u + 3] = m4.w;
+          if (PROD) {
+            const float4 q4 = *reinterpret_cast<const float4*>(qk + c * 32 + 4 * u);
+            qv[4 * u] = q4.x, qv[4 * u + 1] = q4.y, qv[4 * u + 2] = q4.z, qv[4 * u + 3] = q4.w;
+          }
+        }
         tmem_wait_ld();
+        uint32_t hits = 0u;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int col = c * 32 + e;
-          const float m = mk[col];
-          if (m < 0.f) continue;
-          const float s = PROD ? (m * v[e] + qk[col] * vq[e]) * invs : m * v[e] * invs;
-          const int64_t keyi = kt * TN + col;
-          if (a.scores && q < a.nq) a.scores[q * a.N + keyi] = s;
-          if (K > 0 && s > bv[K - 1]) {
-            // insertion into the descending list (ties keep the earlier, lower index)
-            float cv = s;
-            int32_t ci = (int32_t)keyi;
+          const float sc = PROD ? fmaf(mv[e], v[e], qv[e] * vq[e]) * invs : mv[e] * v[e] * invs;
+          v[e] = mv[e] < 0.f ? -FLT_MAX : sc;  // no key in this column
+          hits |= (v[e] > kth ? 1u : 0u) << e;
+        }
+        const int64_t key0 = kt * TN + c * 32;
+        if (a.scores && q < a.nq) {
+          const int nvalid = (int)((a.N - key0) < 32 ? (a.N - key0) : 32);
+          float* dst = a.scores + q * a.N + key0;
+          if (nvalid == 32 && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) {
 #pragma unroll
-            for (int j = 0; j < kKMax; ++j) {
-              if (j < K && cv > bv[j]) {
-                const float tv = bv[j];
-                const int32_t ti = bi[j];
-                bv[j] = cv, bi[j] = ci;
-                cv = tv, ci = ti;
-              }
-            }
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<float4*>(dst + 4 * u) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e < nvalid) dst[e] = v[e];
+          }
+        }
+        if (K > 0 && hits) {
+          // rare after the first keys: walk the candidates from a local copy
+          float cand[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) cand[e] = v[e];
+          while (hits) {
+            const int e = __ffs(hits) - 1;
+            hits &= hits - 1u;
+            if (cand[e] > kth) kth = topk_insert(bv, bi, K, cand[e], (int32_t)(key0 + e));
           }
         }
       }
@@ -421,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
 }
 
 // [q'; q''] s per query (s a power of two putting the largest entry in
-// [2^13, 2^14)) as two fp16 pieces hi + lo, each padded to d_pad per part:
-// row = [hi(q' s), hi(q'' s) | lo(q' s), lo(q'' s)]; 1/s kept
+// [2^13, 2^14)) in fp16, each part padded to d_pad: row = [hi(q' s), hi(q'' s) |
+// lo(q' s)], lo = q' s - hi (exact in fp32, then rounded); 1/s kept
 __global__ void qcat_kernel(const float* qrot, const float* qproj, int64_t nq, int64_t nq_pad, int d, int d_pad,
                             int prod, __half* qcat, float* inv_s) {
   const int64_t qi = blockIdx.x;
   const int half = d_pad * (prod ? 2 : 1);
-  const int kdim = 2 * half;
+  const int kdim = half + d_pad;
   __shared__ float red[32];
   float m = 0.f;
   if (qi < nq)
@@ -452,7 +520,7 @@ __global__ void qcat_kernel(const float* qrot, const float* qproj, int64_t nq, i
     const float vs = v * s;  // exact: s is a power of two
     const __half hi = __float2half_rn(vs);
     qcat[qi * kdim + j] = hi;
-    qcat[qi * kdim + half + j] = __float2half_rn(vs - __half2float(hi));  // the difference is exact in fp32
+    if (j < d_pad) qcat[qi * kdim + half + j] = __float2half_rn(vs - __half2float(hi));
   }
   if (threadIdx.x == 0) inv_s[qi] = (qi < nq) ? 1.f / s : 0.f;
 }
@@ -505,7 +573,7 @@ static ScoresPlan scores_plan(const tq_ctx* h, int64_t nq, int64_t N) {
   p.tn = prod ? Tile<true>::TN : Tile<false>::TN;
   p.nq_pad = (nq + kTM - 1) / kTM * kTM;
   p.d_pad = (h->d + 63) / 64 * 64;
-  p.kdim = 2 * p.d_pad * (prod ? 2 : 1);
+  p.kdim = p.d_pad * (prod ? 3 : 2);  // hi of q' (and q''), lo of q'
   p.qt = p.nq_pad / kTM;
   p.kt = (N + p.tn - 1) / p.tn;
   p.total = p.qt * p.kt;
@@ -591,25 +659,32 @@ int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t
   a.max_seg = p.max_seg;
   for (int k = 0; k < 8; ++k) a.ctab[k] = (uint32_t)h->sc_tab[2 * k] | ((uint32_t)h->sc_tab[2 * k + 1] << 16);
   a.status = h->dev.status;
+  auto launch = [&](auto kern, int smem) -> int {
+    // one attribute call per instantiation
+    static bool attr[2][4] = {};
+    bool& set = attr[prod ? 1 : 0][h->bm];
+    if (!set) {
+      cudaError_t ee = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (ee != cudaSuccess) return (int)ee;
+      set = true;
+    }
+    kern<<<(unsigned)p.G, kThreads, smem, s>>>(map, a);
+    return 0;
+  };
   if (prod) {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t ee = cudaFuncSetAttribute(scores_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            Tile<true>::Smem);
-      if (ee != cudaSuccess) return (int)ee;
-      attr = true;
+    switch (h->bm) {
+      case 1: e = launch(scores_tc_kernel<true, 1>, Tile<true>::Smem); break;
+      case 2: e = launch(scores_tc_kernel<true, 2>, Tile<true>::Smem); break;
+      default: e = launch(scores_tc_kernel<true, 3>, Tile<true>::Smem); break;
     }
-    scores_tc_kernel<true><<<(unsigned)p.G, kThreads, Tile<true>::Smem, s>>>(map, a);
   } else {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t ee = cudaFuncSetAttribute(scores_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            Tile<false>::Smem);
-      if (ee != cudaSuccess) return (int)ee;
-      attr = true;
+    switch (h->bm) {
+      case 1: e = launch(scores_tc_kernel<false, 1>, Tile<false>::Smem); break;
+      case 2: e = launch(scores_tc_kernel<false, 2>, Tile<false>::Smem); break;
+      default: e = launch(scores_tc_kernel<false, 3>, Tile<false>::Smem); break;
     }
-    scores_tc_kernel<false><<<(unsigned)p.G, kThreads, Tile<false>::Smem, s>>>(map, a);
   }
+  if (e) return e;
   if ((e = (int)cudaGetLastError())) return e;
   if (topk > 0) {
     topk_merge_kernel<<<(unsigned)((nq + 127) / 128), 128, 0, s>>>(cv, ci, nq, p.G, p.max_seg, p.total, p.kt, topk,
