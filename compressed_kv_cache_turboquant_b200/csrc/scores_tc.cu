@@ -49,7 +49,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kTM = 128;          // queries per tile
-constexpr int kAStages = 4;
+constexpr int kAStages = 3;
 constexpr int kABytes = kTM * 128;  // one 64-wide fp16 chunk of the query tile
 constexpr int kTabBytes = 32768;
 constexpr int kThreads = 448;
@@ -70,8 +70,9 @@ struct Tile {
   static constexpr int Ring = PROD ? 8 : 4;         // staged chunks ahead per decoder thread
   static constexpr int RingWords = 8;               // words staged per key per chunk (4 per group)
   static constexpr int RingBytes = Ring * TN * RingWords * 4;
+  static constexpr int TopkBytes = 2 * kKMax * kTM * 4;  // running top-k values and indices per query row
   static constexpr int Smem = kAStages * kABytes + BStages * BBytes + Tabs * kTabBytes + kMkBufs * TN * 8 +
-                              RingBytes + 512 + 1024;
+                              RingBytes + TopkBytes + 512 + 1024;
 };
 
 struct ScArgs {
@@ -149,16 +150,19 @@ __device__ __forceinline__ void decode_sign32(uint32_t sw, const uint8_t* tab, i
 // (s > bv[K-1] on entry); an equal score stays behind the earlier, lower key.
 // Rare after the first keys, so kept out of line: the unrolled epilogue only
 // compares against the returned new k-th value.
+// The lists live in shared memory, entry j of row r at [j * 128 + r]: this
+// kernel leaves L1 almost no room beside its shared memory, so a list in local
+// memory would be an L2 round trip per access.
 __device__ __noinline__ float topk_insert(float* bv, int32_t* bi, int K, float s, int32_t key) {
   int j = K - 1;
-  while (j > 0 && bv[j - 1] < s) {
-    bv[j] = bv[j - 1];
-    bi[j] = bi[j - 1];
+  while (j > 0 && bv[(j - 1) * kTM] < s) {
+    bv[j * kTM] = bv[(j - 1) * kTM];
+    bi[j * kTM] = bi[(j - 1) * kTM];
     --j;
   }
-  bv[j] = s;
-  bi[j] = key;
-  return bv[K - 1];
+  bv[j * kTM] = s;
+  bi[j * kTM] = key;
+  return bv[(K - 1) * kTM];
 }
 
 template <bool PROD, int BM>
@@ -175,7 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
   float* mk_s = reinterpret_cast<float*>(mtab + T::Tabs * kTabBytes);  // [kMkBufs][TN]
   float* qk_s = mk_s + kMkBufs * TN;                                   // [kMkBufs][TN]
   uint32_t* ring_s = reinterpret_cast<uint32_t*>(qk_s + kMkBufs * TN); // [Ring][TN][RingWords]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_s + T::Ring * TN * T::RingWords);
+  float* tkv_s = reinterpret_cast<float*>(ring_s + T::Ring * TN * T::RingWords);  // [kKMax][128]
+  int32_t* tki_s = reinterpret_cast<int32_t*>(tkv_s + kKMax * kTM);               // [kKMax][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tki_s + kKMax * kTM);
   uint64_t* a_full = bars;                 // [kAStages]
   uint64_t* a_empty = a_full + kAStages;   // [kAStages]
   uint64_t* b_full = a_empty + kAStages;   // [kBStages] count 128
@@ -393,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     // epilogue: thread = query row of the tile
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    float bv[kKMax];
-    int32_t bi[kKMax];
+    float* bv = tkv_s + row;    // entry j at bv[j * 128]
+    int32_t* bi = tki_s + row;
     const int K = a.topk;
     float kth = -FLT_MAX;  // bv[K - 1], kept in a register
     int64_t cur_qt = -1;
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     auto flush = [&]() {
       if (seg < 0 || K == 0) return;
       const int64_t base = (((int64_t)blockIdx.x * a.max_seg + seg) * kTM + row) * K;
-      for (int j = 0; j < K; ++j) a.cand_val[base + j] = bv[j], a.cand_idx[base + j] = bi[j];
+      for (int j = 0; j < K; ++j) a.cand_val[base + j] = bv[j * kTM], a.cand_idx[base + j] = bi[j * kTM];
     };
     for (int64_t it = it_lo; it < it_hi; ++it, ++i) {
       const int64_t qt = it / a.kt_count, kt = it % a.kt_count;
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         flush();
         ++seg;
         cur_qt = qt;
-        for (int j = 0; j < kKMax; ++j) bv[j] = -FLT_MAX, bi[j] = INT32_MAX;
+        for (int j = 0; j < kKMax; ++j) bv[j * kTM] = -FLT_MAX, bi[j * kTM] = INT32_MAX;
         kth = -FLT_MAX;
       }
       const int ab = i & 1;
@@ -463,15 +469,10 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
           }
         }
         if (K > 0 && hits) {
-          // rare after the first keys: walk the candidates from a local copy
-          float cand[32];
+          // rare after the first keys: insert the candidates straight from registers
 #pragma unroll
-          for (int e = 0; e < 32; ++e) cand[e] = v[e];
-          while (hits) {
-            const int e = __ffs(hits) - 1;
-            hits &= hits - 1u;
-            if (cand[e] > kth) kth = topk_insert(bv, bi, K, cand[e], (int32_t)(key0 + e));
-          }
+          for (int e = 0; e < 32; ++e)
+            if (((hits >> e) & 1u) && v[e] > kth) kth = topk_insert(bv, bi, K, v[e], (int32_t)(key0 + e));
         }
       }
       tc_fence_before();
