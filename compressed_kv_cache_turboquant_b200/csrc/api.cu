@@ -613,6 +613,8 @@ extern "C" size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int
     if (!hk[g]) return 0;
     bytes += 2 * align_up((size_t)B * Hq * hk[g]->d * 4, 256);
   }
+  // fp16 query fragments of the tensor-core path
+  if (ngroups == 2) bytes += logits_mma_workspace((int64_t)B * Hq);
   return bytes;
 }
 
@@ -668,8 +670,13 @@ extern "C" int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* c
     qp[g] = p;
     off += hk[g]->d;
   }
-  if (!e)
-    e = launch_logits(hk, ngroups, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale, logits,
-                      stream);
+  if (!e) {
+    if (logits_mma_supported(hk, ngroups, kv_stride))
+      e = launch_logits_mma(hk, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale, logits, ws,
+                            stream);
+    else
+      e = launch_logits(hk, ngroups, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale,
+                        logits, stream);
+  }
   return e ? cuda_error("tq_attn_logits", e) : clear_error();
 }

@@ -1,0 +1,46 @@
+// Register-fragment helpers shared by the mma.sync kernels over packed codes:
+// byte-permute addressed table lookups (one table copy per lane, so the 32
+// lookups of a warp never meet in a shared-memory bank) and the m16n8k16
+// fp16 MMA with fp32 accumulation.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tqi {
+namespace frag {
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) { return __byte_perm(a, b, s); }
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// the 4 bytes of a code word -> 4 fp16 pairs; `lane_off` holds this lane's
+// column offset in byte 0, `tab` the table's shared-memory address
+__device__ __forceinline__ void lookup4(uint32_t w, uint32_t tab, uint32_t lane_off, uint32_t* out) {
+  out[0] = lds32(tab + prmt(w, lane_off, 0x5504));
+  out[1] = lds32(tab + prmt(w, lane_off, 0x5514));
+  out[2] = lds32(tab + prmt(w, lane_off, 0x5524));
+  out[3] = lds32(tab + prmt(w, lane_off, 0x5534));
+}
+
+}  // namespace frag
+}  // namespace tqi

@@ -100,6 +100,12 @@ int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t
                      const float* norms, const float* rnorms, int64_t N, float* scores, int topk, int32_t* top_idx,
                      float* top_val, void* workspace, void* stream);
 bool logits_supported(const tq_ctx* const* hk, int ngroups);
+bool logits_mma_supported(const tq_ctx* const* hk, int ngroups, int64_t kv_stride);
+size_t logits_mma_workspace(int64_t nq);
+int launch_logits_mma(const tq_ctx* const* hk, const float* const* qrot, const float* const* qproj, int B, int Hq,
+                      int Hkv, int64_t T, int64_t kv_stride, const uint32_t* const* kcodes,
+                      const uint32_t* const* ksigns, const float* const* knorms, const float* const* krnorms,
+                      float scale, float* logits, void* workspace, void* stream);
 int launch_logits(const tq_ctx* const* hk, int ngroups, const float* const* qrot, const float* const* qproj, int B,
                   int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* const* kcodes,
                   const uint32_t* const* ksigns, const float* const* knorms, const float* const* krnorms,
