@@ -18,10 +18,10 @@
 // numbers; the rotated queries enter as two fp16 pieces (hi + lo), the
 // projected queries as one; norms and scales are applied in fp32.
 //
-// Persistent CTAs own equal contiguous ranges of 128-token blocks over all
+// Persistent CTAs own equal contiguous ranges of 192-token blocks over all
 // (batch, kv-head) pairs; warp 0 bulk-copies each block (codes, signs and the
-// four norm arrays of both groups) into a ring; 8 consumer warps take 16
-// tokens each and write the block's 4 x 128 logits.
+// four norm arrays of both groups) into a ring; 12 consumer warps take 16
+// tokens each and write the block's 4 x 192 logits.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -37,9 +37,9 @@ namespace {
 using namespace sm100;
 using namespace frag;
 
-constexpr int kBlk = 128;     // tokens per stage
+constexpr int kCons = 12;     // consumer warps (three per SM sub-partition)
+constexpr int kBlk = 16 * kCons;  // tokens per stage, 16 per consumer warp
 constexpr int kStages = 6;
-constexpr int kCons = 8;      // consumer warps
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kTabBytes = 256 * 256;
 constexpr float kQjl64 = 1.2533141373155003f / 64.f;
@@ -58,6 +58,7 @@ struct LgLayout {
   static constexpr int Stage = R1 + kBlk * 4;
   static constexpr int TokBytes = (W0 + 2 + W1 + 2 + 4) * 4;
   static constexpr int Smem = kStages * Stage + 2 * kTabBytes + kCons * 64 * 4 + 256 + 1024;
+  static_assert(Stage % 16 == 0, "stage offsets stay 16-byte aligned");
 };
 
 struct LgArgs {
