@@ -4,11 +4,12 @@
 // TurboQuant form and QJL is used inside attention; tmdm.cn ("谷歌悄悄扔下一颗
 // “性能核弹”…", 实测数据): attention logits computed directly over a 4-bit cache.
 //
-// Work split: one CTA per (batch, kv-head, context split).  The 4 query heads
-// of the kv-head's group share every key and value read.
-//   warp 0     producer: bulk copies of 64-token blocks (K codes, QJL signs,
-//              V codes and the three norm arrays) into an 8-stage ring
-//   warps 1-4  consumers, 16 tokens of every block each:
+// Work split: persistent CTAs own equal contiguous ranges of 192-token blocks
+// over all (batch, kv-head) pairs; the 4 query heads of a kv-head's group share
+// every key and value read.
+//   warp 0      producer: bulk copies of each block (K codes, QJL signs, V codes
+//               and the three norm arrays) into a 2-stage ring
+//   warps 1-12  consumers (three per SM sub-partition), 16 tokens of every block each:
 //     logits   mma.sync m16n8k16 (fp16 in, fp32 accumulate), keys as M, the
 //              K dimension = 128 mse coordinates then 128 QJL coordinates,
 //              N = 8 columns = 4 rotated queries (mse part) and 4 projected
@@ -16,9 +17,9 @@
 //     softmax  online, per head, in base 2
 //     values   mma.sync with M = 128 coordinates (rotated frame), K = 16 tokens,
 //              N = 4 heads; the weights carry the value norms
-//   the four warps' states merge in shared memory; partial (max, sum, acc[d])
-//   per head goes to the workspace; the merge kernel combines the splits and
-//   rotates back once.
+//   the consumer warps' states merge in shared memory when a CTA leaves a
+//   (batch, kv-head); partial (max, sum, acc[d]) per head goes to the workspace;
+//   the merge kernel combines the CTAs that covered it and rotates back once.
 // Decoding: every byte of key or value codes holds two indices and is turned
 // into an fp16 pair by one lookup in a 256-entry table in shared memory (one
 // table replica per lane, so the 32 lookups of a warp never share a bank); QJL
@@ -39,9 +40,9 @@ using namespace sm100;
 using namespace frag;
 
 constexpr int D = 128;
-constexpr int kBlk = 128;      // tokens per stage (16 per consumer warp)
-constexpr int kStages = 4;
-constexpr int kCons = 8;       // consumer warps
+constexpr int kCons = 12;      // consumer warps (three per SM sub-partition)
+constexpr int kBlk = 16 * kCons;  // tokens per stage (16 per consumer warp)
+constexpr int kStages = 2;
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kKW = 12;        // K code words per token (3 bits x 128 / 32)
 constexpr int kSW = 4;         // sign words
@@ -53,7 +54,8 @@ constexpr int kOffV = kOffS + kBlk * kSW * 4;
 constexpr int kOffN = kOffV + kBlk * kVW * 4;
 constexpr int kOffR = kOffN + kBlk * 4;
 constexpr int kOffVN = kOffR + kBlk * 4;
-constexpr int kStageBytes = kOffVN + kBlk * 4;  // 17920
+constexpr int kStageBytes = kOffVN + kBlk * 4;  // 26880
+static_assert(kStageBytes % 16 == 0 && kOffS % 16 == 0 && kOffV % 16 == 0 && kOffN % 16 == 0, "bulk-copy alignment");
 // Decode tables in shared memory, 256 rows of 256 bytes each, indexed by one
 // byte of codes (two indices, or eight sign bits):
 //   KV table, row B: [K entry, one 4-byte copy per lane][V entry, one per lane]
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
     int seg = -1;
     bool ok = true;
 
-    // publish this warp's state, combine the eight warps, write one partial
+    // publish this warp's state, combine the consumer warps, write one partial
     auto flush = [&](int sg) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
