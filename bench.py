@@ -43,6 +43,12 @@ DEC = dict(B=8, Hq=32, Hkv=8, T=131072)
 METRIC = "vectors quantized/s; packed-KV logits keys/s and % of HBM-bandwidth roofline"
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# sweep kernels, averaged over b = 1..4, from one ncu capture of these kernels;
+# to be re-taken (or set to None) whenever either kernel changes
+MEASURED_TRAFFIC = {"quant_mse": 299.2e6, "dequant_mse": 519.5e6}
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -524,7 +530,7 @@ def run_ours(args):
     achieved = dk["bytes_total"] / (dk["ms_total"] / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
-                "traffic": None,
+                "traffic": MEASURED_TRAFFIC.get(dom) if args.workload == "sweep" else None,
                 "bytes_per_launch": dk["bytes_total"] / dk["launches"]}
     kernels = {k: {"avg_ms": v["ms_total"] / v["launches"],
                    "GBps": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9,
