@@ -13,9 +13,11 @@
 //   warp 1      TMEM allocation and the single-thread MMA issuer:
 //               Y[128 x d] = X[128 x d] . (Pi_hi + Pi_mid + Pi_lo)^T, three
 //               bf16 passes accumulated in fp32 in TMEM (double-buffered)
-//   warps 2..9  epilogue, one thread per vector (TMEM lane) and half of the
-//               columns per warpgroup: n = ||y|| (= ||x||, Pi orthogonal),
-//               cell of every coordinate against n * t_k, packing, stores
+//   warps 2..    epilogue, 4 warps per 32-coordinate group (d / 8 warps): one
+//               thread per vector (TMEM lane) and group; n = ||y|| (= ||x||,
+//               Pi orthogonal) from the groups' partial sums, the cell of every
+//               coordinate against n * t_k, packing, stores.  Four warps per
+//               SM sub-partition keep the issue slots busy.
 //
 // Precision: x is exact in bf16; Pi = hi + mid + lo carries ~24 significant
 // bits, so every product is exact in fp32 and y has fp32-level error (far
@@ -35,7 +37,9 @@ using namespace sm100;
 
 constexpr int kPieces = 3;
 constexpr int kTileM = 128;
-constexpr int kThreads = 320;  // 10 warps
+// warps: TMA producer, MMA issuer, 4 epilogue warps per 32-coordinate group
+template <int D>
+constexpr int threads_for() { return 32 * (2 + 4 * (D / 32)); }
 
 template <int D>
 struct TcShape {
@@ -46,7 +50,7 @@ struct TcShape {
   static constexpr int kPieceBytes = kSlabs * kSlabBytesPi;  // = D * D * 2
   static constexpr int kStages = (D == 128) ? 3 : 4;
   static constexpr int kTmemCols = 2 * D;                    // two accumulators
-  static constexpr int kMiscBytes = 4096;  // barriers, TMEM slot, thresholds, norm partials
+  static constexpr int kMiscBytes = 8192;  // barriers, TMEM slot, thresholds, norm partials
   static constexpr int kSmemBytes = kPieces * kPieceBytes + kStages * kStageBytes + kMiscBytes +
                                     1024 /*alignment*/;
 };
@@ -112,6 +116,65 @@ __device__ __forceinline__ void pack_group(const float* v, const float (&P)[8], 
   }
 }
 
+// The same cells computed on the FMA pipe (the binary search above runs on
+// the ALU pipe, which the epilogue saturates at 3 and 4 bits; half of the
+// groups go each way).  With B = 2^32 / n and C_k = 1 - 2^32 t_k:
+//   sat(|y| B + C_k) = 1 when |y| >= n t_k and 0 when |y| < n t_k (up to a band
+//   of 2^-32 n around the threshold, far inside the parity band), so
+//   m = sum_k sat(|y| B + C_k) counts the positive thresholds at or below |y|,
+//   s = sat(y B + 1) is 1 for y >= 0 (to the same band), and
+//   cell = (H - 1 - m) + s (2m + 1).
+// Adding 2^23 leaves the cell in the low mantissa bits, and integer
+// multiply-adds shift it into place; the constant part of those bit patterns is
+// cancelled by the starting value of each word.  A zero vector (n = 0) takes
+// B = 0, C_k = -1: every count is 0 and s = 1, the cell above the middle.
+template <int BM>
+struct FmaCells {
+  static constexpr int kFields = 32 / (BM == 3 ? 4 : BM);  // cells per word (3 bits: nibbles)
+  static constexpr int kWidth = BM == 3 ? 4 : BM;
+  __host__ __device__ static constexpr uint32_t init() {
+    uint32_t c = 0u;
+    for (int i = 0; i < kFields; ++i) c += (kWidth * i < 32) ? (0x4B000000u << (kWidth * i)) : 0u;
+    return 0u - c;
+  }
+};
+
+template <int BM>
+__device__ __forceinline__ uint32_t cell_fma_bits(float y, float B, const float (&C)[8]) {
+  constexpr int H = 1 << (BM - 1);
+  const float s = __saturatef(fmaf(y, B, 1.f));
+  float m = 0.f;
+#pragma unroll
+  for (int k = 1; k < H; ++k) m += __saturatef(fmaf(fabsf(y), B, C[k]));
+  const float u = fmaf(m, 2.f, 1.f);
+  const float v = ((float)(H - 1) + 8388608.f) - m;
+  return __float_as_uint(fmaf(s, u, v));  // 0x4B000000 | cell
+}
+
+// pack one group of 32 coordinates with the FMA-pipe cells; for 3 bits the
+// cells of coordinates 24..31 (spread over the spare bits) use the ALU search
+template <int BM>
+__device__ __forceinline__ void pack_group_fma(const float* v, const float (&P)[8], float B, const float (&C)[8],
+                                               uint32_t (&w)[BM]) {
+  using F = FmaCells<BM>;
+#pragma unroll
+  for (int k = 0; k < BM; ++k) w[k] = F::init();
+  if constexpr (BM == 3) {
+#pragma unroll
+    for (int i = 0; i < 24; ++i) w[i >> 3] += cell_fma_bits<3>(v[i], B, C) * (1u << (4 * (i & 7)));
+    uint32_t X = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) X |= cell_index<3>(v[24 + j], P) << (4 * j);
+    w[0] |= (X << 3) & 0x88888888u;
+    w[1] |= (X << 2) & 0x88888888u;
+    w[2] |= (X << 1) & 0x88888888u;
+  } else {
+    constexpr int per = 32 / BM;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i / per] += cell_fma_bits<BM>(v[i], B, C) * (1u << (BM * (i % per)));
+  }
+}
+
 template <int BM>
 __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[BM]) {
   if constexpr (BM == 4) {
@@ -125,7 +188,7 @@ __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t (&w)[B
 }
 
 template <int D, int BM>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for<D>(), 1)
     quant_mse_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcArgs a) {
   using S = TcShape<D>;
   constexpr int W = (D / 32) * BM;  // words per vector
@@ -141,10 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;          // [2]
   uint64_t* pi_bar = acc_empty + 2;
   uint64_t* done_bar = pi_bar + 1;
-  uint64_t* npart_bar = done_bar + 1;          // [2] norm partials of both halves written
+  uint64_t* npart_bar = done_bar + 1;          // [2] norm partials of every group written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(npart_bar + 2);
   float* thr_s = reinterpret_cast<float*>(tmem_slot + 4);  // [16]
-  float* npart = thr_s + 16;                               // [2 parity][2 halves][128]
+  float* npart = thr_s + 16;                               // [2 parity][d / 32 groups][128]
+  constexpr int kGroups = D / 32, kEpiWarps = 4 * kGroups;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = (a.N + kTileM - 1) / kTileM;
@@ -156,12 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);
+      mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(pi_bar, 1);
     mbar_init(done_bar, 1);
-    mbar_init(&npart_bar[0], 256);
-    mbar_init(&npart_bar[1], 256);
+    mbar_init(&npart_bar[0], 32 * kEpiWarps);
+    mbar_init(&npart_bar[1], 32 * kEpiWarps);
     fence_mbar_init();
   }
   if (threadIdx.x < K - 1) thr_s[threadIdx.x] = a.thresholds[threadIdx.x];
@@ -225,13 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(done_bar);  // arrives once everything issued above has completed
     }
   } else {
-    // epilogue: 8 warps; warp % 4 selects the TMEM lane quarter, the warpgroup the column half
+    // epilogue: warp % 4 selects the TMEM lane quarter, (warp - 2) / 4 the 32-coordinate group
     const int ew = warp - 2;
-    const int half = ew >> 2;
+    const int grp = ew >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    constexpr int HC = D / 2;   // columns per half
-    constexpr int GH = HC / 32; // code groups per half
     float P[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) P[m] = 0.f;
@@ -244,39 +306,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float v[HC];
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * D + half * HC);
-#pragma unroll
-      for (int c = 0; c < HC / 32; ++c) tmem_ld32(taddr + c * 32, *reinterpret_cast<float(*)[32]>(&v[c * 32]));
+      float v[32];
+      tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * D + grp * 32), v);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
       float ss = 0.f;
 #pragma unroll
-      for (int c = 0; c < HC; ++c) ss = fmaf(v[c], v[c], ss);
-      // exchange the two halves' partial sums of squares (bounded wait)
-      float* np = npart + (i & 1) * 256;
-      np[half * 128 + row] = ss;
+      for (int c = 0; c < 32; ++c) ss = fmaf(v[c], v[c], ss);
+      // exchange the groups' partial sums of squares (bounded wait)
+      float* np = npart + (i & 1) * kGroups * 128;
+      np[grp * 128 + row] = ss;
       mbar_arrive(&npart_bar[i & 1]);
       if (!mbar_wait(&npart_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
-      const float n = sqrtf(np[row] + np[128 + row]);
+      float sq = 0.f;
 #pragma unroll
+      for (int k = 0; k < kGroups; ++k) sq += np[k * 128 + row];
+      const float n = sqrtf(sq);
       // a zero vector has y = 0, which lies below every positive threshold
+#pragma unroll
       for (int m = 1; m < (1 << (BM - 1)); ++m) P[m] = n > 0.f ? n * thr_s[(1 << (BM - 1)) - 1 + m] : INFINITY;
       const int64_t vec = tile * kTileM + row;
       if (vec < a.N) {
-        uint32_t* dst = a.codes + vec * a.out_stride * W + half * GH * BM;
+        uint32_t w[BM];
+        // odd groups count thresholds on the FMA pipe, even ones search on the ALU pipe
+        if (BM >= 2 && (grp & 1)) {
+          const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
+          float Cf[8];
 #pragma unroll
-        for (int g = 0; g < GH; ++g) {
-          uint32_t w[BM];
-          pack_group<BM>(&v[g * 32], P, w);
-          store_words<BM>(dst + g * BM, w);
+          for (int m = 0; m < 8; ++m)
+            Cf[m] = (n > 0.f && m >= 1 && m < (1 << (BM - 1))) ? 1.f - 4294967296.f * thr_s[(1 << (BM - 1)) - 1 + m]
+                                                                : -1.f;
+          pack_group_fma<BM>(v, P, Bf, Cf, w);
+        } else {
+          pack_group<BM>(v, P, w);
         }
-        if (half == 0) a.norms[vec * a.out_stride] = n;
+        store_words<BM>(a.codes + vec * a.out_stride * W + grp * BM, w);
+        if (grp == 0) a.norms[vec * a.out_stride] = n;
       }
     }
   }
@@ -316,7 +386,7 @@ int launch_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint3
   TcArgs a{h->dev.pi_tc, h->dev.thresholds, N, out_stride, codes, norms, h->dev.status};
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);
-  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(map, a);
+  kern<<<grid, threads_for<D>(), S::kSmemBytes, stream>>>(map, a);
   return (int)cudaGetLastError();
 }
 
