@@ -163,15 +163,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i) {
+      BlockCursor cur;
+      cur.init(gb_lo, a.nblk);
+      for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
         const int s = (int)(i % kStages);
         const uint32_t u = (uint32_t)(i / kStages);
         if (!mbar_wait(&empty[s], (u & 1u) ^ 1u)) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }
-        const int64_t bh = gb / a.nblk;
-        const int64_t t0 = (gb % a.nblk) * kBlk;
+        const int64_t bh = cur.bh;
+        const int64_t t0 = cur.blk * kBlk;
         const int n = (int)min((int64_t)kBlk, a.T - t0);
         const int n4 = n & ~3;  // norms are copied in whole 16-byte units
         uint8_t* st = stages + s * kStageBytes;
@@ -255,15 +257,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
       if (!mbar_wait(pub, 1u)) ok = false;
     };
 
-    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i) {
-      const int64_t bh = gb / a.nblk;
+    BlockCursor cur;
+    cur.init(gb_lo, a.nblk);
+    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
+      const int64_t bh = cur.bh;
       if (bh != cur_bh) {
         if (seg >= 0) flush(seg);
         if (!ok) break;
         ++seg;
         cur_bh = bh;
         // queries of this (batch, kv-head): mse columns 0-3 (q' of head g), QJL columns 4-7 (q'' of head g-4)
-        const int64_t b = bh / a.Hkv, hh = bh % a.Hkv;
+        const int64_t b = bh / a.Hkv, hh = bh - b * a.Hkv;
         const int64_t q0 = b * a.Hq + hh * group;
         const uint32_t* qf = a.qfrag + (q0 + (g & 3)) * 2 * 64;
 #pragma unroll
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         break;
       }
       const uint8_t* st = stages + s * kStageBytes;
-      const int64_t t0 = (gb % a.nblk) * kBlk;
+      const int64_t t0 = cur.blk * kBlk;
       const int n = (int)min((int64_t)kBlk, a.T - t0);
       const int tb = cw * 16;  // this warp's 16 tokens within the block
       // ---------------- logits: keys g and g+8 of the sub-block

@@ -164,14 +164,16 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i) {
+      BlockCursor cur;
+      cur.init(gb_lo, a.nblk);
+      for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
         const int s = (int)(i % kStages);
         if (!mbar_wait(&empty[s], (uint32_t)(((i / kStages) & 1) ^ 1))) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }
-        const int64_t bh = gb / a.nblk;
-        const int64_t t0 = (gb % a.nblk) * kBlk;
+        const int64_t bh = cur.bh;
+        const int64_t t0 = cur.blk * kBlk;
         const int n = (int)min((int64_t)kBlk, a.T - t0);
         const int n4 = n & ~3;  // whole 16-byte units; the consumers read the tail from global memory
         uint8_t* st = stages + s * L::Stage;
@@ -201,14 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
     float* ob = obuf + cw * 64;
     uint32_t qh[8][2], ql[8][2], qq[8][2];
     float isq[2][2];  // [head j][0: q' pieces, 1: q''] for this lane's accumulator columns
-    int64_t cur_bh = -1;
+    int64_t cur_bh = -1, q0 = 0;
     bool ok = true;
-    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i) {
-      const int64_t bh = gb / a.nblk;
-      const int64_t b = bh / a.Hkv, hh = bh % a.Hkv;
-      const int64_t q0 = b * a.Hq + hh * 4;  // first query head of the kv-head
+    BlockCursor cur;
+    cur.init(gb_lo, a.nblk);
+    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
+      const int64_t bh = cur.bh;
       if (bh != cur_bh) {
         cur_bh = bh;
+        const int64_t b = bh / a.Hkv, hh = bh - b * a.Hkv;
+        q0 = b * a.Hq + hh * 4;  // first query head of the kv-head
         // B fragments: column g = (group g >> 2, head g & 3); k-steps 0-3 belong to group 0,
         // 4-7 to group 1; coordinates 16c + 4 (kb & 3) .. + 3 of the lane's range
         const int colgrp = g >> 2, colhead = g & 3;
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
         break;
       }
       const uint8_t* st = stages + s * L::Stage;
-      const int64_t t0 = (gb % a.nblk) * kBlk;
+      const int64_t t0 = cur.blk * kBlk;
       const int n = (int)min((int64_t)kBlk, a.T - t0);
       const int n4 = n & ~3;
       const int tb = cw * 16;

@@ -42,5 +42,19 @@ __device__ __forceinline__ void lookup4(uint32_t w, uint32_t tab, uint32_t lane_
   out[3] = lds32(tab + prmt(w, lane_off, 0x5534));
 }
 
+// Position of a global token block gb = bh * nblk + blk, advanced one block at a
+// time: the hot loops never divide 64-bit integers (a software routine of
+// dozens of instructions per division).
+struct BlockCursor {
+  int64_t bh, blk;
+  __device__ __forceinline__ void init(int64_t gb, int64_t nblk) {
+    bh = gb / nblk;
+    blk = gb - bh * nblk;
+  }
+  __device__ __forceinline__ void next(int64_t nblk) {
+    if (++blk == nblk) blk = 0, ++bh;
+  }
+};
+
 }  // namespace frag
 }  // namespace tqi

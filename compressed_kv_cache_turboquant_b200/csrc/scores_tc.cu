@@ -314,10 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
     const int kr = PROD ? (t & 127) : t;      // key row in the tile
     const int hf = PROD ? (t >> 7) : 0;       // first group (within the chunk)
     const int64_t nch = (it_hi - it_lo) * nkc;
-    auto issue = [&](int64_t c) {
+    // the next chunk to stage, as (flattened index, key tile, key chunk), advanced by one
+    // per call (no 64-bit division per chunk)
+    int64_t iss_c = 0, iss_kt = it_lo % a.kt_count;
+    int iss_kc = 0;
+    auto issue = [&]() {
+      const int64_t c = iss_c;
       if (c < nch) {
-        const int64_t kt = (it_lo + c / nkc) % a.kt_count;
-        const int kc = (int)(c % nkc);
+        const int64_t kt = iss_kt;
+        const int kc = iss_kc;
         const bool qpart = PROD && kc >= nkc_m;
         const int g0 = 2 * (qpart ? kc - nkc_m : kc);
         const int64_t key = kt * TN + kr;
@@ -343,8 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         }
       }
       cp_async_commit();  // one group per chunk, empty or not
+      ++iss_c;
+      if (++iss_kc == nkc) {
+        iss_kc = 0;
+        if (++iss_kt == a.kt_count) iss_kt = 0;
+      }
     };
-    for (int64_t c = 0; c < R - 1; ++c) issue(c);
+    for (int64_t c = 0; c < R - 1; ++c) issue();
     int64_t ch = 0;
     int i = 0;
     bool ok = true;
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
       float* mk = mk_s + (i % kMkBufs) * TN;
       float* qk = qk_s + (i % kMkBufs) * TN;
       for (int kc = 0; kc < nkc; ++kc, ++ch) {
-        issue(ch + R - 1);
+        issue();  // chunk ch + R - 1
         cp_async_wait<R - 1>();  // this thread's copies of chunk ch have landed
         const uint32_t* slot = ring_s + ((size_t)(ch % R) * TN + kr) * RW;
         if (kc == 0) {
