@@ -86,10 +86,16 @@ __device__ __forceinline__ uint32_t ctab_half(const uint32_t (&t)[8], uint32_t k
   return (t[k >> 1] >> (16 * (k & 1u))) & 0xFFFFu;
 }
 
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 // 16 coordinates (one half of a 32-coordinate group) of a key -> 8 fp16 pairs
 // in coordinate order.  3-bit layout: half 0 is in the nibbles of w0, w1; half 1
 // in w2 and in the spare fourth bits of w0..w2.  2-bit layout: half h is word h,
-// whose low nibbles hold coordinate pairs (4i, 4i+1) and high nibbles (4i+2, 4i+3).
+// byte i holding coordinates 4i .. 4i+3.
 template <int BM>
 __device__ __forceinline__ void decode_half(const uint32_t* w, int half, uint32_t tab, uint32_t off3,
                                             uint32_t off2, uint32_t (&h)[8]) {
@@ -100,13 +106,13 @@ __device__ __forceinline__ void decode_half(const uint32_t* w, int half, uint32_
     lookup4(wa, tab, off3, h);
     lookup4(wb, tab, off3, h + 4);
   } else {
+    // one byte = four 2-bit codes = two fp16 pairs: one 8-byte lookup per byte
     const uint32_t x = half ? w[1] : w[0];
-    const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
-    uint32_t a[4], b[4];
-    lookup4(lo, tab, off2, a);
-    lookup4(hi, tab, off2, b);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) h[2 * i] = a[i], h[2 * i + 1] = b[i];
+    for (int i = 0; i < 4; ++i) {
+      const uint2 v = lds64(tab + prmt(x, off2, 0x5504 | (i << 4)));
+      h[2 * i] = v.x, h[2 * i + 1] = v.y;
+    }
   }
 }
 
@@ -123,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
   using L = LgLayout<BM0, BM1>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stages = smem;
-  uint8_t* ktab = smem + kStages * L::Stage;   // row B: [3-bit pair, one copy per lane][2-bit pair, one per lane]
+  uint8_t* ktab = smem + kStages * L::Stage;   // row B: [3-bit pair, one copy per lane][2-bit pair pair, 16 copies]
   uint8_t* sgtab = ktab + kTabBytes;           // row B: 16 copies of the four +-1 pairs of B's bits
   float* obuf = reinterpret_cast<float*>(sgtab + kTabBytes);  // [kCons][4 heads][16 tokens]
   uint64_t* full = reinterpret_cast<uint64_t*>(obuf + kCons * 64);
@@ -148,8 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
     for (int w = threadIdx.x; w < kTabBytes / 4; w += blockDim.x) {
       const uint32_t row = (uint32_t)w >> 6, col = (uint32_t)w & 63u;
       uint32_t v;
-      if (col < 32) v = ctab_half(a.ctab[g3], row & 7u) | (ctab_half(a.ctab[g3], (row >> 4) & 7u) << 16);
-      else v = ctab_half(a.ctab[g2], row & 3u) | (ctab_half(a.ctab[g2], (row >> 2) & 3u) << 16);
+      if (col < 32) {
+        v = ctab_half(a.ctab[g3], row & 7u) | (ctab_half(a.ctab[g3], (row >> 4) & 7u) << 16);
+      } else {
+        // (c[b0], c[b1]) in the low word, (c[b2], c[b3]) in the high word of each 8-byte copy
+        const uint32_t sh = (col & 1u) ? 4u : 0u;
+        v = ctab_half(a.ctab[g2], (row >> sh) & 3u) | (ctab_half(a.ctab[g2], (row >> (sh + 2)) & 3u) << 16);
+      }
       kt[w] = v;
     }
     uint32_t* sg = reinterpret_cast<uint32_t*>(sgtab);
@@ -198,12 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
     // lane's accumulator columns 2c, 2c + 1 belong to channel group c >> 1 as well
     const int half = c & 1, grp_of_c = c >> 1;
     const uint32_t kt = smem_u32(ktab), sgt = smem_u32(sgtab);
-    const uint32_t off3 = (uint32_t)lane * 4u, off2 = 128u + (uint32_t)lane * 4u;
+    const uint32_t off3 = (uint32_t)lane * 4u, off2 = 128u + (uint32_t)(lane & 15) * 8u;
     const uint32_t s_off = (uint32_t)(lane & 15) * 16u;
     float* ob = obuf + cw * 64;
     uint32_t qh[8][2], ql[8][2], qq[8][2];
     float isq[2][2];  // [head j][0: q' pieces, 1: q''] for this lane's accumulator columns
     int64_t cur_bh = -1, q0 = 0;
+    int stg = 0;
+    uint32_t phase = 0u;
     bool ok = true;
     BlockCursor cur;
     cur.init(gb_lo, a.nblk);
@@ -236,8 +249,10 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
           isq[j][1] = qs[1] * kQjl64;
         }
       }
-      const int s = (int)(i % kStages);
-      if (!mbar_wait(&full[s], (uint32_t)((i / kStages) & 1))) {
+      const int s = stg;
+      const uint32_t ph = phase;
+      if (++stg == kStages) stg = 0, phase ^= 1u;
+      if (!mbar_wait(&full[s], ph)) {
         ok = false;
         break;
       }
@@ -249,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
       const int64_t row0 = bh * a.kv_stride + t0;
       // the words of this lane's code groups for tokens g and g + 8
       uint32_t w0[2][3], w1[2][3], sw0[2], sw1[2];
-      float nn[2][2], rr[2][2];  // [token][group]
+      float nn[2], rr[2];  // [token], of the lane's accumulator group
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int tok = tb + g + 8 * r;
@@ -263,10 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
           }
           sw0[r] = reinterpret_cast<const uint32_t*>(st + L::S0)[tok * 2 + grp_of_c];
           sw1[r] = reinterpret_cast<const uint32_t*>(st + L::S1)[tok * 2 + grp_of_c];
-          nn[r][0] = reinterpret_cast<const float*>(st + L::N0)[tok];
-          rr[r][0] = reinterpret_cast<const float*>(st + L::R0)[tok];
-          nn[r][1] = reinterpret_cast<const float*>(st + L::N1)[tok];
-          rr[r][1] = reinterpret_cast<const float*>(st + L::R1)[tok];
+          nn[r] = reinterpret_cast<const float*>(st + (grp_of_c ? L::N1 : L::N0))[tok];
+          rr[r] = reinterpret_cast<const float*>(st + (grp_of_c ? L::R1 : L::R0))[tok];
         } else if (tok < n) {
           const int64_t rw = row0 + tok;
           const uint32_t* c0 = a.codes[0] + rw * L::W0 + grp_of_c * BM0;
@@ -278,13 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
           }
           sw0[r] = a.signs[0][rw * 2 + grp_of_c];
           sw1[r] = a.signs[1][rw * 2 + grp_of_c];
-          nn[r][0] = a.norms[0][rw], rr[r][0] = a.rnorms[0][rw];
-          nn[r][1] = a.norms[1][rw], rr[r][1] = a.rnorms[1][rw];
+          nn[r] = (grp_of_c ? a.norms[1] : a.norms[0])[rw];
+          rr[r] = (grp_of_c ? a.rnorms[1] : a.rnorms[0])[rw];
         } else {
 #pragma unroll
           for (int k = 0; k < 3; ++k) w0[r][k] = w1[r][k] = 0u;
           sw0[r] = sw1[r] = 0u;
-          nn[r][0] = nn[r][1] = rr[r][0] = rr[r][1] = 0.f;
+          nn[r] = rr[r] = 0.f;
         }
       }
       // codebook dots (k-steps 0-3 group 0, 4-7 group 1), q' as hi + lo
@@ -324,9 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
       const float ia = grp_of_c ? a.inv_alpha[1] : a.inv_alpha[0];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        // selects, not indexing: a runtime index would put the arrays in local memory
-        const float nr = grp_of_c ? nn[r][1] : nn[r][0];
-        const float rn = grp_of_c ? rr[r][1] : rr[r][0];
+        const float nr = nn[r], rn = rr[r];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int e = 2 * r + j;
