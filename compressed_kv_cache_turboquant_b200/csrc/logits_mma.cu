@@ -214,6 +214,18 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
     float* ob = obuf + cw * 64;
     uint32_t qh[8][2], ql[8][2], qq[8][2];
     float isq[2][2];  // [head j][0: q' pieces, 1: q''] for this lane's accumulator columns
+    // byte offsets within a stage of this lane's words for tokens g and g + 8
+    uint32_t o_c0[2], o_c1[2], o_s0[2], o_s1[2], o_n[2], o_r[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int tok = cw * 16 + g + 8 * r;
+      o_c0[r] = L::C0 + (tok * L::W0 + grp_of_c * BM0) * 4;
+      o_c1[r] = L::C1 + (tok * L::W1 + grp_of_c * BM1) * 4;
+      o_s0[r] = L::S0 + (tok * 2 + grp_of_c) * 4;
+      o_s1[r] = L::S1 + (tok * 2 + grp_of_c) * 4;
+      o_n[r] = (grp_of_c ? L::N1 : L::N0) + tok * 4;
+      o_r[r] = (grp_of_c ? L::R1 : L::R0) + tok * 4;
+    }
     int64_t cur_bh = -1, q0 = 0;
     int stg = 0;
     uint32_t phase = 0u;
@@ -265,6 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
       // the words of this lane's code groups for tokens g and g + 8
       uint32_t w0[2][3], w1[2][3], sw0[2], sw1[2];
       float nn[2], rr[2];  // [token], of the lane's accumulator group
+      if (n4 == kBlk) {
+        // whole block in the stage (every block but a context's last): fixed per-lane offsets
+        const uint32_t sb = smem_u32(st);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            w0[r][k] = k < BM0 ? lds32(sb + o_c0[r] + 4 * k) : 0u;
+            w1[r][k] = k < BM1 ? lds32(sb + o_c1[r] + 4 * k) : 0u;
+          }
+          sw0[r] = lds32(sb + o_s0[r]);
+          sw1[r] = lds32(sb + o_s1[r]);
+          nn[r] = __uint_as_float(lds32(sb + o_n[r]));
+          rr[r] = __uint_as_float(lds32(sb + o_r[r]));
+        }
+      } else
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int tok = tb + g + 8 * r;
