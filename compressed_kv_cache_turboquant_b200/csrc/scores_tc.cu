@@ -103,8 +103,26 @@ __device__ __forceinline__ uint32_t ctab_at(const ScArgs& a, uint32_t k) {
 
 // one group of 32 coordinates (BM words) -> 16 fp16 pairs (coordinate order)
 // of the scaled codebook, by byte-indexed lookups in per-lane table copies
+__device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_s128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// (the table addresses below are 32-bit shared-window addresses: this kernel aligns its
+// shared base through an integer, after which plain pointers would compile to generic loads)
 template <int BM>
-__device__ __forceinline__ void decode_mse32(const uint32_t* p, const uint8_t* tab, int lane, uint32_t (&o)[16]) {
+__device__ __forceinline__ void decode_mse32(const uint32_t* p, uint32_t tab, int lane, uint32_t (&o)[16]) {
   if constexpr (BM == 3) {
     const uint32_t s3 = ((p[0] >> 3) & 0x11111111u) | ((p[1] >> 2) & 0x22222222u) | ((p[2] >> 1) & 0x44444444u);
     const uint32_t ws[4] = {p[0], p[1], p[2], s3};
@@ -112,20 +130,20 @@ __device__ __forceinline__ void decode_mse32(const uint32_t* p, const uint8_t* t
     for (int q = 0; q < 4; ++q)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        o[4 * q + i] = *reinterpret_cast<const uint32_t*>(tab + ((ws[q] >> (8 * i)) & 0xFFu) * 128 + lane * 4);
+        o[4 * q + i] = ld_s32(tab + ((ws[q] >> (8 * i)) & 0xFFu) * 128 + lane * 4);
   } else if constexpr (BM == 2) {
 #pragma unroll
     for (int k = 0; k < 2; ++k)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint2 v = *reinterpret_cast<const uint2*>(tab + ((p[k] >> (8 * i)) & 0xFFu) * 128 + (lane & 15) * 8);
+        const uint2 v = ld_s64(tab + ((p[k] >> (8 * i)) & 0xFFu) * 128 + (lane & 15) * 8);
         o[8 * k + 2 * i] = v.x;
         o[8 * k + 2 * i + 1] = v.y;
       }
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(tab + ((p[0] >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
+      const uint4 v = ld_s128(tab + ((p[0] >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
       o[4 * i + 0] = v.x;
       o[4 * i + 1] = v.y;
       o[4 * i + 2] = v.z;
@@ -135,10 +153,10 @@ __device__ __forceinline__ void decode_mse32(const uint32_t* p, const uint8_t* t
 }
 
 // 32 sign bits -> 16 fp16 pairs of +-1
-__device__ __forceinline__ void decode_sign32(uint32_t sw, const uint8_t* tab, int lane, uint32_t (&o)[16]) {
+__device__ __forceinline__ void decode_sign32(uint32_t sw, uint32_t tab, int lane, uint32_t (&o)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 v = *reinterpret_cast<const uint4*>(tab + ((sw >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
+    const uint4 v = ld_s128(tab + ((sw >> (8 * i)) & 0xFFu) * 128 + (lane & 7) * 16);
     o[4 * i + 0] = v.x;
     o[4 * i + 1] = v.y;
     o[4 * i + 2] = v.z;
@@ -389,9 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
           } else if (!qpart) {
             const uint4 w = *reinterpret_cast<const uint4*>(slot + 4 * gj);
             const uint32_t p[3] = {w.x, w.y, w.z};
-            decode_mse32<BM>(p, mtab, lane, o);
+            decode_mse32<BM>(p, smem_u32(mtab), lane, o);
           } else {
-            decode_sign32(slot[4 * gj], stab, lane, o);
+            decode_sign32(slot[4 * gj], smem_u32(stab), lane, o);
           }
           // 16-byte units 4 gj .. 4 gj + 3 of the key's row, 128B-swizzled
 #pragma unroll
