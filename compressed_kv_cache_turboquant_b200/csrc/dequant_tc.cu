@@ -14,7 +14,8 @@
 //   1..4   decoders: one thread per vector unpacks its codes, looks the two
 //          fp16 pieces up in a 16-entry table and writes them into the
 //          128B-swizzled K-major A tiles (double-buffered)
-//   5..8   epilogue: one thread per vector reads both accumulators from TMEM,
+//   5..12  epilogue, two warps per TMEM lane quarter taking half of the column
+//          chunks each: one thread per vector reads both accumulators from TMEM,
 //          combines and scales by n; each warp stages its 32 rows x 128 B
 //          column chunk in 128B-swizzled shared memory (two buffers) and
 //          writes it with one TMA tensor store, so global writes are whole
@@ -32,7 +33,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 288;  // 9 warps
+constexpr int kThreads = 416;  // 13 warps
 
 template <int D>
 struct DqShape {
@@ -45,7 +46,7 @@ struct DqShape {
   static constexpr int kTmemCols = (4 * D <= 256) ? 256 : 512;  // 2 buffers x 2 accumulators
   static constexpr int kMiscBytes = 1024;
   static constexpr int kStageOut = 32 * 128;  // one warp's output chunk: 32 rows x 128 B
-  static constexpr int kOutBytes = 4 * 2 * kStageOut;
+  static constexpr int kOutBytes = 8 * kStageOut;  // one staging box per epilogue warp
   static constexpr int kSmemBytes = 2 * kBBytes + kStages * 2 * kABytes + kOutBytes + kMiscBytes + 1024;
 };
 
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* b_s = smem;                      // [2 pieces][kBBytes]
   uint8_t* a_s = smem + 2 * S::kBBytes;     // [stage][2 pieces][kABytes]
-  uint8_t* o_s = a_s + S::kStages * 2 * S::kABytes;  // [4 warps][2][kStageOut], 1024-aligned
+  uint8_t* o_s = a_s + S::kStages * 2 * S::kABytes;  // [8 warps][kStageOut], 1024-aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(o_s + S::kOutBytes);
   uint64_t* a_full = bars;              // [2]  decoders -> MMA (count 128)
   uint64_t* a_empty = bars + 2;         // [2]  MMA commit -> decoders
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       mbar_init(&a_full[s], 128);
       mbar_init(&a_empty[s], 1);
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);
+      mbar_init(&acc_empty[s], 8);
     }
     mbar_init(b_bar, 1);
     mbar_init(done_bar, 1);
@@ -213,10 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       mbar_arrive(&a_full[s]);
     }
   } else {
-    // epilogue: warp % 4 selects the TMEM lane quarter
+    // epilogue: warp % 4 selects the TMEM lane quarter, (warp - 5) / 4 the half of the chunks
     const int quarter = warp & 3;
+    const int part = (warp - 5) >> 2;
     const int r = quarter * 32 + lane;
-    uint8_t* stage = o_s + quarter * 2 * S::kStageOut;
+    uint8_t* buf = o_s + (warp - 5) * S::kStageOut;
     constexpr int kCols = 32;  // fp32 columns per 128-byte chunk (bf16: 64)
     int nst = 0;
     int i = 0;
@@ -233,10 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       tc_fence_after();
       const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 2 * D);
       const int nchunks = a.out_bf16 ? D / 64 : D / 32;
-      for (int c = 0; c < nchunks; ++c, ++nst) {
-        uint8_t* buf = stage + (nst & 1) * S::kStageOut;
-        // the store issued from this buffer two chunks ago must have read it
-        if (lane == 0) bulk_wait_read<1>();
+      const int c_lo = part * (nchunks / 2), c_hi = (nchunks == 1) ? (part == 0 ? 1 : 0) : c_lo + nchunks / 2;
+      for (int c = c_lo; c < c_hi; ++c, ++nst) {
+        // the previous store from this warp's buffer must have read it
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
         uint32_t pk[32];
         if (a.out_bf16) {
