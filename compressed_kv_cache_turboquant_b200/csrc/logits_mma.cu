@@ -18,10 +18,10 @@
 // numbers; the rotated queries enter as two fp16 pieces (hi + lo), the
 // projected queries as one; norms and scales are applied in fp32.
 //
-// Persistent CTAs own equal contiguous ranges of 192-token blocks over all
+// Persistent CTAs own equal contiguous ranges of 240-token blocks over all
 // (batch, kv-head) pairs; warp 0 bulk-copies each block (codes, signs and the
-// four norm arrays of both groups) into a ring; 12 consumer warps take 16
-// tokens each and write the block's 4 x 192 logits.
+// four norm arrays of both groups) into a ring; 15 consumer warps take 16
+// tokens each and write the block's 4 x 240 logits.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -37,9 +37,9 @@ namespace {
 using namespace sm100;
 using namespace frag;
 
-constexpr int kCons = 12;     // consumer warps (three per SM sub-partition)
+constexpr int kCons = 15;     // consumer warps (with the producer, four per SM sub-partition)
 constexpr int kBlk = 16 * kCons;  // tokens per stage, 16 per consumer warp
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kTabBytes = 256 * 256;
 constexpr float kQjl64 = 1.2533141373155003f / 64.f;
