@@ -8,7 +8,8 @@
 // over all (batch, kv-head) pairs; the 4 query heads of a kv-head's group share
 // every key and value read.
 //   warp 0      producer: bulk copies of each block (K codes, QJL signs, V codes
-//               and the three norm arrays) into a 2-stage ring
+//               and the three norm arrays) into a 4-stage ring (three blocks in
+//               flight while the consumers work on the fourth)
 //   warps 1-12  consumers (three per SM sub-partition), 16 tokens of every block each:
 //     logits   mma.sync m16n8k16 (fp16 in, fp32 accumulate), keys as M, the
 //              K dimension = 128 mse coordinates then 128 QJL coordinates,
@@ -42,7 +43,7 @@ using namespace frag;
 constexpr int D = 128;
 constexpr int kCons = 12;      // consumer warps (three per SM sub-partition)
 constexpr int kBlk = 16 * kCons;  // tokens per stage (16 per consumer warp)
-constexpr int kStages = 2;
+constexpr int kStages = 4;
 constexpr int kThreads = 32 * (1 + kCons);
 constexpr int kKW = 12;        // K code words per token (3 bits x 128 / 32)
 constexpr int kSW = 4;         // sign words
@@ -61,12 +62,18 @@ static_assert(kStageBytes % 16 == 0 && kOffS % 16 == 0 && kOffV % 16 == 0 && kOf
 //   KV table, row B: [K entry, one 4-byte copy per lane][V entry, one per lane]
 //     K entry = fp16 pair (cK[B & 7], cK[(B >> 4) & 7])   (3-bit codes; bits 3, 7 ignored)
 //     V entry = fp16 pair (cV[B & 15], cV[B >> 4])         (4-bit codes)
-//   sign table, row B: 16 copies of 16 bytes = four fp16 pairs (s0,s1)..(s6,s7),
+//   sign table, row B: 8 copies of 16 bytes = four fp16 pairs (s0,s1)..(s6,s7),
 //     s_i = +1.0 if bit i of B is set, else -1.0
-// With a copy per lane (per 16-byte lane group for the sign rows) the lookups
-// of a warp never meet in a bank, and the address of a lookup is one byte
-// permute: (code byte) << 8 | (lane offset).
+// With a copy per lane the 32-bit lookups of a warp never meet in a bank, and
+// the address of a lookup is one byte permute: (code byte) << 8 | (lane
+// offset).  A 16-byte load is served a quarter-warp at a time, so 8 copies of
+// a sign row (one per lane of a quarter) are enough; its address is
+// (sign byte) << 7 | (lane offset), a shift and a masked merge.
 constexpr int kTabBytes = 256 * 256;
+constexpr int kSgTabBytes = 256 * 128;
+constexpr int kSmemBytes = kStages * kStageBytes + kTabBytes + kSgTabBytes + (2 * kStages + 2) * 8 + kCons * 64 * 2 +
+                           kCons * 4 * (2 + D) * 4;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 4.0f;        // rescale only when a logit passes the running max by 2^4
 constexpr float kPScale = 0.0625f;   // fp16 weights p * ||v|| / 16 stay below ||v||
@@ -110,11 +117,13 @@ __device__ __forceinline__ void decode_k3(uint32_t w0, uint32_t w1, uint32_t w2,
   lookup4(s3, tab, lane_off, h + 12);
 }
 
-// 32 QJL sign bits -> 16 fp16 pairs (+-1.0) in coordinate order
+// 32 QJL sign bits -> 16 fp16 pairs (+-1.0) in coordinate order; `lane_off` =
+// (lane & 7) * 16, the lane's copy within a 128-byte sign row
 __device__ __forceinline__ void decode_signs(uint32_t w, uint32_t tab, uint32_t lane_off, uint32_t (&h)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint4 v = lds128(tab + prmt(w, lane_off, 0x5504 | (i << 4)));
+    const uint32_t row = (i == 0) ? (w << 7) : (w >> (8 * i - 7));  // byte i at bits 7..14
+    const uint4 v = lds128(tab + ((row & 0x7F80u) | lane_off));
     h[4 * i + 0] = v.x, h[4 * i + 1] = v.y, h[4 * i + 2] = v.z, h[4 * i + 3] = v.w;
   }
 }
@@ -124,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
   uint8_t* stages = smem;
   uint8_t* kvtab = smem + kStages * kStageBytes;
   uint8_t* sgtab = kvtab + kTabBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sgtab + kTabBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sgtab + kSgTabBytes);
   uint64_t* empty = full + kStages;
   uint64_t* pub = empty + kStages;                                        // consumer sync at segment ends
   __half* pbuf = reinterpret_cast<__half*>(pub + 2);                     // [kCons][4 heads][16 tokens]
@@ -152,8 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
                          : ((a.vlut[row & 15u] & 0xFFFFu) | (a.vlut[row >> 4] << 16));
     }
     uint32_t* sg = reinterpret_cast<uint32_t*>(sgtab);
-    for (int w = threadIdx.x; w < kTabBytes / 4; w += blockDim.x) {
-      const uint32_t row = (uint32_t)w >> 6, pair = (uint32_t)w & 3u;
+    for (int w = threadIdx.x; w < kSgTabBytes / 4; w += blockDim.x) {
+      const uint32_t row = (uint32_t)w >> 5, pair = (uint32_t)w & 3u;
       const uint32_t lo = ((row >> (2 * pair)) & 1u) ? 0x3C00u : 0xBC00u;
       const uint32_t hi = ((row >> (2 * pair + 1)) & 1u) ? 0x3C00u : 0xBC00u;
       sg[w] = lo | (hi << 16);
@@ -197,13 +206,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
     const int group = a.Hq / a.Hkv;    // 4
     const uint32_t kvt = smem_u32(kvtab), sgt = smem_u32(sgtab);
     const uint32_t k_off = (uint32_t)lane * 4u, v_off = 128u + (uint32_t)lane * 4u;
-    const uint32_t s_off = (uint32_t)(lane & 15) * 16u;
-    uint32_t bm[8][2], bq[8][2];
+    const uint32_t s_off = (uint32_t)(lane & 7) * 16u;
+    // Value MMA k index -> token: k and k ^ 1 trade places in the pairs that
+    // lanes c = 2, 3 hold, so that at each value-code load half the lanes of
+    // a half-warp read even tokens and half odd ones (64-byte rows: two bank
+    // groups instead of one).  The weights are stored in the same order.
+    const int vsw = c >> 1;
+    const int pslot = g ^ ((g >> 2) & 1);  // position of tokens g, g + 8 among the k indices
+    // this lane's byte offsets within a stage (tokens of warp cw start at 16 cw)
+    const int tb = cw * 16;
+    const uint32_t o_k = kOffK + (uint32_t)((tb + g) * kKW + 3 * c) * 4u;    // +0, +4, +8; key g + 8 at +8 kKW words
+    const uint32_t o_s = kOffS + (uint32_t)((tb + g) * kSW + c) * 4u;        // key g + 8 at +8 kSW words
+    const uint32_t o_va = kOffV + (uint32_t)((tb + 2 * c + vsw) * kVW + 2 * g) * 4u;      // +8 tokens: +8 kVW words
+    const uint32_t o_vb = kOffV + (uint32_t)((tb + 2 * c + 1 - vsw) * kVW + 2 * g) * 4u;
+    const uint32_t o_n = kOffN + (uint32_t)(tb + g) * 4u;                   // R and VN follow at +kBlk floats
+    const uint32_t st0 = smem_u32(stages);
+    int stg = 0;
+    uint32_t phase = 0u;
+    uint32_t bf[8][2];  // query B fragments: q' of head g (g < 4), q'' of head g - 4 (g >= 4)
     float inv_s1[2], inv_s2[2];
     float m_ref[2], l_run[2];
     float acc[8][4];
     __half* pb = pbuf + cw * 64;
-    int64_t cur_bh = -1;
     int seg = -1;
     bool ok = true;
 
@@ -259,25 +283,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
 
     BlockCursor cur;
     cur.init(gb_lo, a.nblk);
-    for (int64_t gb = gb_lo, i = 0; ok && gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
+    const int nblocks = (int)(gb_hi - gb_lo);
+    for (int it = 0; ok && it < nblocks; ++it, cur.next(a.nblk)) {
       const int64_t bh = cur.bh;
-      if (bh != cur_bh) {
+      if (it == 0 || cur.blk == 0) {  // a new (batch, kv-head) segment
         if (seg >= 0) flush(seg);
         if (!ok) break;
         ++seg;
-        cur_bh = bh;
-        // queries of this (batch, kv-head): mse columns 0-3 (q' of head g), QJL columns 4-7 (q'' of head g-4)
+        // queries of this (batch, kv-head): columns 0-3 q' of the 4 heads, columns 4-7 q''; both MMA passes
+        // take all 8 columns, the code pass is read from columns 0-3 and the sign pass from columns 4-7
         const int64_t b = bh / a.Hkv, hh = bh - b * a.Hkv;
         const int64_t q0 = b * a.Hq + hh * group;
         const uint32_t* qf = a.qfrag + (q0 + (g & 3)) * 2 * 64;
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
-          const uint2 vm = *reinterpret_cast<const uint2*>(qf + 16 * c + 2 * kb);
-          const uint2 vq = *reinterpret_cast<const uint2*>(qf + 64 + 16 * c + 2 * kb);
-          bm[kb][0] = (g < 4) ? vm.x : 0u;
-          bm[kb][1] = (g < 4) ? vm.y : 0u;
-          bq[kb][0] = (g >= 4) ? vq.x : 0u;
-          bq[kb][1] = (g >= 4) ? vq.y : 0u;
+          const uint2 v = *reinterpret_cast<const uint2*>(qf + (g < 4 ? 0 : 64) + 16 * c + 2 * kb);
+          bf[kb][0] = v.x;
+          bf[kb][1] = v.y;
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -291,51 +313,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
       }
-      const int s = (int)(i % kStages);
-      const uint32_t u = (uint32_t)(i / kStages);
-      if (!mbar_wait(&full[s], u & 1u)) {
+      const int s = stg;
+      if (!mbar_wait(&full[s], phase)) {
         ok = false;
         break;
       }
+      if (++stg == kStages) stg = 0, phase ^= 1u;
       const uint8_t* st = stages + s * kStageBytes;
+      const uint32_t sb = st0 + (uint32_t)(s * kStageBytes);
       const int64_t t0 = cur.blk * kBlk;
       const int n = (int)min((int64_t)kBlk, a.T - t0);
-      const int tb = cw * 16;  // this warp's 16 tokens within the block
       // ---------------- logits: keys g and g+8 of the sub-block
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      float sm[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
       {
         uint32_t h0[16], h1[16];
-        const uint32_t* kc0 = reinterpret_cast<const uint32_t*>(st + kOffK) + (tb + g) * kKW + 3 * c;
-        const uint32_t* kc1 = kc0 + 8 * kKW;
-        decode_k3(kc0[0], kc0[1], kc0[2], kvt, k_off, h0);
-        decode_k3(kc1[0], kc1[1], kc1[2], kvt, k_off, h1);
+        const uint32_t ka = sb + o_k, kb8 = ka + 8 * kKW * 4;
+        decode_k3(lds32(ka), lds32(ka + 4), lds32(ka + 8), kvt, k_off, h0);
+        decode_k3(lds32(kb8), lds32(kb8 + 4), lds32(kb8 + 8), kvt, k_off, h1);
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb)
-          mma16816(sc, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bm[kb][0], bm[kb][1]);
-        const uint32_t* sw = reinterpret_cast<const uint32_t*>(st + kOffS);
-        decode_signs(sw[(tb + g) * kSW + c], sgt, s_off, h0);
-        decode_signs(sw[(tb + g + 8) * kSW + c], sgt, s_off, h1);
+          mma16816(sm, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bf[kb][0], bf[kb][1]);
+        decode_signs(lds32(sb + o_s), sgt, s_off, h0);
+        decode_signs(lds32(sb + o_s + 8 * kSW * 4), sgt, s_off, h1);
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb)
-          mma16816(sc, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bq[kb][0], bq[kb][1]);
+          mma16816(sq, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bf[kb][0], bf[kb][1]);
       }
-      // lanes c and c^2 hold the mse and QJL dots of the same heads
+      // lane c < 2 holds the code dots of heads 2c, 2c+1 (columns 2c, 2c+1 of sm), lane c + 2 their sign dots
+      // (columns 4 + 2c, 5 + 2c of sq): each sends the half the other needs
       float ot[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) ot[e] = __shfl_xor_sync(0xffffffffu, sc[e], 2);
-      const float* mse = (c < 2) ? sc : ot;
-      const float* qjl = (c < 2) ? ot : sc;
+      for (int e = 0; e < 4; ++e) ot[e] = __shfl_xor_sync(0xffffffffu, (c < 2) ? sm[e] : sq[e], 2);
+      const float* mse = (c < 2) ? sm : ot;
+      const float* qjl = (c < 2) ? ot : sq;
       // norms of keys g and g+8; a partial last block reads its tail from global memory
       float kn[2], kr[2], vn[2];
       if (n == kBlk) {
-        const float* N0 = reinterpret_cast<const float*>(st + kOffN);
-        const float* R0 = reinterpret_cast<const float*>(st + kOffR);
-        const float* V0 = reinterpret_cast<const float*>(st + kOffVN);
+        const uint32_t na = sb + o_n;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          kn[r] = N0[tb + g + 8 * r];
-          kr[r] = R0[tb + g + 8 * r];
-          vn[r] = V0[tb + g + 8 * r];
+          kn[r] = __uint_as_float(lds32(na + 32 * r));
+          kr[r] = __uint_as_float(lds32(na + (kOffR - kOffN) + 32 * r));
+          vn[r] = __uint_as_float(lds32(na + (kOffVN - kOffN) + 32 * r));
         }
       } else {
         const int n4 = n & ~3;
@@ -395,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         const float p1 = v1 ? exp2f(lg[1][j] - m_ref[j]) : 0.f;
         l_run[j] += (p0 + p1) * kPScale;
         if (c < 2) {
-          pb[(2 * cp + j) * 16 + g] = __float2half_rn(p0 * vn[0] * kPScale);
-          pb[(2 * cp + j) * 16 + g + 8] = __float2half_rn(p1 * vn[1] * kPScale);
+          pb[(2 * cp + j) * 16 + pslot] = __float2half_rn(p0 * vn[0] * kPScale);
+          pb[(2 * cp + j) * 16 + pslot + 8] = __float2half_rn(p1 * vn[1] * kPScale);
         }
       }
       __syncwarp();
@@ -405,14 +424,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         pw0 = *reinterpret_cast<const uint32_t*>(pb + g * 16 + 2 * c);
         pw1 = *reinterpret_cast<const uint32_t*>(pb + g * 16 + 2 * c + 8);
       }
-      // ---------------- values: tokens 2c, 2c+1, 2c+8, 2c+9; coordinates 16g .. 16g+15
+      // ---------------- values: k indices 2c, 2c+1, 2c+8, 2c+9 (tokens k ^ vsw); coordinates 16g .. 16g+15
       {
-        const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + kOffV);
         uint32_t xa[8], xb[8], xc[8], xd[8];
-        const uint2 wa = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c) * kVW + 2 * g);
-        const uint2 wb = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 1) * kVW + 2 * g);
-        const uint2 wc = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 8) * kVW + 2 * g);
-        const uint2 wd = *reinterpret_cast<const uint2*>(vc + (tb + 2 * c + 9) * kVW + 2 * g);
+        const uint2 wa = lds64(sb + o_va);
+        const uint2 wb = lds64(sb + o_vb);
+        const uint2 wc = lds64(sb + o_va + 8 * kVW * 4);
+        const uint2 wd = lds64(sb + o_vb + 8 * kVW * 4);
         lookup4(wa.x, kvt, v_off, xa);
         lookup4(wa.y, kvt, v_off, xa + 4);
         lookup4(wb.x, kvt, v_off, xb);
@@ -544,8 +562,7 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.partials = partials;
   a.status = hk->dev.status;
   const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
-  const int smem = kStages * kStageBytes + 2 * kTabBytes + (2 * kStages + 2) * 8 + kCons * 64 * 2 +
-                   kCons * 4 * (2 + D) * 4;
+  const int smem = kSmemBytes;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -86,12 +86,6 @@ __device__ __forceinline__ uint32_t ctab_half(const uint32_t (&t)[8], uint32_t k
   return (t[k >> 1] >> (16 * (k & 1u))) & 0xFFFFu;
 }
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
 // 16 coordinates (one half of a 32-coordinate group) of a key -> 8 fp16 pairs
 // in coordinate order.  3-bit layout: half 0 is in the nibbles of w0, w1; half 1
 // in w2 and in the spare fourth bits of w0..w2.  2-bit layout: half h is word h,
