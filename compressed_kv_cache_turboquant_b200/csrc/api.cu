@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -321,6 +322,12 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess && K > 1)
     e = cudaMemcpy(h->dev.thresholds, tf.data(), (K - 1) * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(h->dev.status, 0, 256);
+  {
+    // TQ_RUNTIME_TABLE_ADDRESSES=1 keeps the kernels that add table addresses at run time
+    const char* ev = getenv("TQ_RUNTIME_TABLE_ADDRESSES");
+    if (e == cudaSuccess && !(ev && ev[0] == '1'))
+      e = (cudaError_t)probe_dyn_smem_base((uint32_t*)(h->dev.status + 16), &h->dyn_base);
+  }
   if (e == cudaSuccess && tc)
     e = cudaMemcpy(h->dev.pi_tc, pieces.data(), pieces.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && tc)

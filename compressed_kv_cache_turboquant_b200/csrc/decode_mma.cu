@@ -107,29 +107,40 @@ __host__ __device__ __forceinline__ int64_t cta_first_block(int64_t i, int64_t t
 }
 
 // one 3-bit group of 32 coordinates (words w0..w2, layout of tq.h) -> 16 fp16 pairs in coordinate order
+template <uint32_t ADDR>
 __device__ __forceinline__ void decode_k3(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t tab, uint32_t lane_off,
                                           uint32_t (&h)[16]) {
   // coordinates 24..31 live in the fourth bit of every nibble of w0..w2
   const uint32_t s3 = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
-  lookup4(w0, tab, lane_off, h + 0);
-  lookup4(w1, tab, lane_off, h + 4);
-  lookup4(w2, tab, lane_off, h + 8);
-  lookup4(s3, tab, lane_off, h + 12);
+  lookup4<ADDR>(w0, tab, lane_off, h + 0);
+  lookup4<ADDR>(w1, tab, lane_off, h + 4);
+  lookup4<ADDR>(w2, tab, lane_off, h + 8);
+  lookup4<ADDR>(s3, tab, lane_off, h + 12);
 }
 
 // 32 QJL sign bits -> 16 fp16 pairs (+-1.0) in coordinate order; `lane_off` =
 // (lane & 7) * 16, the lane's copy within a 128-byte sign row
+template <uint32_t ADDR>
 __device__ __forceinline__ void decode_signs(uint32_t w, uint32_t tab, uint32_t lane_off, uint32_t (&h)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t row = (i == 0) ? (w << 7) : (w >> (8 * i - 7));  // byte i at bits 7..14
-    const uint4 v = lds128(tab + ((row & 0x7F80u) | lane_off));
+    const uint4 v = tab_ld128<ADDR>(tab, (row & 0x7F80u) | lane_off);
     h[4 * i + 0] = v.x, h[4 * i + 1] = v.y, h[4 * i + 2] = v.z, h[4 * i + 3] = v.w;
   }
 }
 
+// DB: shared address of the dynamic window (the tables' addresses become load
+// immediates), or kDynRuntime (table addresses added at run time)
+template <uint32_t DB>
 __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
+  constexpr uint32_t KV = tab_addr(DB, kStages * kStageBytes);
+  constexpr uint32_t SG = tab_addr(DB, kStages * kStageBytes + kTabBytes);
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (DB != kDynRuntime && smem_u32(smem) != DB) {  // not the window this instance was built for
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusLayout);
+    return;
+  }
   uint8_t* stages = smem;
   uint8_t* kvtab = smem + kStages * kStageBytes;
   uint8_t* sgtab = kvtab + kTabBytes;
@@ -328,13 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
       {
         uint32_t h0[16], h1[16];
         const uint32_t ka = sb + o_k, kb8 = ka + 8 * kKW * 4;
-        decode_k3(lds32(ka), lds32(ka + 4), lds32(ka + 8), kvt, k_off, h0);
-        decode_k3(lds32(kb8), lds32(kb8 + 4), lds32(kb8 + 8), kvt, k_off, h1);
+        decode_k3<KV>(lds32(ka), lds32(ka + 4), lds32(ka + 8), kvt, k_off, h0);
+        decode_k3<KV>(lds32(kb8), lds32(kb8 + 4), lds32(kb8 + 8), kvt, k_off, h1);
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb)
           mma16816(sm, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bf[kb][0], bf[kb][1]);
-        decode_signs(lds32(sb + o_s), sgt, s_off, h0);
-        decode_signs(lds32(sb + o_s + 8 * kSW * 4), sgt, s_off, h1);
+        decode_signs<SG>(lds32(sb + o_s), sgt, s_off, h0);
+        decode_signs<SG>(lds32(sb + o_s + 8 * kSW * 4), sgt, s_off, h1);
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb)
           mma16816(sq, h0[2 * kb], h1[2 * kb], h0[2 * kb + 1], h1[2 * kb + 1], bf[kb][0], bf[kb][1]);
@@ -431,14 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         const uint2 wb = lds64(sb + o_vb);
         const uint2 wc = lds64(sb + o_va + 8 * kVW * 4);
         const uint2 wd = lds64(sb + o_vb + 8 * kVW * 4);
-        lookup4(wa.x, kvt, v_off, xa);
-        lookup4(wa.y, kvt, v_off, xa + 4);
-        lookup4(wb.x, kvt, v_off, xb);
-        lookup4(wb.y, kvt, v_off, xb + 4);
-        lookup4(wc.x, kvt, v_off, xc);
-        lookup4(wc.y, kvt, v_off, xc + 4);
-        lookup4(wd.x, kvt, v_off, xd);
-        lookup4(wd.y, kvt, v_off, xd + 4);
+        lookup4<KV>(wa.x, kvt, v_off, xa);
+        lookup4<KV>(wa.y, kvt, v_off, xa + 4);
+        lookup4<KV>(wb.x, kvt, v_off, xb);
+        lookup4<KV>(wb.y, kvt, v_off, xb + 4);
+        lookup4<KV>(wc.x, kvt, v_off, xc);
+        lookup4<KV>(wc.y, kvt, v_off, xc + 4);
+        lookup4<KV>(wd.x, kvt, v_off, xd);
+        lookup4<KV>(wd.y, kvt, v_off, xd + 4);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           // rows (coords 16g + 2mt, 16g + 2mt + 1), token pairs (2c, 2c+1) and (2c+8, 2c+9)
@@ -563,14 +574,16 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.status = hk->dev.status;
   const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
   const int smem = kSmemBytes;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const bool fixed = hk->dyn_base == kDynBaseSm100;
+  auto kern = fixed ? decode_mma_kernel<kDynBaseSm100> : decode_mma_kernel<kDynRuntime>;
+  static bool attr[2] = {false, false};
+  if (!attr[fixed]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return (int)e;
-    attr = true;
+    attr[fixed] = true;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  decode_mma_kernel<<<G, kThreads, smem, s>>>(a);
+  kern<<<G, kThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   decode_merge_persistent_kernel<<<B * Hq, 128, 0, s>>>(partials, G, a.max_seg, a.nblk, a.total, Hq, Hkv,
@@ -607,11 +620,28 @@ __global__ void qfrag_kernel(const float* qrot, const float* qproj, int64_t nq, 
   }
 }
 
+// Shared-memory address at which the dynamic window of a kernel without
+// static shared memory starts (written by one thread into `out`).
+__global__ void dyn_smem_base_kernel(uint32_t* out) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  if (threadIdx.x == 0) out[0] = sm100::smem_u32(dsm);
+}
+
 }  // namespace
 
 int launch_qfrag(const float* qrot, const float* qproj, int64_t nq, void* qfrag, float* qscale, void* stream) {
   qfrag_kernel<<<(unsigned)nq, 128, 0, (cudaStream_t)stream>>>(qrot, qproj, nq, (__half*)qfrag, qscale);
   return (int)cudaGetLastError();
+}
+
+// One launch of a 32-thread kernel with 16 bytes of dynamic shared memory;
+// `scratch` is 4 bytes of device memory.  Synchronous.  Returns a CUDA error
+// code; on success *base holds the address.
+int probe_dyn_smem_base(uint32_t* scratch, uint32_t* base) {
+  dyn_smem_base_kernel<<<1, 32, 16>>>(scratch);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpy(base, scratch, 4, cudaMemcpyDeviceToHost);
+  return (int)e;
 }
 
 }  // namespace tqi

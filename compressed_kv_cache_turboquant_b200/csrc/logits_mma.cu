@@ -90,38 +90,47 @@ __device__ __forceinline__ uint32_t ctab_half(const uint32_t (&t)[8], uint32_t k
 // in coordinate order.  3-bit layout: half 0 is in the nibbles of w0, w1; half 1
 // in w2 and in the spare fourth bits of w0..w2.  2-bit layout: half h is word h,
 // byte i holding coordinates 4i .. 4i+3.
-template <int BM>
+template <int BM, uint32_t ADDR>
 __device__ __forceinline__ void decode_half(const uint32_t* w, int half, uint32_t tab, uint32_t off3,
                                             uint32_t off2, uint32_t (&h)[8]) {
   if constexpr (BM == 3) {
     const uint32_t s3 = ((w[0] >> 3) & 0x11111111u) | ((w[1] >> 2) & 0x22222222u) | ((w[2] >> 1) & 0x44444444u);
     const uint32_t wa = half ? w[2] : w[0];
     const uint32_t wb = half ? s3 : w[1];
-    lookup4(wa, tab, off3, h);
-    lookup4(wb, tab, off3, h + 4);
+    lookup4<ADDR>(wa, tab, off3, h);
+    lookup4<ADDR>(wb, tab, off3, h + 4);
   } else {
     // one byte = four 2-bit codes = two fp16 pairs: one 8-byte lookup per byte
     const uint32_t x = half ? w[1] : w[0];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint2 v = lds64(tab + prmt(x, off2, 0x5504 | (i << 4)));
+      const uint2 v = tab_ld64<ADDR>(tab, prmt(x, off2, 0x5504 | (i << 4)));
       h[2 * i] = v.x, h[2 * i + 1] = v.y;
     }
   }
 }
 
 // 16 sign bits (bits 0..15 of w) -> 8 fp16 pairs of +-1
+template <uint32_t ADDR>
 __device__ __forceinline__ void decode_signs16(uint32_t w, uint32_t tab, uint32_t s_off, uint32_t (&h)[8]) {
-  const uint4 v0 = lds128(tab + prmt(w, s_off, 0x5504));
-  const uint4 v1 = lds128(tab + prmt(w, s_off, 0x5514));
+  const uint4 v0 = tab_ld128<ADDR>(tab, prmt(w, s_off, 0x5504));
+  const uint4 v1 = tab_ld128<ADDR>(tab, prmt(w, s_off, 0x5514));
   h[0] = v0.x, h[1] = v0.y, h[2] = v0.z, h[3] = v0.w;
   h[4] = v1.x, h[5] = v1.y, h[6] = v1.z, h[7] = v1.w;
 }
 
-template <int BM0, int BM1>
+// DB: shared address of the dynamic window (table addresses become load
+// immediates), or kDynRuntime
+template <int BM0, int BM1, uint32_t DB>
 __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
   using L = LgLayout<BM0, BM1>;
+  constexpr uint32_t KT = tab_addr(DB, kStages * L::Stage);
+  constexpr uint32_t SG = tab_addr(DB, kStages * L::Stage + kTabBytes);
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (DB != kDynRuntime && smem_u32(smem) != DB) {  // not the window this instance was built for
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusLayout);
+    return;
+  }
   uint8_t* stages = smem;
   uint8_t* ktab = smem + kStages * L::Stage;   // row B: [3-bit pair, one copy per lane][2-bit pair pair, 16 copies]
   uint8_t* sgtab = ktab + kTabBytes;           // row B: 16 copies of the four +-1 pairs of B's bits
@@ -326,28 +335,28 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
       float sm[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
       {
         uint32_t ha[8], hb[8];
-        decode_half<BM0>(w0[0], half, kt, off3, off2, ha);
-        decode_half<BM0>(w0[1], half, kt, off3, off2, hb);
+        decode_half<BM0, KT>(w0[0], half, kt, off3, off2, ha);
+        decode_half<BM0, KT>(w0[1], half, kt, off3, off2, hb);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           mma16816(sm, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], qh[kb][0], qh[kb][1]);
           mma16816(sm, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], ql[kb][0], ql[kb][1]);
         }
-        decode_half<BM1>(w1[0], half, kt, off3, off2, ha);
-        decode_half<BM1>(w1[1], half, kt, off3, off2, hb);
+        decode_half<BM1, KT>(w1[0], half, kt, off3, off2, ha);
+        decode_half<BM1, KT>(w1[1], half, kt, off3, off2, hb);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           mma16816(sm, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], qh[4 + kb][0], qh[4 + kb][1]);
           mma16816(sm, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], ql[4 + kb][0], ql[4 + kb][1]);
         }
         // sign dots: bits 16 half .. 16 half + 15 of the group's sign word
-        decode_signs16(sw0[0] >> (16 * half), sgt, s_off, ha);
-        decode_signs16(sw0[1] >> (16 * half), sgt, s_off, hb);
+        decode_signs16<SG>(sw0[0] >> (16 * half), sgt, s_off, ha);
+        decode_signs16<SG>(sw0[1] >> (16 * half), sgt, s_off, hb);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb)
           mma16816(sq, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], qq[kb][0], qq[kb][1]);
-        decode_signs16(sw1[0] >> (16 * half), sgt, s_off, ha);
-        decode_signs16(sw1[1] >> (16 * half), sgt, s_off, hb);
+        decode_signs16<SG>(sw1[0] >> (16 * half), sgt, s_off, ha);
+        decode_signs16<SG>(sw1[1] >> (16 * half), sgt, s_off, hb);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb)
           mma16816(sq, ha[2 * kb], hb[2 * kb], ha[2 * kb + 1], hb[2 * kb + 1], qq[4 + kb][0], qq[4 + kb][1]);
@@ -494,9 +503,10 @@ int launch_logits_mma(const tq_ctx* const* hk, const float* const* qrot, const f
   a.logits = logits;
   a.status = hk[0]->dev.status;
   const int grid = (int)(a.total < hk[0]->sm_count ? a.total : hk[0]->sm_count);
+  const bool fixed = hk[0]->dyn_base == kDynBaseSm100;
   auto go = [&](auto kern, int smem) -> int {
-    static bool set[4][4] = {};
-    bool& done = set[hk[0]->bm][hk[1]->bm];
+    static bool set[2][4][4] = {};
+    bool& done = set[fixed][hk[0]->bm][hk[1]->bm];
     if (!done) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return (int)e;
@@ -506,10 +516,14 @@ int launch_logits_mma(const tq_ctx* const* hk, const float* const* qrot, const f
     return (int)cudaGetLastError();
   };
   const int b0 = hk[0]->bm, b1 = hk[1]->bm;
-  if (b0 == 3 && b1 == 2) return go(logits_mma_kernel<3, 2>, LgLayout<3, 2>::Smem);
-  if (b0 == 2 && b1 == 3) return go(logits_mma_kernel<2, 3>, LgLayout<2, 3>::Smem);
-  if (b0 == 3 && b1 == 3) return go(logits_mma_kernel<3, 3>, LgLayout<3, 3>::Smem);
-  return go(logits_mma_kernel<2, 2>, LgLayout<2, 2>::Smem);
+  constexpr uint32_t F = kDynBaseSm100, R = kDynRuntime;
+  if (b0 == 3 && b1 == 2)
+    return fixed ? go(logits_mma_kernel<3, 2, F>, LgLayout<3, 2>::Smem) : go(logits_mma_kernel<3, 2, R>, LgLayout<3, 2>::Smem);
+  if (b0 == 2 && b1 == 3)
+    return fixed ? go(logits_mma_kernel<2, 3, F>, LgLayout<2, 3>::Smem) : go(logits_mma_kernel<2, 3, R>, LgLayout<2, 3>::Smem);
+  if (b0 == 3 && b1 == 3)
+    return fixed ? go(logits_mma_kernel<3, 3, F>, LgLayout<3, 3>::Smem) : go(logits_mma_kernel<3, 3, R>, LgLayout<3, 3>::Smem);
+  return fixed ? go(logits_mma_kernel<2, 2, F>, LgLayout<2, 2>::Smem) : go(logits_mma_kernel<2, 2, R>, LgLayout<2, 2>::Smem);
 }
 
 }  // namespace tqi

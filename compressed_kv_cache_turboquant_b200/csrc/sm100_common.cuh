@@ -16,6 +16,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // device status bits (written with atomicOr)
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusLayout = 2;  // a kernel built for fixed shared addresses found its window elsewhere
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

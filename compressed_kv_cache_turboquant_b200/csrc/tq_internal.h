@@ -68,12 +68,14 @@ struct tq_ctx {
   uint16_t sc_tab[16] = {0};
   float sc_inv_alpha = 1.f;
   int gen_d_pad = 0;
+  uint32_t dyn_base = 0xFFFFFFFFu;  // shared address of a kernel's dynamic window (probed at creation)
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 
 namespace tqi {
 
 // number of context splits tq_attn_decode uses for a (B, Hq, T) problem
+int probe_dyn_smem_base(uint32_t* scratch, uint32_t* base);
 int decode_splits(int B, int Hq, int64_t T, int sm_count);
 
 // ---- launchers (kernels_*.cu); all return cudaError_t as int ----

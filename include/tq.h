@@ -123,7 +123,12 @@ TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
  *   centroids  host in, [2^bm] ascending (bm = b for TQ_MSE, b-1 for TQ_PROD),
  *              or NULL to use tq_make_codebook(bm, d)
  * Allocates device memory for the constants on the current device (the only
- * allocation the library makes) and synchronises with it.
+ * allocation the library makes), launches one 32-thread kernel that reports
+ * where a kernel's dynamic shared-memory window starts (the decode and logits
+ * kernels address their lookup tables from it), and synchronises.  With the
+ * environment variable TQ_RUNTIME_TABLE_ADDRESSES=1 the probe is skipped and
+ * those kernels add the table addresses at run time (a slower instance of the
+ * same arithmetic).
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
  */
 TQ_API int tq_create(tq_handle* h, int d, int b, int variant, const double* Pi, const double* S,
@@ -350,10 +355,14 @@ TQ_API size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, 
  * tq_device_status -- read and clear the handle's device status word
  * (synchronous).  0 = no event.  Bit 0 (TQ_STATUS_TIMEOUT): a tensor-core
  * kernel gave up a wait on one of its own pipeline barriers after ~2 s and
- * returned early; its outputs for that call are incomplete.
+ * returned early; its outputs for that call are incomplete.  Bit 1
+ * (TQ_STATUS_LAYOUT): a decode or logits kernel built for the shared-memory
+ * address that tq_create measured found its dynamic shared window elsewhere
+ * and returned without writing its outputs.
  * Errors: TQ_EINVAL, TQ_ECUDA.
  */
 #define TQ_STATUS_TIMEOUT 1
+#define TQ_STATUS_LAYOUT 2
 TQ_API int tq_device_status(tq_handle h, int* status);
 
 /* tq_last_error -- message of the last failing call on this thread ("" if none). */

@@ -333,6 +333,13 @@ def test_decode_fallback_shapes():
     _decode_case(B=2, Hq=4, Hkv=2, T=500, d=128, sample=[(0, 1), (1, 0)], seed=4)
 
 
+def test_decode_runtime_table_addresses(monkeypatch):
+    """The decode kernel instance that adds its table addresses at run time (taken when the
+    dynamic shared window is not where the library expects it) agrees just the same."""
+    monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
+    _decode_case(B=2, Hq=8, Hkv=2, T=1531, d=128, sample=[(0, 1), (1, 0)], seed=5, stride_extra=5)
+
+
 # ------------------------------------------------------------------ channel groups (3.5-bit streaming cache)
 
 def _split_instances(d=128, n_hi=64, seed=0):
@@ -424,6 +431,11 @@ def _logits_case(B, Hq, Hkv, T, sample, seed=0):
 
 def test_split_group_logits_small_ragged():
     _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 0), (1, 1)], seed=1)
+
+
+def test_split_group_logits_runtime_table_addresses(monkeypatch):
+    monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
+    _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 1), (1, 0)], seed=2)
 
 
 def test_split_group_logits_full_context_sampled():
