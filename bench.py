@@ -361,14 +361,17 @@ class Stream:
                                signs=c["signs"][t:], rnorms=c["rnorms"][t:], out_stride=self.T)
         if record:
             e1.record(self.stream)
-        tq.tq_attn_logits(self.h, self.channels, self.q, self.Hkv, self.T, self.T,
-                          [c["codes"] for c in self.cache], [c["signs"] for c in self.cache],
-                          [c["norms"] for c in self.cache], [c["rnorms"] for c in self.cache],
-                          1.0 / math.sqrt(D), self.logits, self.ws)
+        self.logits_only()
         if record:
             e2.record(self.stream)
             self.app.append((e0, e1))
             self.lgt.append((e1, e2))
+
+    def logits_only(self):
+        self.tq.tq_attn_logits(self.h, self.channels, self.q, self.Hkv, self.T, self.T,
+                               [c["codes"] for c in self.cache], [c["signs"] for c in self.cache],
+                               [c["norms"] for c in self.cache], [c["rnorms"] for c in self.cache],
+                               1.0 / math.sqrt(D), self.logits, self.ws)
 
     def bytes_logits(self):
         # per token per kv-head: group A 24 B codes + 8 B signs + 8 B norms, group B 16 + 8 + 8, logits 4 x 4 B
@@ -615,6 +618,49 @@ def run_ours(args):
     ranks.close()
 
 
+PROFILE_CASES = {
+    "decode": "decode attention, config-4 shape at context --profile-t (default 32768)",
+    "logits": "split-cache logits, config-5 shape at context --profile-t (default 2^18)",
+    "search": "quantize + fused top-10 scoring: d = --search-d, --profile-n keys (default 200000), "
+              "--profile-nq queries (default 1280)",
+    "sweep": "the sweep step (quantize + dequantize at b = 1..4, 2^20 bf16 vectors)",
+}
+
+
+def run_profile_case(args):
+    """Small cases of the hot-path calls for ncu captures: set-up, then
+    --profile-launches calls of the case's step, and one JSON line with each
+    call's CUDA-event time.  Not a bench result."""
+    import torch
+    import compressed_kv_cache_turboquant_b200 as tq
+
+    torch.cuda.set_device(0)
+    dev, case = "cuda:0", args.profile_case
+    if case == "decode":
+        DEC["T"] = args.profile_t or 32768
+        wl = Decode(tq, torch, 0, dev)
+        call, size = wl.step, {"T": DEC["T"]}
+    elif case == "logits":
+        wl = Stream(tq, torch, 0, dev, T=args.profile_t or (1 << 18))
+        call, size = wl.logits_only, {"T": wl.T}
+    elif case == "search":
+        n, nq = args.profile_n or 200000, args.profile_nq or 1280
+        wl = Search(tq, torch, 0, dev, d=args.search_d, N=n, nq=nq)
+        call, size = wl.step, {"d": args.search_d, "N": n, "nq": nq}
+    else:
+        wl = Sweep(tq, torch, 0, dev)
+        call, size = wl.step, {"N": SWEEP_N}
+    ms = []
+    for _ in range(args.profile_launches):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    print(json.dumps({"profile_case": case, "what": PROFILE_CASES[case], "size": size, "ms": ms}), flush=True)
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -654,7 +700,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-search", action="store_true")
     ap.add_argument("--search-d", type=int, default=200)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run a small case of one workload for an ncu capture instead of the bench")
+    ap.add_argument("--profile-launches", type=int, default=3)
+    ap.add_argument("--profile-t", type=int, default=None)
+    ap.add_argument("--profile-n", type=int, default=None)
+    ap.add_argument("--profile-nq", type=int, default=None)
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.cpu_sample is None:
