@@ -133,8 +133,12 @@ __global__ void __launch_bounds__(128) quant_simple_kernel(QuantArgs a) {
     }
     const float n = sqrtf(block_sum(ss, red));  // block_sum syncs: xs visible
     if (threadIdx.x < K - 1) thr[threadIdx.x] = n * a.thresholds[threadIdx.x];
+    // the loads of Pi^T are independent of the FMA chain: a deep unroll keeps
+    // many of them in flight (a small batch, e.g. one appended token per head,
+    // is bound by their latency)
     for (int j = threadIdx.x; j < d; j += blockDim.x) {
       float acc = 0.f;
+#pragma unroll 16
       for (int i = 0; i < d; ++i) acc = fmaf(a.PiT[(int64_t)i * d + j], xs[i], acc);
       ys[j] = acc;
     }
@@ -159,6 +163,7 @@ __global__ void __launch_bounds__(128) quant_simple_kernel(QuantArgs a) {
       __syncthreads();
       for (int j = threadIdx.x; j < d; j += blockDim.x) {
         float acc = 0.f;
+#pragma unroll 16
         for (int i = 0; i < d; ++i) acc = fmaf(a.TT[(int64_t)i * d + j], us[i], acc);
         sidx[j] = (acc >= 0.f) ? 1 : 0;
       }
