@@ -217,6 +217,17 @@ class Sweep:
         return self.N * len(SWEEP_BITS)
 
     # ---- end to end through host buffers
+    def distortion(self):
+        """Per b: the measured mean ||x - x_hat||^2 / ||x||^2 of the batch (an untimed
+        round trip) beside 4^-b, the lower bound the pages compare it with."""
+        out = {}
+        for b in SWEEP_BITS:
+            self.tq.tq_quant_mse(self.h[b], self.x, self.codes[b], self.norms[b])
+            self.tq.tq_dequant_mse(self.h[b], self.codes[b], self.norms[b], self.xh)
+            D = mean_relative_sq_error(self.torch, self.x, self.xh)
+            out[f"b{b}"] = {"D": D, "4^-b": 4.0 ** -b, "D_times_4^b": D * 4.0 ** b}
+        return out
+
     def e2e(self, steps, warmup):
         tq, torch = self.tq, self.torch
         xh_host = self.x.cpu().pin_memory()
@@ -422,6 +433,14 @@ class Search:
             self.quant.append((e0, e1))
             self.score.append((e1, e2))
 
+    def recall(self, nsample=100):
+        """recall@topk of the last fused top-k against exact fp32 inner products
+        <q, x> (a library GEMM, outside the timed region) for the first queries."""
+        ns = min(nsample, self.nq)
+        exact = self.torch.matmul(self.q[:ns], self.x.t())
+        return {"recall_at_k": recall_at_k(self.torch, exact, self.ti[:ns], self.topk), "k": self.topk,
+                "queries": ns, "against": "exact fp32 <q, x> of the unquantized vectors"}
+
     def summary(self, hbm, tc_peak):
         qms = sum(a.elapsed_time(b) for a, b in self.quant) / len(self.quant)
         sms = sum(a.elapsed_time(b) for a, b in self.score) / len(self.score)
@@ -473,6 +492,28 @@ class Ranks:
     def close(self):
         if self.world > 1 and self.dist.is_initialized():
             self.dist.destroy_process_group()
+
+
+def mean_relative_sq_error(torch, x, xh, chunk=1 << 16) -> float:
+    """Mean over rows of ||x - xh||^2 / ||x||^2 (rows with x = 0 left out): the
+    distortion of a quantize + dequantize round trip, per vector."""
+    tot, cnt = 0.0, 0
+    for i in range(0, x.shape[0], chunk):
+        a = x[i:i + chunk].float()
+        e = (a - xh[i:i + chunk].float()).pow(2).sum(1)
+        n = a.pow(2).sum(1)
+        m = n > 0
+        tot += (e[m] / n[m]).double().sum().item()
+        cnt += int(m.sum().item())
+    return tot / max(cnt, 1)
+
+
+def recall_at_k(torch, exact_scores, got_idx, k) -> float:
+    """Share of each row's exact top-k (by score) found among the k returned
+    indices, averaged over rows."""
+    ex = torch.topk(exact_scores, k, dim=1).indices
+    hit = (ex.unsqueeze(2) == got_idx[:, :k].long().unsqueeze(1)).any(dim=2)
+    return hit.float().mean().item()
 
 
 def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
@@ -552,6 +593,12 @@ def run_ours(args):
               "config": config, "roofline": roofline, "kernels": kernels, "e2e": e2e,
               "gpu_launches": launches, "clocks": clk.summary()}
 
+    if args.workload == "sweep":
+        try:
+            result["distortion"] = wl.distortion()
+        except Exception as exc:  # a quality figure must not cost the bench line
+            result["distortion"] = {"error": repr(exc)}
+
     if args.workload == "sweep" and not args.no_decode:
         del wl
         torch.cuda.empty_cache()
@@ -602,6 +649,10 @@ def run_ours(args):
             sr.step(record=True)
         torch.cuda.synchronize()
         result["search"] = sr.summary(hbm, bf16)
+        try:
+            result["search"]["recall"] = sr.recall()
+        except Exception as exc:
+            result["search"]["recall"] = {"error": repr(exc)}
         del sr
 
     if rank == 0 and world == 1 and not args.no_cpu:

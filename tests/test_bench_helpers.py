@@ -1,0 +1,38 @@
+"""Host-side helpers of bench.py that turn GPU outputs into quality figures
+(sweep distortion, search recall@k), checked on small CPU tensors."""
+import os
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_mean_relative_sq_error_by_hand():
+    x = torch.tensor([[3.0, 4.0], [1.0, 0.0], [0.0, 0.0]])
+    xh = torch.tensor([[3.0, 3.0], [0.0, 0.0], [5.0, 5.0]])
+    # rows: 1/25, 1/1; the zero row is left out
+    got = bench.mean_relative_sq_error(torch, x, xh, chunk=2)
+    assert got == pytest.approx((1 / 25 + 1.0) / 2)
+
+
+def test_mean_relative_sq_error_bf16_input():
+    x = torch.randn(1000, 16).to(torch.bfloat16)
+    assert bench.mean_relative_sq_error(torch, x, x.float()) == 0.0
+
+
+def test_recall_at_k():
+    s = torch.tensor([[5.0, 4.0, 3.0, 2.0, 1.0],
+                      [1.0, 2.0, 3.0, 4.0, 5.0]])
+    got = torch.tensor([[0, 1, 4], [4, 3, 2]], dtype=torch.int32)
+    # row 0: exact top-3 {0, 1, 2}, found {0, 1} -> 2/3; row 1: all found
+    assert bench.recall_at_k(torch, s, got, 3) == pytest.approx((2 / 3 + 1) / 2)
+
+
+def test_recall_order_does_not_matter():
+    s = torch.randn(4, 50)
+    ex = torch.topk(s, 10, dim=1).indices
+    assert bench.recall_at_k(torch, s, ex.flip(1).to(torch.int32), 10) == 1.0
