@@ -186,7 +186,7 @@ __device__ __noinline__ float topk_insert(float* bv, int32_t* bi, int K, float s
 template <bool PROD, int BM>
 __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ CUtensorMap qmap, ScArgs a) {
   using T = Tile<PROD>;
-  constexpr int TN = T::TN, KPT = T::KPT, kBStages = T::BStages, kBBytes = T::BBytes;
+  constexpr int TN = T::TN, kBStages = T::BStages, kBBytes = T::BBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_s = smem;                                  // [kAStages][kABytes]

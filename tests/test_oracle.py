@@ -233,6 +233,29 @@ def test_one_bit_mse_inner_product_bias_is_two_over_pi():
     assert abs(slope - 2 / math.pi) < 0.02
 
 
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_mse_inner_product_shrinks_by_one_minus_distortion(b):
+    # The Lloyd centroid condition and the sphere's symmetry give
+    # E<q, x_hat> = (1 - D(b, d)) <q, x> at every b (the b = 1 case is the 2/pi
+    # above): a wrong centroid, threshold or rotation orientation moves the slope.
+    d, n = 128, 40000
+    Pi = tq.haar_rotation(synth.gaussian_matrix(d, d, 4, synth.ROT_K))
+    c, t = cb.lloyd_max(b, d)
+    x = synth.unit_rows(n, d, 21 + b)
+    q = synth.unit_rows(n, d, 31 + b)
+    idx, norms, _ = tq.quant_mse(x, Pi, t)
+    xh = tq.dequant_mse(idx, norms, Pi, c)
+    a = np.sum(q * x, axis=1)
+    e = np.sum(q * xh, axis=1)
+    slope = np.sum(a * e) / np.sum(a * a)
+    expect = 1 - cb.distortion(c, d)
+    resid = e - expect * a
+    se = math.sqrt(np.sum((a * resid) ** 2)) / np.sum(a * a)
+    assert abs(slope - expect) < 5 * se
+    # and the slope is not 1: the shrinkage is resolved at this sample size
+    assert (1 - slope) > 5 * se
+
+
 # --------------------------------------------------------------------- prod / QJL
 
 @pytest.mark.parametrize("d,b", [(64, 3), (128, 3), (256, 2), (512, 4)])
