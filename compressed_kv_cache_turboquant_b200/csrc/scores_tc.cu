@@ -63,7 +63,6 @@ constexpr int kMkBufs = 8;
 template <bool PROD>
 struct Tile {
   static constexpr int TN = PROD ? 128 : 256;       // keys per tile
-  static constexpr int KPT = TN / 128;              // keys per decoder thread
   static constexpr int BStages = PROD ? 3 : 2;
   static constexpr int BBytes = TN * 128;           // one 64-wide fp16 chunk of the key tile
   static constexpr int Tabs = PROD ? 2 : 1;         // codebook table (+ sign table)
