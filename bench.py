@@ -141,6 +141,13 @@ def oracle_sweep_rate(n_sample: int, bits=SWEEP_BITS, seed: int = 0):
     return n_sample * len(bits) / dt, dt
 
 
+def single_thread(fn, *args):
+    """fn(*args) with the BLAS thread pools held to one thread."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        return fn(*args)
+
+
 def oracle_decode_rate(T_sample: int, seed: int = 0):
     """Oracle decode for one (batch, kv-head) slice of T_sample tokens and its
     4 q-heads (logits, softmax, value sum).  Returns keys/s."""
@@ -710,6 +717,13 @@ def run_ours(args):
             sample = f"one (batch, kv-head) slice of {args.cpu_sample} tokens, 4 q-heads ({dt:.1f} s)"
         result["cpu_baseline"] = {"value": rate, "unit": unit_name, "cores": cpu_threads(), "kind": "oracle",
                                   "sample": sample}
+        try:  # the same oracle on one core, on an eighth of the sample
+            fn = oracle_sweep_rate if args.workload == "sweep" else oracle_decode_rate
+            rate1, dt1 = single_thread(fn, max(1, args.cpu_sample // 8))
+            result["cpu_baseline"]["single_thread"] = {"value": rate1, "unit": unit_name, "cores": 1,
+                                                       "sample": f"{args.cpu_sample // 8} units ({dt1:.1f} s)"}
+        except Exception as exc:
+            result["cpu_baseline"]["single_thread"] = {"error": repr(exc)}
     if rank == 0:
         print(json.dumps(result), flush=True)
     ranks.close()

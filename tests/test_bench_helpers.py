@@ -36,3 +36,10 @@ def test_recall_order_does_not_matter():
     s = torch.randn(4, 50)
     ex = torch.topk(s, 10, dim=1).indices
     assert bench.recall_at_k(torch, s, ex.flip(1).to(torch.int32), 10) == 1.0
+
+
+def test_single_thread_holds_blas_to_one_thread():
+    got = bench.single_thread(bench.cpu_threads)
+    assert got == 1
+    rate, dt = bench.single_thread(bench.oracle_sweep_rate, 256)
+    assert rate > 0 and dt > 0
