@@ -1,5 +1,5 @@
 // Thin wrappers over the sm_100a instructions the tensor-core kernels use:
-// mbarriers, TMA (no multicast), bulk copies, tcgen05 MMA / TMEM.  Every
+// mbarriers, TMA (single-CTA loads and stores), bulk copies, tcgen05 MMA / TMEM.  Every
 // wait is bounded in time; on expiry it reports failure so the caller can set
 // the device status word and leave without hanging the GPU.
 #pragma once
