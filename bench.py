@@ -606,21 +606,14 @@ def run_ours(args):
         ks = wl.kernel_stats()
         dom = max(ks, key=lambda k: ks[k]["ms_total"])
         unit_name = "vectors/s"
-        config = {"workload": "TurboQuant_mse quant+dequant sweep b=1..4, N=2^20 bf16, d=128, lognormal(0,1) "
-                              "channel scales, 4 channels x20 outliers",
-                  "N": SWEEP_N, "d": D, "bits": list(SWEEP_BITS), "input_dtype": "bf16",
-                  "dequant_dtype": "f32", "l2": "inputs larger than L2 (256 MiB bf16 per step per b)",
-                  "parallelism": f"dp{world} (independent batches, no collective)"}
+        config = workload_config("sweep", world)
         launches = wl.launches_per_step * args.steps
     else:
         k_ms = sum(a.elapsed_time(b) for a, b in wl.kern)
         ks = {"attn_decode": dict(ms_total=k_ms, launches=len(wl.kern), bytes_total=wl.bytes_per_step() * len(wl.kern))}
         dom = "attn_decode"
         unit_name = "keys/s"
-        config = {"workload": "decode attention over TurboQuant K/V: B=8, Hq=32, Hkv=8, d=128, T=131072, "
-                              "K prod 4b (3+1 QJL), V mse 4b, bf16 queries",
-                  "B": DEC["B"], "Hq": DEC["Hq"], "Hkv": DEC["Hkv"], "T": DEC["T"], "d": D,
-                  "l2": "packed cache 1.17 GB > L2", "parallelism": f"dp{world} (independent caches)"}
+        config = workload_config("decode", world)
         launches = 3 * args.steps
     dk = ks[dom]
     achieved = dk["bytes_total"] / (dk["ms_total"] / 1e3) / 1e9
@@ -772,6 +765,20 @@ def run_profile_case(args):
     print(json.dumps({"profile_case": case, "what": PROFILE_CASES[case], "size": size, "ms": ms}), flush=True)
 
 
+def workload_config(workload: str, world: int) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    if workload == "sweep":
+        return {"workload": "TurboQuant_mse quant+dequant sweep b=1..4, N=2^20 bf16, d=128, lognormal(0,1) "
+                            "channel scales, 4 channels x20 outliers",
+                "N": SWEEP_N, "d": D, "bits": list(SWEEP_BITS), "input_dtype": "bf16",
+                "dequant_dtype": "f32", "l2": "inputs larger than L2 (256 MiB bf16 per step per b)",
+                "parallelism": f"dp{world} (independent batches, no collective)"}
+    return {"workload": "decode attention over TurboQuant K/V: B=8, Hq=32, Hkv=8, d=128, T=131072, "
+                        "K prod 4b (3+1 QJL), V mse 4b, bf16 queries",
+            "B": DEC["B"], "Hq": DEC["Hq"], "Hkv": DEC["Hkv"], "T": DEC["T"], "d": D,
+            "l2": "packed cache 1.17 GB > L2", "parallelism": f"dp{world} (independent caches)"}
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -791,9 +798,12 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "sample_per_step": args.ref_sample},
+        "config": workload_config(args.workload, world),
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": f"{args.ref_sample} units per step of the {args.workload} workload"},
+                         "sample": (f"{args.ref_sample} vectors at each b = 1..4 per step (a bounded sample of the "
+                                    f"sweep)" if args.workload == "sweep" else
+                                    f"{args.ref_sample} tokens of one (batch, kv-head) slice, 4 q-heads, per step "
+                                    f"(a bounded sample of the decode workload)")},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
 
 

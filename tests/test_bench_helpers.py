@@ -43,3 +43,10 @@ def test_single_thread_holds_blas_to_one_thread():
     assert got == 1
     rate, dt = bench.single_thread(bench.oracle_sweep_rate, 256)
     assert rate > 0 and dt > 0
+
+
+def test_both_arms_share_the_workload_config():
+    c = bench.workload_config("sweep", 2)
+    assert c["N"] == 1 << 20 and c["bits"] == [1, 2, 3, 4] and c["parallelism"].startswith("dp2")
+    d = bench.workload_config("decode", 1)
+    assert (d["B"], d["Hq"], d["Hkv"], d["T"], d["d"]) == (8, 32, 8, 131072, 128)
