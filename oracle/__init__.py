@@ -1,7 +1,8 @@
 """Float64 CPU oracle for the TurboQuant hot path -- TEST INFRASTRUCTURE ONLY.
 
-Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  The product (the CUDA library and its
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU legs of ``bench.py``
+(its ``cpu_baseline`` and its reference arm, ``--impl reference``) may import
+this package.  The product (the CUDA library and its
 Python binding) never imports, links or calls anything here, and this package
 imports nothing from the product.  The only code the two sides share is the
 seeded input generator module ``synth``, which holds no quantizer arithmetic.
