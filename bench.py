@@ -44,9 +44,38 @@ METRIC = "vectors quantized/s; packed-KV logits keys/s and % of HBM-bandwidth ro
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# sweep kernels, averaged over b = 1..4, from one ncu capture of these kernels;
-# to be re-taken (or set to None) whenever either kernel changes
-MEASURED_TRAFFIC = {"quant_mse": 299.7e6, "dequant_mse": 521.1e6}
+# sweep kernels, averaged over b = 1..4, from one ncu capture (the summary file
+# named in "capture").  "sources" fingerprints the kernel sources the capture
+# ran: when they differ from the files in this tree the figure is stale and
+# roofline.traffic is reported as null.
+MEASURED_TRAFFIC = {
+    "quant_mse": {"bytes": None, "sources": None, "capture": None},
+    "dequant_mse": {"bytes": None, "sources": None, "capture": None},
+}
+TRAFFIC_SOURCES = {
+    "quant_mse": ["quant_tc.cu", "sm100_common.cuh"],
+    "dequant_mse": ["dequant_tc.cu", "sm100_common.cuh"],
+}
+
+
+def source_fingerprint(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "compressed_kv_cache_turboquant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str):
+    """(bytes per launch, note): the ncu figure if the kernel is unchanged since
+    it was captured, else (None, why)."""
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if not rec or rec["bytes"] is None:
+        return None, "no ncu capture of the current kernel"
+    if rec["sources"] != source_fingerprint(kernel):
+        return None, "stale: the kernel changed since the capture"
+    return rec["bytes"], rec["capture"]
 
 
 def peaks():
@@ -169,6 +198,67 @@ def oracle_decode_rate(T_sample: int, seed: int = 0):
                                                              Pk, Sk, c3, 4), lambda b, h: vhat, 1)
     dt = time.perf_counter() - t0
     return T_sample / dt, dt
+
+
+def oracle_search_rate(N: int, nq: int, d: int, b: int = 4, seed: int = 0):
+    """The oracle on a bounded sample of the search workload: quantize N unit
+    database vectors (prod, b bits), then score nq queries against all of them
+    with the estimator.  Returns (vectors/s, pairs/s, seconds)."""
+    from oracle import codebook as ocb
+    from oracle import turboquant as oq
+    P = oq.haar_rotation(synth.gaussian_matrix(d, d, seed, synth.ROT_K))
+    S = synth.gaussian_matrix(d, d, seed, synth.QJL_K)
+    c, t = ocb.lloyd_max(b - 1, d)
+    x = synth.unit_rows(N, d, seed)
+    q = synth.unit_rows(nq, d, seed, stream=synth.QUERY)
+    t0 = time.perf_counter()
+    st = oq.quant_prod(x, b, P, S, t, c)
+    t1 = time.perf_counter()
+    oq.prod_estimate(q, st["idx"], st["norms"], st["signs"], st["rnorms"], P, S, c, b)
+    t2 = time.perf_counter()
+    return N / (t1 - t0), N * nq / (t2 - t1), t2 - t0
+
+
+def oracle_stream_rate(T_sample: int, seed: int = 0):
+    """The oracle's full-context logits for one kv-head of the split cache (64
+    channels at prod 4 bits + 64 at prod 3 bits, 4 q-heads) over T_sample
+    tokens.  Returns (keys/s, seconds)."""
+    from oracle import codebook as ocb
+    from oracle import turboquant as oq
+    scales = synth.lognormal_channel_scales(D, 1.0, seed, 30)
+    hi, lo = oq.channel_split(scales, 64)
+    k = synth.rng(seed, synth.DATA, 40, 0).standard_normal((T_sample, D)) * scales[None, :]
+    q = synth.decode_queries(1, 4, D, seed=seed)[0]
+    groups = []
+    for grp, (b, ch) in enumerate(((4, hi), (3, lo))):
+        P = oq.haar_rotation(synth.gaussian_matrix(64, 64, seed, synth.ROT_K, grp))
+        S = synth.gaussian_matrix(64, 64, seed, synth.QJL_K, grp)
+        c, t = ocb.lloyd_max(b - 1, 64)
+        groups.append((b, ch, P, S, c, oq.quant_prod(k[:, ch], b, P, S, t, c)))
+    t0 = time.perf_counter()
+    logits = np.zeros((4, T_sample))
+    for b, ch, P, S, c, st in groups:
+        logits += oq.prod_estimate(q[:, ch], st["idx"], st["norms"], st["signs"], st["rnorms"], P, S, c, b)
+    dt = time.perf_counter() - t0
+    return T_sample / dt, dt
+
+
+def oracle_sub_baselines(search_d: int):
+    """Oracle rates beside the decode, stream and search sub-results (bounded
+    samples, all host threads); each entry says what its sample was."""
+    cores = cpu_threads()
+    out = {}
+    r, dt = oracle_decode_rate(1 << 16)
+    out["decode"] = {"value": r, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                     "sample": f"one (batch, kv-head) slice of 65536 tokens, 4 q-heads ({dt:.1f} s)"}
+    r, dt = oracle_stream_rate(1 << 16)
+    out["stream"] = {"value": r, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                     "sample": f"logits of one kv-head over 65536 tokens of the split cache, 4 q-heads ({dt:.1f} s)"}
+    qv, pr, dt = oracle_search_rate(10 ** 5, 64, search_d)
+    out["search"] = {"quantize_vectors_per_s": qv, "score_pairs_per_s": pr, "cores": cores, "kind": "oracle",
+                     "sample": f"quantize 10^5 vectors, then 64 queries x 10^5 keys, d={search_d}, prod b=4 "
+                               f"({dt:.1f} s)"}
+    return out
 
 
 # ----------------------------------------------------------------- GPU workloads
@@ -619,8 +709,9 @@ def run_ours(args):
     achieved = dk["bytes_total"] / (dk["ms_total"] / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
-                "traffic": MEASURED_TRAFFIC.get(dom) if args.workload == "sweep" else None,
-                "bytes_per_launch": dk["bytes_total"] / dk["launches"]}
+                "traffic": None, "bytes_per_launch": dk["bytes_total"] / dk["launches"]}
+    if args.workload == "sweep":
+        roofline["traffic"], roofline["traffic_source"] = measured_traffic(dom)
     kernels = {k: {"avg_ms": v["ms_total"] / v["launches"],
                    "GBps": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9,
                    "frac_hbm": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9 / hbm} for k, v in ks.items()}
@@ -717,6 +808,14 @@ def run_ours(args):
                                                        "sample": f"{args.cpu_sample // 8} units ({dt1:.1f} s)"}
         except Exception as exc:
             result["cpu_baseline"]["single_thread"] = {"error": repr(exc)}
+        if args.workload == "sweep":
+            try:
+                subs = oracle_sub_baselines(args.search_d)
+                for k, v in subs.items():
+                    if k in result:
+                        result[k]["cpu_baseline"] = v
+            except Exception as exc:
+                result["cpu_baseline"]["sub_results"] = {"error": repr(exc)}
     if rank == 0:
         print(json.dumps(result), flush=True)
     ranks.close()

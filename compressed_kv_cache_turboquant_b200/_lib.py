@@ -16,6 +16,7 @@ TQ_F32, TQ_BF16 = 0, 1
 TQ_MSE, TQ_PROD = 0, 1
 TQ_MAX_DIM = 4096
 TQ_MAX_TOPK = 64
+TQ_STATUS_TIMEOUT, TQ_STATUS_LAYOUT = 1, 2
 TQ_DECODE_STATIC_SCRATCH = 4 * 1024 * 1024
 
 if not os.path.exists(LIB_PATH):

@@ -12,10 +12,11 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (TQ_BF16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQError, check, lib)
+from ._lib import (TQ_BF16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQ_STATUS_LAYOUT, TQ_STATUS_TIMEOUT, TQError,
+                   check, lib)
 
 __all__ = [
-    "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQError", "Handle", "code_words", "sign_words",
+    "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQ_STATUS_TIMEOUT", "TQ_STATUS_LAYOUT", "TQError", "Handle", "code_words", "sign_words",
     "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
     "tq_quant_prod_workspace",
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",

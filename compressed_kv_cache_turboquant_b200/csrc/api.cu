@@ -9,7 +9,10 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <set>
+#include <tuple>
 #include <vector>
 
 #include "tq_internal.h"
@@ -29,6 +32,20 @@ int set_error(int code, const char* fmt, ...) {
 int clear_error() {
   g_err[0] = '\0';
   return TQ_OK;
+}
+
+int ensure_dyn_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, int, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(kernel, dev, bytes);
+  if (done.count(key)) return (int)cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return (int)e;
 }
 
 static int cuda_error(const char* where, int e) {
@@ -327,6 +344,13 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
     const char* ev = getenv("TQ_RUNTIME_TABLE_ADDRESSES");
     if (e == cudaSuccess && !(ev && ev[0] == '1'))
       e = (cudaError_t)probe_dyn_smem_base((uint32_t*)(h->dev.status + 16), &h->dyn_base);
+    const char* st = getenv("TQ_DEBUG_STALL_MS");
+    if (st && atof(st) > 0) h->debug_stall_ns = (uint64_t)(atof(st) * 1e6);
+    const char* db = getenv("TQ_DEBUG_DYN_BASE");
+    if (db && db[0]) {
+      h->dyn_base = (uint32_t)strtoul(db, nullptr, 0);
+      h->debug_fixed_tables = true;
+    }
   }
   if (e == cudaSuccess && tc)
     e = cudaMemcpy(h->dev.pi_tc, pieces.data(), pieces.size() * 2, cudaMemcpyHostToDevice);

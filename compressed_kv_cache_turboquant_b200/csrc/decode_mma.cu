@@ -98,6 +98,9 @@ struct DecArgs {
   float qjl_coef;          // sqrt(pi/2) / d
   float* partials;         // [CTA][max_seg][4 heads][d + 2]: acc[d], m (natural log), l
   int* status;
+  uint32_t dyn_base;       // where the host measured the dynamic window to start
+  uint64_t wait_ns;        // limit of every pipeline wait
+  int stall;               // diagnostic: consumers first wait on a barrier nothing completes
 };
 
 // CTA i of G owns the global blocks [i*total/G, (i+1)*total/G); a global block
@@ -137,7 +140,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
   constexpr uint32_t KV = tab_addr(DB, kStages * kStageBytes);
   constexpr uint32_t SG = tab_addr(DB, kStages * kStageBytes + kTabBytes);
   extern __shared__ __align__(1024) uint8_t smem[];
-  if (DB != kDynRuntime && smem_u32(smem) != DB) {  // not the window this instance was built for
+  // the instance built for the host's measurement of the window start (DB ==
+  // a.dyn_base) finds the window elsewhere: report, write nothing
+  if (DB != kDynRuntime && (smem_u32(smem) != DB || a.dyn_base != DB)) {
     if (threadIdx.x == 0) atomicOr(a.status, kStatusLayout);
     return;
   }
@@ -147,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
   uint64_t* full = reinterpret_cast<uint64_t*>(sgtab + kSgTabBytes);
   uint64_t* empty = full + kStages;
   uint64_t* pub = empty + kStages;                                        // consumer sync at segment ends
+  uint64_t* never = pub + 1;                                              // diagnostic: nothing arrives
   __half* pbuf = reinterpret_cast<__half*>(pub + 2);                     // [kCons][4 heads][16 tokens]
   float* mrg = reinterpret_cast<float*>(pbuf + kCons * 64);               // [kCons][4][2 + D]
 
@@ -161,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
       mbar_init(&empty[s], kCons);
     }
     mbar_init(pub, 32 * kCons);
+    mbar_init(never, 1);
     fence_mbar_init();
   }
   // tables
@@ -185,13 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
     if (lane == 0) {
       BlockCursor cur;
       cur.init(gb_lo, a.nblk);
+      int64_t issued = 0;
       for (int64_t gb = gb_lo, i = 0; gb < gb_hi; ++gb, ++i, cur.next(a.nblk)) {
         const int s = (int)(i % kStages);
         const uint32_t u = (uint32_t)(i / kStages);
-        if (!mbar_wait(&empty[s], (u & 1u) ^ 1u)) {
+        if (!mbar_wait_ns(&empty[s], (u & 1u) ^ 1u, a.wait_ns)) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }
+        issued = i + 1;
         const int64_t bh = cur.bh;
         const int64_t t0 = cur.blk * kBlk;
         const int n = (int)min((int64_t)kBlk, a.T - t0);
@@ -206,6 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
           bulk_load(st + kOffN, a.knorms + r, n4 * 4, &full[s]);
           bulk_load(st + kOffR, a.krnorms + r, n4 * 4, &full[s]);
           bulk_load(st + kOffVN, a.vnorms + r, n4 * 4, &full[s]);
+        }
+      }
+      // Before the CTA may exit, every copy issued into its shared memory must
+      // have landed, also when the consumers gave up early: wait (bounded) for
+      // the last phase of each stage that received a block.
+      for (int64_t i = issued - kStages > 0 ? issued - kStages : 0; i < issued; ++i) {
+        if (!mbar_wait(&full[i % kStages], (uint32_t)((i / kStages) & 1))) {
+          atomicOr(a.status, kStatusTimeout);
+          break;
         }
       }
     }
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         }
       }
       mbar_arrive(pub);
-      if (!mbar_wait(pub, 0u)) {
+      if (!mbar_wait_ns(pub, 0u, a.wait_ns)) {
         ok = false;
         return;
       }
@@ -289,9 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
       }
       // second phase: everyone has read the merge buffer before it is written again
       mbar_arrive(pub);
-      if (!mbar_wait(pub, 1u)) ok = false;
+      if (!mbar_wait_ns(pub, 1u, a.wait_ns)) ok = false;
     };
 
+    if (a.stall && !mbar_wait_ns(never, 0u, a.wait_ns)) ok = false;
     BlockCursor cur;
     cur.init(gb_lo, a.nblk);
     const int nblocks = (int)(gb_hi - gb_lo);
@@ -325,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
           for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
       }
       const int s = stg;
-      if (!mbar_wait(&full[s], phase)) {
+      if (!mbar_wait_ns(&full[s], phase, a.wait_ns)) {
         ok = false;
         break;
       }
@@ -572,16 +591,14 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.qjl_coef = 1.2533141373155003f / 128.0f;
   a.partials = partials;
   a.status = hk->dev.status;
+  a.dyn_base = hk->dyn_base;
+  a.wait_ns = hk->debug_stall_ns ? hk->debug_stall_ns : kWaitLimitNs;
+  a.stall = hk->debug_stall_ns ? 1 : 0;
   const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
   const int smem = kSmemBytes;
-  const bool fixed = hk->dyn_base == kDynBaseSm100;
+  const bool fixed = hk->dyn_base == kDynBaseSm100 || hk->debug_fixed_tables;
   auto kern = fixed ? decode_mma_kernel<kDynBaseSm100> : decode_mma_kernel<kDynRuntime>;
-  static bool attr[2] = {false, false};
-  if (!attr[fixed]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    attr[fixed] = true;
-  }
+  if (int e = ensure_dyn_smem((const void*)kern, smem)) return e;
   cudaStream_t s = (cudaStream_t)stream;
   kern<<<G, kThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();

@@ -309,12 +309,7 @@ int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return (int)cudaErrorInvalidValue;
   auto kern = dequant_tc_kernel<D, BM>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
+  if (int e = ensure_dyn_smem((const void*)kern, S::kSmemBytes)) return e;
   DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, h->dev.status};
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);

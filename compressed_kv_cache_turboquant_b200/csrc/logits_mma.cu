@@ -76,6 +76,7 @@ struct LgArgs {
   float scale;
   float* logits;          // [B][Hq][T]
   int* status;
+  uint32_t dyn_base;      // where the host measured the dynamic window to start
 };
 
 __host__ __device__ __forceinline__ int64_t lg_first_block(int64_t i, int64_t total, int64_t G) {
@@ -127,7 +128,9 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
   constexpr uint32_t KT = tab_addr(DB, kStages * L::Stage);
   constexpr uint32_t SG = tab_addr(DB, kStages * L::Stage + kTabBytes);
   extern __shared__ __align__(1024) uint8_t smem[];
-  if (DB != kDynRuntime && smem_u32(smem) != DB) {  // not the window this instance was built for
+  // the instance built for the host's measurement of the window start (DB ==
+  // a.dyn_base) finds the window elsewhere: report, write nothing
+  if (DB != kDynRuntime && (smem_u32(smem) != DB || a.dyn_base != DB)) {
     if (threadIdx.x == 0) atomicOr(a.status, kStatusLayout);
     return;
   }
@@ -502,16 +505,11 @@ int launch_logits_mma(const tq_ctx* const* hk, const float* const* qrot, const f
   a.scale = scale;
   a.logits = logits;
   a.status = hk[0]->dev.status;
+  a.dyn_base = hk[0]->dyn_base;
   const int grid = (int)(a.total < hk[0]->sm_count ? a.total : hk[0]->sm_count);
-  const bool fixed = hk[0]->dyn_base == kDynBaseSm100;
+  const bool fixed = hk[0]->dyn_base == kDynBaseSm100 || hk[0]->debug_fixed_tables;
   auto go = [&](auto kern, int smem) -> int {
-    static bool set[2][4][4] = {};
-    bool& done = set[fixed][hk[0]->bm][hk[1]->bm];
-    if (!done) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return (int)e;
-      done = true;
-    }
+    if (int e = ensure_dyn_smem((const void*)kern, smem)) return e;
     kern<<<grid, kThreads, smem, s>>>(a);
     return (int)cudaGetLastError();
   };

@@ -570,12 +570,7 @@ template <int STAGE>
 int launch_stage(const tq_ctx* h, const GenArgs& a, const CUtensorMap& map, const CUtensorMap& umap, int grid,
                  cudaStream_t s) {
   auto pick = [&](auto kern) -> int {
-    static bool set[3][5] = {};
-    if (!set[STAGE - 1][h->bm]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-      if (e != cudaSuccess) return (int)e;
-      set[STAGE - 1][h->bm] = true;
-    }
+    if (int e = ensure_dyn_smem((const void*)kern, kSmem)) return e;
     kern<<<grid, kThreads, kSmem, s>>>(map, umap, a);
     return (int)cudaGetLastError();
   };

@@ -118,9 +118,13 @@ __device__ __forceinline__ void pack_group(const float* v, const float (&P)[8], 
 
 // The same cells computed on the FMA pipe (the binary search above runs on
 // the ALU pipe, which the epilogue saturates at 3 and 4 bits; half of the
-// groups go each way).  With B = 2^32 / n and C_k = 1 - 2^32 t_k:
-//   sat(|y| B + C_k) = 1 when |y| >= n t_k and 0 when |y| < n t_k (up to a band
-//   of 2^-32 n around the threshold, far inside the parity band), so
+// groups go each way).  With B = 2^32 / n and C_k = 1 - 2^32 t_k, both rounded
+// to float32:
+//   sat(|y| B + C_k) = 1 when |y| >= n t_k and 0 when |y| < n t_k, up to a band
+//   around the threshold: B carries the 2^-24 relative rounding of 2^32 / n and
+//   C_k that of 2^32 t_k (its ulp is 32 to 256 for the thresholds here), so the
+//   decision can move by about 2^-23 |t_k| in the unit frame y / n -- under
+//   3e-8 at d = 128, some 30 times inside the parity band 1e-5 / sqrt(d) -- so
 //   m = sum_k sat(|y| B + C_k) counts the positive thresholds at or below |y|,
 //   s = sat(y B + 1) is 1 for y >= 0 (to the same band), and
 //   cell = (H - 1 - m) + s (2m + 1).
@@ -376,13 +380,8 @@ int launch_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_stride, uint3
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
-  static bool attr_set[5][2] = {};
   auto kern = quant_mse_tc_kernel<D, BM>;
-  if (!attr_set[BM][D == 128]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-    if (e != cudaSuccess) return (int)e;
-    attr_set[BM][D == 128] = true;
-  }
+  if (int e = ensure_dyn_smem((const void*)kern, S::kSmemBytes)) return e;
   TcArgs a{h->dev.pi_tc, h->dev.thresholds, N, out_stride, codes, norms, h->dev.status};
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);

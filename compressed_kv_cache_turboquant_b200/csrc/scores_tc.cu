@@ -688,14 +688,7 @@ int launch_scores_tc(const tq_ctx* h, const float* q, int64_t nq, const uint32_t
   for (int k = 0; k < 8; ++k) a.ctab[k] = (uint32_t)h->sc_tab[2 * k] | ((uint32_t)h->sc_tab[2 * k + 1] << 16);
   a.status = h->dev.status;
   auto launch = [&](auto kern, int smem) -> int {
-    // one attribute call per instantiation
-    static bool attr[2][4] = {};
-    bool& set = attr[prod ? 1 : 0][h->bm];
-    if (!set) {
-      cudaError_t ee = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (ee != cudaSuccess) return (int)ee;
-      set = true;
-    }
+    if (int ee = ensure_dyn_smem((const void*)kern, smem)) return ee;
     kern<<<(unsigned)p.G, kThreads, smem, s>>>(map, a);
     return 0;
   };

@@ -76,14 +76,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // a suspended wait re-checks the time limit at least this often
 constexpr uint32_t kWaitSleepNs = 200000u;
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete, giving up (false)
+// after limit_ns nanoseconds of device time.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint32_t hint = limit_ns < kWaitSleepNs ? (uint32_t)limit_ns : kWaitSleepNs;
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
+}
+
+// Bounded wait (kWaitLimitNs) for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_ns(bar, parity, kWaitLimitNs);
 }
 
 // 2D tiled TMA load into shared memory, completion counted on `bar`.

@@ -12,6 +12,12 @@ namespace tqi {
 int set_error(int code, const char* fmt, ...);
 int clear_error();
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The setting belongs to the device that is current when it is made,
+// so it is applied once per (kernel, device); safe to call from several host
+// threads.  Returns a cudaError_t.
+int ensure_dyn_smem(const void* kernel, int bytes);
+
 constexpr int kMaxMseBits = 4;
 
 // Device-resident constants of one quantizer instance (one cudaMalloc block).
@@ -69,6 +75,17 @@ struct tq_ctx {
   float sc_inv_alpha = 1.f;
   int gen_d_pad = 0;
   uint32_t dyn_base = 0xFFFFFFFFu;  // shared address of a kernel's dynamic window (probed at creation)
+  // Diagnostics read from the environment at creation (normally off):
+  //   TQ_DEBUG_STALL_MS=m   the decode kernel's consumer warps first wait, m ms
+  //                         at most, on a barrier that nothing completes, and
+  //                         every other wait of that kernel gives up after m ms:
+  //                         the timeout path runs and reports TQ_STATUS_TIMEOUT
+  //   TQ_DEBUG_DYN_BASE=a   record `a` as the measured shared-window address:
+  //                         the decode and logits kernels built for the usual
+  //                         address run and find the window elsewhere
+  //                         (TQ_STATUS_LAYOUT)
+  uint64_t debug_stall_ns = 0;
+  bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 

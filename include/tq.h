@@ -26,6 +26,12 @@
  *   by tq_create to the device that was current at that time.  Concurrent
  *   calls on one handle from several streams are safe; destroying a handle
  *   while work that uses it is in flight is not.
+ * - A kernel that meets a condition it cannot finish under (a pipeline wait
+ *   that runs past its time limit, a shared-memory window that is not where
+ *   tq_create measured it) leaves early and sets a bit in the handle's device
+ *   status word; the call has already returned TQ_OK by then, and that call's
+ *   outputs are incomplete.  Callers that must know poll tq_device_status
+ *   after their stream has reached the calls in question.
  *
  * Packed code layout (the pages say only that 32-bit coordinates become 2- or
  * 4-bit integers, [ttakun, "为什么随机旋转是整个算法的底层杠杆"]).  A vector's d rotated
@@ -129,6 +135,16 @@ TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
  * environment variable TQ_RUNTIME_TABLE_ADDRESSES=1 the probe is skipped and
  * those kernels add the table addresses at run time (a slower instance of the
  * same arithmetic).
+ * Two diagnostic settings, also read from the environment here, exist so that
+ * the status word's reports can be exercised without faulting a GPU (both are
+ * off unless set):
+ *   TQ_DEBUG_STALL_MS=m  tq_attn_decode's kernel first waits, m ms at most, on
+ *                        a barrier that nothing completes, and every other wait
+ *                        of that kernel gives up after m ms: the call reports
+ *                        TQ_STATUS_TIMEOUT and its output is undefined
+ *   TQ_DEBUG_DYN_BASE=a  record `a` as the measured shared-window address, so
+ *                        the decode and logits kernels built for the usual
+ *                        address report TQ_STATUS_LAYOUT and write nothing
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
  */
 TQ_API int tq_create(tq_handle* h, int d, int b, int variant, const double* Pi, const double* S,
@@ -286,7 +302,9 @@ TQ_API size_t tq_attn_decode_workspace(tq_handle hk, int B, int Hq, int Hkv, int
  *   The array (TQ_DECODE_STATIC_SCRATCH bytes) is held on every GPU that loads
  *   the library until the process exits.  The first call on a device looks up
  *   the array's device address (cudaGetSymbolAddress) with that device
- *   current; make that first call before any stream capture.
+ *   current; make that first call before any stream capture.  The address is
+ *   kept for the life of the process: after a cudaDeviceReset both it and
+ *   every handle of that device are stale and must not be used again.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents; nothing in it has to start at zero (every scratch value is
  *   written before it is read within a call).  Calls that overlap on the GPU
@@ -353,7 +371,9 @@ TQ_API size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, 
 
 /*
  * tq_device_status -- read and clear the handle's device status word
- * (synchronous).  0 = no event.  Bit 0 (TQ_STATUS_TIMEOUT): a tensor-core
+ * (synchronous: waits for the device).  0 = no event.  A kernel that sets a
+ * bit has left before writing all of its outputs, and the call that launched
+ * it has returned TQ_OK: callers that need to know poll this word.  Bit 0 (TQ_STATUS_TIMEOUT): a tensor-core
  * kernel gave up a wait on one of its own pipeline barriers after ~2 s and
  * returned early; its outputs for that call are incomplete.  Bit 1
  * (TQ_STATUS_LAYOUT): a decode or logits kernel built for the shared-memory

@@ -127,3 +127,13 @@ def upload_words(w: np.ndarray) -> torch.Tensor:
 
 def sqrt_half_pi_over(d: int) -> float:
     return math.sqrt(math.pi / 2) / d
+
+
+def assert_status_clean(*handles):
+    """Every bounded wait of the calls made so far completed and every kernel
+    found its shared-memory window where it was built to (reads and clears the
+    handles' device status words)."""
+    for h in handles:
+        h = h.h if isinstance(h, Instance) else h
+        st = tq.tq_device_status(h)
+        assert st == 0, f"device status {st:#x} (1 = a wait gave up, 2 = shared-memory layout mismatch)"

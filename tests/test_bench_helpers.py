@@ -50,3 +50,21 @@ def test_both_arms_share_the_workload_config():
     assert c["N"] == 1 << 20 and c["bits"] == [1, 2, 3, 4] and c["parallelism"].startswith("dp2")
     d = bench.workload_config("decode", 1)
     assert (d["B"], d["Hq"], d["Hkv"], d["T"], d["d"]) == (8, 32, 8, 131072, 128)
+
+
+def test_traffic_figure_is_dropped_when_the_kernel_changed(monkeypatch):
+    fp = bench.source_fingerprint("dequant_mse")
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "dequant_mse",
+                        {"bytes": 5.0e8, "sources": fp, "capture": "profiles/x.md"})
+    assert bench.measured_traffic("dequant_mse") == (5.0e8, "profiles/x.md")
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "dequant_mse",
+                        {"bytes": 5.0e8, "sources": "0" * 16, "capture": "profiles/x.md"})
+    got, why = bench.measured_traffic("dequant_mse")
+    assert got is None and "stale" in why
+
+
+def test_oracle_sub_baselines_small_samples():
+    r, dt = bench.oracle_stream_rate(512)
+    assert r > 0 and dt > 0
+    qv, pr, dt = bench.oracle_search_rate(300, 4, 64)
+    assert qv > 0 and pr > 0 and dt > 0

@@ -16,8 +16,8 @@ import torch
 import synth
 from oracle import turboquant as oq
 
-from cases import (DEV, Instance, bf16_exact, compare_codes, compare_signs, rel_err, rel_l2_rows,
-                   to_device, upload_words, words_u32)
+from cases import (DEV, Instance, assert_status_clean, bf16_exact, compare_codes, compare_signs, rel_err,
+                   rel_l2_rows, to_device, upload_words, words_u32)
 
 import compressed_kv_cache_turboquant_b200 as tq
 
@@ -38,6 +38,7 @@ def _check_quant(inst: Instance, x64: np.ndarray, out: dict, rows=None):
         compare_signs(words_u32(out["signs"])[rows], ref["signs"], ref["Sr"], ref["norms"], exact)
         rn = out["rnorms"].cpu().numpy()[rows]
         assert np.max(rel_err(rn[exact], ref["rnorms"][exact])) <= NORM_RTOL
+    assert_status_clean(inst)
     return ref, exact
 
 
@@ -200,6 +201,39 @@ def test_dequant_matches_oracle(b, d):
     torch.cuda.synchronize()
     assert np.max(rel_l2_rows(out.cpu().numpy(), ref)) <= 1e-5
     assert np.max(rel_l2_rows(outb.float().cpu().numpy(), ref)) <= 2 ** -8
+    assert_status_clean(inst)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_sweep_dequant_full_size_every_row(b):
+    """The sweep batch (N = 2^20 bf16 rows, d = 128, lognormal(0, 1) scales, 4
+    outlier channels x20) quantized by the oracle, dequantized on the GPU in the
+    launch the bench times, and every row compared with the oracle's
+    reconstruction (relative L2 <= 1e-5).  At this size each persistent CTA
+    walks dozens of 128-row tiles, so the code prefetch of the next tile and
+    the reuse of every output staging box are compared, not only the first
+    tile of each CTA."""
+    N, d, chunk = 1 << 20, 128, 1 << 16
+    inst = Instance(d, b, tq.TQ_MSE)
+    x64 = bf16_exact(synth.scaled_gaussian_rows(N, d, 1.0, seed=0, outliers=4))
+    codes = torch.empty((N, inst.h.words), dtype=torch.int32, device=DEV)
+    norms = torch.empty(N, dtype=torch.float32, device=DEV)
+    parts = []
+    for r0 in range(0, N, chunk):
+        idx, n, _ = oq.quant_mse(x64[r0:r0 + chunk], inst.Pi_o, inst.t_o)
+        codes[r0:r0 + chunk] = upload_words(oq.pack_codes_vec(idx, b))
+        norms[r0:r0 + chunk] = torch.tensor(n, device=DEV)
+        parts.append((idx, n))
+    out = torch.empty((N, d), dtype=torch.float32, device=DEV)
+    tq.tq_dequant_mse(inst.h, codes, norms, out)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for k, r0 in enumerate(range(0, N, chunk)):
+        idx, n = parts[k]
+        ref = oq.dequant_mse(idx, n, inst.Pi_o, inst.c_o)
+        worst = max(worst, float(np.max(rel_l2_rows(out[r0:r0 + chunk].cpu().numpy(), ref))))
+    assert worst <= 1e-5, worst
+    assert_status_clean(inst)
 
 
 # ------------------------------------------------------------------ scores
@@ -229,6 +263,7 @@ def _score_case(inst, N, nq, seed, topk=0):
     tol = 1e-4 * np.linalg.norm(q64, axis=1)[:, None] * np.linalg.norm(x64, axis=1)[None, :]
     err = np.abs(scores.cpu().numpy() - ref)
     assert np.all(err <= tol), float(np.max(err / tol))
+    assert_status_clean(inst)
     return ref, tol, kw
 
 
@@ -296,18 +331,21 @@ def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
     gsz = Hq // Hkv
     for (b, h), (kst, vhat) in refs.items():
         qs = q64[b, h * gsz:(h + 1) * gsz]
-        est = oq.prod_estimate(qs, kst["idx"], kst["norms"], kst["signs"], kst["rnorms"], hk.Pi_o, hk.S,
-                               hk.c_o, 4)
-        logits = est * scale
+        # the oracle's attention step on this (batch, kv-head) as a one-head problem
+        est = lambda _b, _h, rows: oq.prod_estimate(rows, kst["idx"], kst["norms"], kst["signs"], kst["rnorms"],
+                                                    hk.Pi_o, hk.S, hk.c_o, 4)
+        ref_out, ref_logits = oq.attention_decode(qs[None], est, lambda _b, _h: vhat, 1, scale=scale)
+        ref = ref_out[0]
+        logits = ref_logits[(0, 0)]
         p = np.exp(logits - logits.max(axis=1, keepdims=True))
         p /= p.sum(axis=1, keepdims=True)
-        ref = p @ vhat
         # logit tolerance of the score bound, propagated through the softmax
         eps = scale * 1e-4 * np.linalg.norm(qs, axis=1)[:, None] * (np.asarray(kst["norms"], dtype=np.float64)[None, :])
         spread = np.linalg.norm(vhat[None, :, :] - ref[:, None, :], axis=2)
         tol = 2 * np.sum(p * eps * spread, axis=1) + 1e-3 * np.linalg.norm(ref, axis=1)
         err = np.linalg.norm(got[b, h * gsz:(h + 1) * gsz] - ref, axis=1)
         assert np.all(err <= tol), (b, h, err, tol)
+    assert_status_clean(hk, hv)
 
 
 def test_decode_small_ragged():
@@ -427,6 +465,7 @@ def _logits_case(B, Hq, Hkv, T, sample, seed=0):
             tol = scale * 1e-4 * np.linalg.norm(qv) * np.linalg.norm(k64, axis=1)
             err = np.abs(got[b, 4 * h + j] - ref)
             assert np.all(err <= tol), (b, h, j, float(np.max(err / tol)))
+    assert_status_clean(ia, ib)
 
 
 def test_split_group_logits_small_ragged():
@@ -461,11 +500,9 @@ def _search_case(d, b, N, nq, sample, seed=0, with_scores=False, k=10):
     tq.tq_ip_scores(inst.h, q, codes, signs, norms, rnorms, scores=scores, topk=k, top_idx=ti, top_val=tv)
     torch.cuda.synchronize()
     ti, tv = ti.cpu().numpy(), tv.cpu().numpy()
-    xh = oq.dequant_mse(st["idx"], st["norms"], inst.Pi_o, inst.c_o)
-    Sx = np.where(st["signs"], 1.0, -1.0)
-    coef = st["rnorms"].astype(np.float64) * math.sqrt(math.pi / 2) / d
-    for r in sample:
-        ref = xh @ q64[r] + coef * (Sx @ (inst.S @ q64[r]))
+    refs = oq.prod_estimate(q64[sample], st["idx"], st["norms"], st["signs"], st["rnorms"], inst.Pi_o, inst.S,
+                            inst.c_o, b)
+    for ref, r in zip(refs, sample):
         tol = 1e-4 * np.linalg.norm(q64[r]) * np.linalg.norm(x64, axis=1)
         assert np.all(np.abs(tv[r] - ref[ti[r]]) <= tol[ti[r]]), r
         assert np.all(np.diff(tv[r]) <= 0) and len(set(ti[r].tolist())) == k
@@ -475,6 +512,7 @@ def _search_case(d, b, N, nq, sample, seed=0, with_scores=False, k=10):
         if with_scores:
             err = np.abs(scores[r].cpu().numpy() - ref)
             assert np.all(err <= tol), (r, float(np.max(err / tol)))
+    assert_status_clean(inst)
     return inst
 
 

@@ -161,6 +161,30 @@ def test_threshold_count_equals_bruteforce_nearest(d, b):
     assert np.array_equal(tq.quantize_indices(t, t), np.arange(1, 2 ** b))
 
 
+@pytest.mark.parametrize("d", [128, 1536])
+def test_near_threshold_band_is_one_e_minus_5_over_sqrt_d(d):
+    # The parity rule excuses a code only where the rotated unit-frame value lies
+    # within 1e-5/sqrt(d) of a decision threshold.  Hand-placed values just inside
+    # and just outside the band of every threshold of a real codebook, one exactly
+    # on the band edge (the rule is "<="), and values on the centroids (far from
+    # every threshold) pin the scale (tol/sqrt(d), not tol*sqrt(d) or tol), the
+    # comparison and the reference points (thresholds, not centroids).
+    c, t = cb.lloyd_max(3, d)
+    w = 1e-5 / math.sqrt(d)
+    inside = np.concatenate([t + 0.99 * w, t - 0.99 * w])
+    outside = np.concatenate([t + 1.01 * w, t - 1.01 * w])
+    assert np.all(tq.near_threshold_mask(inside, t, d))
+    assert not np.any(tq.near_threshold_mask(outside, t, d))
+    assert not np.any(tq.near_threshold_mask(c, t, d))
+    assert np.all(tq.near_threshold_mask(t, t, d))
+    # exact band edge: thresholds (0, 0.25) and y = w are represented exactly
+    edge = np.array([w, 0.25 + 2 * w, -w])
+    assert np.array_equal(tq.near_threshold_mask(edge, np.array([0.0, 0.25]), d), [True, False, True])
+    # the mask keeps the shape of its input and judges each coordinate on its own
+    y = np.array([[t[0] + 0.5 * w, c[0]], [c[7], t[6] - 2 * w]])
+    assert np.array_equal(tq.near_threshold_mask(y, t, d), [[True, False], [False, False]])
+
+
 @pytest.mark.parametrize("b", [1, 2, 3, 4])
 def test_empirical_mse_matches_closed_form(b):
     d, n = 128, 20000
