@@ -12,11 +12,12 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA, TQ_ENOMEM, TQ_EWORKSPACE = range(7)
-TQ_F32, TQ_BF16 = 0, 1
+TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 TQ_MSE, TQ_PROD = 0, 1
 TQ_MAX_DIM = 4096
 TQ_MAX_TOPK = 64
 TQ_STATUS_TIMEOUT, TQ_STATUS_LAYOUT = 1, 2
+TQ_MAX_SHARDS = 64
 TQ_DECODE_STATIC_SCRATCH = 4 * 1024 * 1024
 
 if not os.path.exists(LIB_PATH):
@@ -53,6 +54,14 @@ SIGNATURES = {
     "tq_attn_decode_workspace": (_sz, [_p, _i, _i, _i, _i64]),
     "tq_attn_decode_static": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,
                                    _p, _p]),
+    "tq_attn_decode_partial": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f,
+                                    _p, _p, _sz, _p]),
+    "tq_attn_decode_partial_workspace": (_sz, [_p, _i, _i, _i, _i64]),
+    "tq_attn_merge": (_i, [_p, _p, _i, _i64, _p, _p]),
+    "tq_topk_merge": (_i, [_p, _p, _i, _i64, _i, ctypes.POINTER(ctypes.c_int64), _p, _p, _p]),
+    "tq_quant_paged": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _i, _p]),
+    "tq_attn_decode_paged": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _p, _i, _i, _p, _p, _p, _p, _i, _p, _p, _f, _p,
+                                  _p, _sz, _p]),
     "tq_device_status": (_i, [_p, ctypes.POINTER(_i)]),
     "tq_quant_gather": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _i64, _p]),
     "tq_attn_logits": (_i, [ctypes.POINTER(_p), _i, _p, _p, _i, _i, _i, _i, _i, _i64, _i64, ctypes.POINTER(_p),

@@ -12,15 +12,17 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (TQ_BF16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQ_STATUS_LAYOUT, TQ_STATUS_TIMEOUT, TQError,
+from ._lib import (TQ_BF16, TQ_F16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQ_STATUS_LAYOUT, TQ_STATUS_TIMEOUT, TQError,
                    check, lib)
 
 __all__ = [
-    "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_MAX_TOPK", "TQ_STATUS_TIMEOUT", "TQ_STATUS_LAYOUT", "TQError", "Handle", "code_words", "sign_words",
+    "TQ_MSE", "TQ_PROD", "TQ_F32", "TQ_BF16", "TQ_F16", "TQ_MAX_TOPK", "TQ_STATUS_TIMEOUT", "TQ_STATUS_LAYOUT", "TQError", "Handle", "code_words", "sign_words",
     "tq_make_codebook", "tq_make_rotation", "tq_create", "tq_quant_mse", "tq_dequant_mse", "tq_quant_prod",
     "tq_quant_prod_workspace",
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
     "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
+    "tq_attn_decode_partial", "tq_attn_decode_partial_workspace", "tq_attn_merge", "tq_topk_merge",
+    "tq_quant_paged", "tq_attn_decode_paged",
 ]
 
 
@@ -194,6 +196,68 @@ def tq_attn_decode_static(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: 
     check("tq_attn_decode_static", lib.tq_attn_decode_static(
         hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, kv_stride, _ptr(kcodes), _ptr(ksigns),
         _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out), _stream(stream)))
+
+
+def tq_attn_decode_partial_workspace(hk: Handle, B: int, Hq: int, Hkv: int, T: int) -> int:
+    return int(lib.tq_attn_decode_partial_workspace(hk.ptr, B, Hq, Hkv, T))
+
+
+def tq_attn_decode_partial(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, kv_stride: int,
+                           kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale: float, partial: torch.Tensor,
+                           workspace=None, stream=None) -> None:
+    """Softmax state [B*Hq][d + 2] (acc in the rotated value frame, m, l) of the
+    decode step over the context slice held here (T may be 0)."""
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_attn_decode_partial_workspace(hk, B, Hq, Hkv, T)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_attn_decode_partial", lib.tq_attn_decode_partial(
+        hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, kv_stride, _ptr(kcodes), _ptr(ksigns),
+        _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(partial), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+
+
+def tq_attn_merge(hv: Handle, partials: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Combine [R][rows][d + 2] slice records into out [rows][d]."""
+    R, rows = partials.shape[0], partials.shape[1]
+    check("tq_attn_merge", lib.tq_attn_merge(hv.ptr, _ptr(partials), R, rows, _ptr(out), _stream(stream)))
+
+
+def tq_topk_merge(val: torch.Tensor, idx: torch.Tensor, offsets, out_idx: torch.Tensor, out_val: torch.Tensor,
+                  stream=None) -> None:
+    """Global top-k from [R][nq][k] per-slice lists; offsets[r] = first global index of slice r."""
+    R, nq, k = val.shape
+    offs = (ctypes.c_int64 * R)(*[int(o) for o in offsets])
+    check("tq_topk_merge", lib.tq_topk_merge(_ptr(val), _ptr(idx), R, nq, k, offs, _ptr(out_idx), _ptr(out_val),
+                                             _stream(stream)))
+
+
+def _rn_code(t) -> int:
+    return TQ_F16 if t.dtype == torch.float16 else TQ_F32
+
+
+def tq_quant_paged(h: Handle, x: torch.Tensor, slots: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,
+                   signs=None, rnorms=None, channels=None, stream=None) -> None:
+    """Quantize the rows of x into cache rows slots[i] (int64); rnorms may be
+    float32 or float16 storage."""
+    rn_dtype = _rn_code(rnorms) if rnorms is not None else TQ_F32
+    check("tq_quant_paged", lib.tq_quant_paged(h.ptr, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1], _ptr(channels),
+                                               _ptr(slots), _ptr(codes), _ptr(signs), _ptr(norms), _ptr(rnorms),
+                                               rn_dtype, _stream(stream)))
+
+
+def tq_attn_decode_paged(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, block_table: torch.Tensor,
+                         page_size: int, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale: float,
+                         out: torch.Tensor, workspace=None, stream=None) -> None:
+    """Decode over a paged cache; block_table is [B*Hkv][max_pages] int32."""
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_attn_decode_workspace(hk, B, Hq, Hkv, T)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_attn_decode_paged", lib.tq_attn_decode_paged(
+        hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, _ptr(block_table), block_table.shape[1], page_size,
+        _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _rn_code(krnorms), _ptr(vcodes), _ptr(vnorms),
+        float(scale), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def tq_device_status(h: Handle) -> int:

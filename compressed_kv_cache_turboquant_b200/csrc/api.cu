@@ -257,6 +257,25 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
         split_into(Td[(size_t)n * d + k], &gst[(size_t)n * w2 + dp + k], &gst[((size_t)dp + n) * w2 + dp + k]);
       }
   }
+  // fused quantizer pieces (d <= 256): hi and remainder of kFusedPieceScale * Pi / T
+  std::vector<uint16_t> fzp, fzt;
+  const int n16 = (d + 15) / 16 * 16, k64 = (d + 63) / 64 * 64;
+  if (d <= 256) {
+    auto fill = [&](const double* M, std::vector<uint16_t>& out) {
+      out.assign((size_t)2 * n16 * k64, 0);
+      for (int n = 0; n < d; ++n)
+        for (int k = 0; k < d; ++k) {
+          const double v = (double)kFusedPieceScale * M[(size_t)n * d + k];
+          const uint16_t hb = half_bits(v);
+          out[(size_t)n * k64 + k] = hb;
+          out[((size_t)n16 + n) * k64 + k] = half_bits(v - half_value(hb));
+        }
+    };
+    fill(Pi, fzp);
+    if (variant == TQ_PROD) fill(Td.data(), fzt);
+    h->fz_n16 = n16;
+    h->fz_k64 = k64;
+  }
   std::vector<float> cf(K), tf(K);
   for (int k = 0; k < K; ++k) cf[k] = (float)h->host_centroids[k];
   for (int k = 0; k + 1 < K; ++k) tf[k] = (float)h->host_thresholds[k];
@@ -310,6 +329,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   const size_t oTabs = take(8 * 4);
   const size_t oGenPi = take(gpi.size() * 2);
   const size_t oGenSt = gst.empty() ? 0 : take(gst.size() * 2);
+  const size_t oFzPi = fzp.empty() ? 0 : take(fzp.size() * 2);
+  const size_t oFzT = fzt.empty() ? 0 : take(fzt.size() * 2);
   h->block_bytes = off;
   e = cudaMalloc(&h->block, h->block_bytes);
   if (e != cudaSuccess) {
@@ -327,6 +348,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   h->dev.lut_dq = (uint32_t*)(base + oLut);
   h->dev.gen_pi = (uint16_t*)(base + oGenPi);
   if (!gst.empty()) h->dev.gen_st = (uint16_t*)(base + oGenSt);
+  if (!fzp.empty()) h->dev.fz_pi = (uint16_t*)(base + oFzPi);
+  if (!fzt.empty()) h->dev.fz_t = (uint16_t*)(base + oFzT);
   if (has_ktab) h->dev.ktab = (uint32_t*)(base + oTabs);
   if (has_vtab) h->dev.vtab = (uint32_t*)(base + oTabs + 16);
   if (variant == TQ_PROD) {
@@ -362,6 +385,10 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   if (e == cudaSuccess) e = cudaMemcpy(h->dev.gen_pi, gpi.data(), gpi.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && !gst.empty())
     e = cudaMemcpy(h->dev.gen_st, gst.data(), gst.size() * 2, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !fzp.empty())
+    e = cudaMemcpy(h->dev.fz_pi, fzp.data(), fzp.size() * 2, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !fzt.empty())
+    e = cudaMemcpy(h->dev.fz_t, fzt.data(), fzt.size() * 2, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && variant == TQ_PROD) {
     e = cudaMemcpy(h->dev.S, Sf.data(), dd * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dev.TT, TTf.data(), dd * 4, cudaMemcpyHostToDevice);
@@ -426,6 +453,8 @@ extern "C" int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, in
   if (N == 0) return clear_error();
   int e = quant_tc_supported(h, dtype)
               ? launch_quant_mse_tc(h, x, N, x_stride, codes, norms, out_stride, stream)
+          : quant_fused_supported(h)
+              ? launch_quant_fused(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream)
           : quant_gen_supported(h)
               ? launch_quant_gen(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, nullptr, 0,
                                  stream)
@@ -449,7 +478,9 @@ static int quant_prod_impl(const char* fn, tq_handle h, const void* x, int dtype
                      (size_t)128 * quant_gen_workspace_rows_bytes(h));
   // tensor cores unless this d needs the residual workspace and none was given
   const bool gen = quant_gen_supported(h) && (!need_ws || workspace);
-  int e = gen ? launch_quant_gen(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, workspace,
+  int e = quant_fused_supported(h)
+              ? launch_quant_fused(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream)
+          : gen ? launch_quant_gen(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, workspace,
                                  ws_bytes, stream)
               : launch_quant_simple(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream);
   return e ? cuda_error(fn, e) : clear_error();
@@ -557,7 +588,7 @@ size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t 
 int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
                     int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
                     const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
-                    float scale, float* out, void* workspace, void* stream) {
+                    float scale, float* out, void* workspace, void* stream, int partial_out, PagedCache pg) {
   const size_t nq = (size_t)B * Hq;
   char* ws = (char*)workspace;
   const size_t q32 = align_up(nq * hk->d * 4, 256);
@@ -568,15 +599,17 @@ int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dty
   float* partials = (float*)((char*)qscale + align_up(nq * 2 * 4, 256));
   int e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)nq, qrot, qproj, stream);
   if (e) return e;
-  if (decode_mma_supported(hk, hv, Hq, Hkv, kv_stride)) {
+  const bool mma = pg.page ? decode_mma_supported(hk, hv, Hq, Hkv, 4) && pg.page % 8 == 0
+                            : decode_mma_supported(hk, hv, Hq, Hkv, kv_stride) && (!pg.rn16 || kv_stride % 8 == 0);
+  if (mma) {
     e = launch_qfrag(qrot, qproj, (int64_t)nq, qfrag, qscale, stream);
     if (e) return e;
     return launch_decode_mma(hk, hv, (const uint32_t*)qfrag, qscale, B, Hq, Hkv, T, kv_stride, kcodes, ksigns,
-                             knorms, krnorms, vcodes, vnorms, scale, partials, out, stream);
+                             knorms, krnorms, vcodes, vnorms, scale, partials, out, stream, partial_out, pg);
   }
   const int splits = decode_splits(B, Hq, T, hk->sm_count);
   return launch_decode_simple(hk, hv, qrot, qproj, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms,
-                              vcodes, vnorms, scale, splits, partials, out, stream);
+                              vcodes, vnorms, scale, splits, partials, out, stream, partial_out, pg);
 }
 
 }  // namespace tqi

@@ -101,7 +101,22 @@ struct DecArgs {
   uint32_t dyn_base;       // where the host measured the dynamic window to start
   uint64_t wait_ns;        // limit of every pipeline wait
   int stall;               // diagnostic: consumers first wait on a barrier nothing completes
+  // paged cache (page > 0): token t of (batch, kv-head) bh is row
+  // block_table[bh * max_pages + t / page] * page + t % page of every array
+  const int32_t* block_table;
+  int max_pages, page;
+  int rn16;                // residual norms stored as fp16
 };
+
+// cache row of token t of (batch, kv-head) bh
+__device__ __forceinline__ int64_t cache_row(const DecArgs& a, int64_t bh, int64_t t) {
+  if (a.page == 0) return bh * a.kv_stride + t;
+  return (int64_t)a.block_table[bh * a.max_pages + t / a.page] * a.page + t % a.page;
+}
+
+__device__ __forceinline__ float rnorm_at(const DecArgs& a, int64_t row) {
+  return a.rn16 ? __half2float(reinterpret_cast<const __half*>(a.krnorms)[row]) : a.krnorms[row];
+}
 
 // CTA i of G owns the global blocks [i*total/G, (i+1)*total/G); a global block
 // gb is block gb % nblk of (batch, kv-head) gb / nblk
@@ -204,17 +219,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         const int64_t bh = cur.bh;
         const int64_t t0 = cur.blk * kBlk;
         const int n = (int)min((int64_t)kBlk, a.T - t0);
-        const int n4 = n & ~3;  // norms are copied in whole 16-byte units
         uint8_t* st = stages + s * kStageBytes;
-        const int64_t r = bh * a.kv_stride + t0;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(n * (kKW + kSW + kVW) * 4 + 3 * n4 * 4));
-        bulk_load(st + kOffK, a.kcodes + r * kKW, n * kKW * 4, &full[s]);
-        bulk_load(st + kOffS, a.ksigns + r * kSW, n * kSW * 4, &full[s]);
-        bulk_load(st + kOffV, a.vcodes + r * kVW, n * kVW * 4, &full[s]);
-        if (n4) {
-          bulk_load(st + kOffN, a.knorms + r, n4 * 4, &full[s]);
-          bulk_load(st + kOffR, a.krnorms + r, n4 * 4, &full[s]);
-          bulk_load(st + kOffVN, a.vnorms + r, n4 * 4, &full[s]);
+        // The block's rows come in contiguous pieces: the whole block of a dense
+        // cache, or its part in each page.  Norms move in whole 16-byte units
+        // (4 fp32 or 8 fp16 rows); piece starts are multiples of 8 rows, so only
+        // the block's last few rows can be left for the consumers to read
+        // from global memory.
+        const int rnu = a.rn16 ? 8 : 4;
+        for (int pass = 0; pass < 2; ++pass) {
+          uint32_t tx = 0;
+          for (int off = 0; off < n;) {
+            const int64_t t = t0 + off;
+            const int len = a.page ? (int)min((int64_t)(n - off), (int64_t)(a.page - t % a.page)) : n;
+            const int64_t r = cache_row(a, bh, t);
+            const int l4 = len & ~3, lr = len & ~(rnu - 1);
+            if (pass == 0) {
+              tx += (uint32_t)(len * (kKW + kSW + kVW) * 4 + 2 * l4 * 4 + lr * (a.rn16 ? 2 : 4));
+            } else {
+              bulk_load(st + kOffK + off * kKW * 4, a.kcodes + r * kKW, len * kKW * 4, &full[s]);
+              bulk_load(st + kOffS + off * kSW * 4, a.ksigns + r * kSW, len * kSW * 4, &full[s]);
+              bulk_load(st + kOffV + off * kVW * 4, a.vcodes + r * kVW, len * kVW * 4, &full[s]);
+              if (l4) {
+                bulk_load(st + kOffN + off * 4, a.knorms + r, l4 * 4, &full[s]);
+                bulk_load(st + kOffVN + off * 4, a.vnorms + r, l4 * 4, &full[s]);
+              }
+              if (lr) {
+                const int esz = a.rn16 ? 2 : 4;
+                bulk_load(st + kOffR + off * esz, reinterpret_cast<const uint8_t*>(a.krnorms) + r * esz, lr * esz,
+                          &full[s]);
+              }
+            }
+            off += len;
+          }
+          if (pass == 0) mbar_arrive_expect_tx(&full[s], tx);
         }
       }
       // Before the CTA may exit, every copy issued into its shared memory must
@@ -383,26 +420,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           kn[r] = __uint_as_float(lds32(na + 32 * r));
-          kr[r] = __uint_as_float(lds32(na + (kOffR - kOffN) + 32 * r));
           vn[r] = __uint_as_float(lds32(na + (kOffVN - kOffN) + 32 * r));
         }
+        if (a.rn16) {
+          const __half* rh = reinterpret_cast<const __half*>(st + kOffR);
+          kr[0] = __half2float(rh[tb + g]);
+          kr[1] = __half2float(rh[tb + g + 8]);
+        } else {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) kr[r] = __uint_as_float(lds32(na + (kOffR - kOffN) + 32 * r));
+        }
       } else {
-        const int n4 = n & ~3;
-        const int64_t row0 = bh * a.kv_stride + t0;
+        const int n4 = n & ~3, nr = a.rn16 ? (n & ~7) : n4;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int tok = tb + g + 8 * r;
           if (tok < n4) {
             kn[r] = reinterpret_cast<const float*>(st + kOffN)[tok];
-            kr[r] = reinterpret_cast<const float*>(st + kOffR)[tok];
             vn[r] = reinterpret_cast<const float*>(st + kOffVN)[tok];
           } else if (tok < n) {
-            kn[r] = a.knorms[row0 + tok];
-            kr[r] = a.krnorms[row0 + tok];
-            vn[r] = a.vnorms[row0 + tok];
+            const int64_t row = cache_row(a, bh, t0 + tok);
+            kn[r] = a.knorms[row];
+            vn[r] = a.vnorms[row];
           } else {
-            kn[r] = kr[r] = vn[r] = 0.f;
+            kn[r] = vn[r] = 0.f;
           }
+          if (tok < nr)
+            kr[r] = a.rn16 ? __half2float(reinterpret_cast<const __half*>(st + kOffR)[tok])
+                           : reinterpret_cast<const float*>(st + kOffR)[tok];
+          else
+            kr[r] = tok < n ? rnorm_at(a, cache_row(a, bh, t0 + tok)) : 0.f;
         }
       }
       // logits in base 2: [token r][head j]; tokens past the context end are -inf
@@ -491,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
 // One CTA per (batch, q-head).
 __global__ void __launch_bounds__(128) decode_merge_persistent_kernel(const float* partials, int64_t G, int max_seg,
                                                                       int64_t nblk, int64_t total, int Hq, int Hkv,
-                                                                      const float* PiV, float* out) {
+                                                                      const float* PiV, float* out, int partial_out) {
   __shared__ float orot[D];
   __shared__ float ML[2];
   __shared__ int64_t range[2];
@@ -532,7 +579,13 @@ __global__ void __launch_bounds__(128) decode_merge_persistent_kernel(const floa
       const float* p = partials + ((k * max_seg + sg) * 4 + hd) * (D + 2);
       v += p[j] * __expf(p[D] - M);
     }
-    orot[j] = v * invL;
+    orot[j] = partial_out ? v : v * invL;
+  }
+  if (partial_out) {  // the merged record (acc, m, l) in the rotated frame
+    float* o = out + bq * (D + 2);
+    for (int j = threadIdx.x; j < D; j += blockDim.x) o[j] = orot[j];
+    if (threadIdx.x == 0) o[D] = M, o[D + 1] = ML[1];
+    return;
   }
   __syncthreads();
   for (int i2 = threadIdx.x; i2 < D; i2 += blockDim.x) {
@@ -567,7 +620,8 @@ int decode_mma_max_seg(int B, int Hkv, int64_t T, int sm_count) {
 int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
                       int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
-                      const float* vnorms, float scale, float* partials, float* out, void* stream) {
+                      const float* vnorms, float scale, float* partials, float* out, void* stream,
+                      int partial_out, PagedCache pg) {
   DecArgs a;
   a.kcodes = kcodes;
   a.ksigns = ksigns;
@@ -594,6 +648,10 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   a.dyn_base = hk->dyn_base;
   a.wait_ns = hk->debug_stall_ns ? hk->debug_stall_ns : kWaitLimitNs;
   a.stall = hk->debug_stall_ns ? 1 : 0;
+  a.block_table = pg.block_table;
+  a.max_pages = pg.max_pages;
+  a.page = pg.page;
+  a.rn16 = pg.rn16;
   const int G = decode_mma_grid(B, Hkv, T, hk->sm_count);
   const int smem = kSmemBytes;
   const bool fixed = hk->dyn_base == kDynBaseSm100 || hk->debug_fixed_tables;
@@ -604,7 +662,7 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
   decode_merge_persistent_kernel<<<B * Hq, 128, 0, s>>>(partials, G, a.max_seg, a.nblk, a.total, Hq, Hkv,
-                                                        hv->dev.Pi, out);
+                                                        hv->dev.Pi, out, partial_out);
   return (int)cudaGetLastError();
 }
 

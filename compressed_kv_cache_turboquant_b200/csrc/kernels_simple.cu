@@ -304,7 +304,13 @@ struct DecodeArgs {
   const float* vcent;
   float scale;
   float* partials;  // [B][Hq][splits][d + 2]
+  PagedCache pg;    // page > 0: rows through the block table; rn16: fp16 residual norms
 };
+
+__device__ __forceinline__ int64_t dec_row(const DecodeArgs& a, int64_t bh, int64_t t) {
+  if (a.pg.page == 0) return bh * a.kv_stride + t;
+  return (int64_t)a.pg.block_table[bh * a.pg.max_pages + t / a.pg.page] * a.pg.page + t % a.pg.page;
+}
 
 __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) {
   extern __shared__ float sm[];
@@ -313,13 +319,14 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) 
   float* qp = sm + d;        // [d]
   float* pw = sm + 2 * d;    // [blockDim] weights p_t * n_t of the chunk
   __shared__ float red[32];
+  __shared__ int64_t prow[128];  // cache rows of the chunk
   const int split = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int h = hq / (a.Hq / a.Hkv);
   const int64_t q_off = ((int64_t)b * a.Hq + hq) * d;
   for (int j = threadIdx.x; j < d; j += blockDim.x) qr[j] = a.qrot[q_off + j], qp[j] = a.qproj[q_off + j];
   const int64_t per = (a.T + a.splits - 1) / a.splits;
   const int64_t t0 = split * per, t1 = min(a.T, t0 + per);
-  const int64_t row0 = ((int64_t)b * a.Hkv + h) * a.kv_stride;
+  const int64_t bh = (int64_t)b * a.Hkv + h;
   const int kw = ((d + 31) >> 5) * a.bk, vw = ((d + 31) >> 5) * a.bv, G = (d + 31) >> 5;
   float m = -FLT_MAX, l = 0.f;
   float acc[TQ_MAX_DIM / 128];
@@ -328,8 +335,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) 
   for (int64_t c0 = t0; c0 < t1; c0 += blockDim.x) {
     const int64_t t = c0 + threadIdx.x;
     float logit = -FLT_MAX;
+    const int64_t row = t < t1 ? dec_row(a, bh, t) : 0;
     if (t < t1) {
-      const int64_t row = row0 + t;
       const uint32_t* w = a.kcodes + row * kw;
       const uint32_t* s = a.ksigns + row * G;
       float mse = 0.f, qjl = 0.f;
@@ -337,7 +344,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) 
         mse = fmaf(qr[j], a.kcent[code_at(w, a.bk, j)], mse);
         qjl += ((s[j >> 5] >> (j & 31)) & 1u) ? qp[j] : -qp[j];
       }
-      logit = a.scale * (a.knorms[row] * mse + a.krnorms[row] * (kSqrtHalfPi / d) * qjl);
+      const float rn = a.pg.rn16 ? __half2float(reinterpret_cast<const __half*>(a.krnorms)[row]) : a.krnorms[row];
+      logit = a.scale * (a.knorms[row] * mse + rn * (kSqrtHalfPi / d) * qjl);
     }
     const float cm = block_max(logit, red);
     const float mn = fmaxf(m, cm);
@@ -346,13 +354,14 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) 
     const float corr = __expf(m - mn);
     l = l * corr + cs;
     m = mn;
-    pw[threadIdx.x] = (t < t1) ? p * a.vnorms[row0 + t] : 0.f;
+    pw[threadIdx.x] = (t < t1) ? p * a.vnorms[row] : 0.f;
+    if (t < t1) prow[threadIdx.x] = row;
     __syncthreads();
     const int cnt = (int)min((int64_t)blockDim.x, t1 - c0);
     for (int r = 0, j = threadIdx.x; j < d; ++r, j += blockDim.x) {
       float s = acc[r] * corr;
       for (int i = 0; i < cnt; ++i) {
-        const uint32_t* w = a.vcodes + (row0 + c0 + i) * vw;
+        const uint32_t* w = a.vcodes + prow[i] * vw;
         s = fmaf(pw[i], a.vcent[code_at(w, a.bv, j)], s);
       }
       acc[r] = s;
@@ -365,20 +374,30 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeArgs a) 
 }
 
 // Merge the splits with the log-sum-exp rescale, divide by the sum, rotate back
-// once: out = Pi_V^T (acc / l).  One CTA per (batch, q-head).
-__global__ void __launch_bounds__(128) decode_merge_kernel(const float* partials, int splits, int d,
-                                                           const float* PiV, float* out) {
+// once: out = Pi_V^T (acc / l).  One CTA per (batch, q-head).  Split s of row
+// bh is the (acc[d], m, l) record at partials + bh * row_stride + s * split_stride.
+// With partial_out the merged record itself (sum_s acc_s e^(m_s - M), M,
+// sum_s l_s e^(m_s - M)), still in the rotated frame, goes to out[bh][d + 2].
+__global__ void __launch_bounds__(128) decode_merge_kernel(const float* partials, int splits, int64_t split_stride,
+                                                           int64_t row_stride, int d, const float* PiV, float* out,
+                                                           int partial_out) {
   extern __shared__ float orot[];
   const int64_t bh = blockIdx.x;
-  const float* P = partials + bh * splits * (d + 2);
+  const float* P = partials + bh * row_stride;
   float M = -FLT_MAX;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, P[s * (d + 2) + d]);
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, P[s * split_stride + d]);
   float L = 0.f;
-  for (int s = 0; s < splits; ++s) L += P[s * (d + 2) + d + 1] * __expf(P[s * (d + 2) + d] - M);
+  for (int s = 0; s < splits; ++s) L += P[s * split_stride + d + 1] * __expf(P[s * split_stride + d] - M);
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     float a = 0.f;
-    for (int s = 0; s < splits; ++s) a += P[s * (d + 2) + j] * __expf(P[s * (d + 2) + d] - M);
-    orot[j] = a / L;
+    for (int s = 0; s < splits; ++s) a += P[s * split_stride + j] * __expf(P[s * split_stride + d] - M);
+    orot[j] = partial_out ? a : a / L;
+  }
+  if (partial_out) {
+    float* o = out + bh * (d + 2);
+    for (int j = threadIdx.x; j < d; j += blockDim.x) o[j] = orot[j];
+    if (threadIdx.x == 0) o[d] = M, o[d + 1] = L;
+    return;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
@@ -454,22 +473,24 @@ int launch_decode_simple(const tq_ctx* hk, const tq_ctx* hv, const float* qrot,
                          const float* qproj, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
                          const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
                          const float* krnorms, const uint32_t* vcodes, const float* vnorms,
-                         float scale, int splits, float* partials, float* out, void* stream) {
+                         float scale, int splits, float* partials, float* out, void* stream, int partial_out,
+                         PagedCache pg) {
   DecodeArgs a{qrot, qproj, B, Hq, Hkv, hk->d, hk->bm, hv->bm, splits, T, kv_stride, kcodes,
                ksigns, knorms, krnorms, vcodes, vnorms, hk->dev.centroids, hv->dev.centroids,
-               scale, partials};
+               scale, partials, pg};
   cudaStream_t s = (cudaStream_t)stream;
   const size_t smem = (2 * (size_t)hk->d + 128) * sizeof(float);
   decode_split_simple_kernel<<<dim3(splits, Hq, B), 128, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  return launch_decode_merge(partials, (int64_t)B * Hq, splits, hv, out, stream);
+  return launch_decode_merge(partials, (int64_t)B * Hq, splits, hv, out, stream, hv->d + 2,
+                             (int64_t)splits * (hv->d + 2), partial_out);
 }
 
-int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out,
-                        void* stream) {
-  decode_merge_kernel<<<(unsigned)BH, 128, hv->d * sizeof(float), (cudaStream_t)stream>>>(partials, splits, hv->d,
-                                                                                      hv->dev.Pi, out);
+int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out, void* stream,
+                        int64_t split_stride, int64_t row_stride, int partial_out) {
+  decode_merge_kernel<<<(unsigned)BH, 128, hv->d * sizeof(float), (cudaStream_t)stream>>>(
+      partials, splits, split_stride, row_stride, hv->d, hv->dev.Pi, out, partial_out);
   return (int)cudaGetLastError();
 }
 

@@ -156,7 +156,7 @@ __device__ __forceinline__ uint32_t code_of(const uint32_t* w /*BM words of the 
 }
 
 __global__ void gen_norms_kernel(const void* x, int xbf16, int64_t x_stride, int64_t N, int d, float* norms,
-                                 int64_t out_stride) {
+                                 int64_t out_stride, const int32_t* channels, const int64_t* slots) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t v = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; v < N; v += warps) {
@@ -164,18 +164,18 @@ __global__ void gen_norms_kernel(const void* x, int xbf16, int64_t x_stride, int
     if (xbf16) {
       const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(x) + v * x_stride;
       for (int j = lane; j < d; j += 32) {
-        const double t = (double)__bfloat162float(p[j]);
+        const double t = (double)__bfloat162float(p[channels ? channels[j] : j]);
         acc = fma(t, t, acc);
       }
     } else {
       const float* p = static_cast<const float*>(x) + v * x_stride;
       for (int j = lane; j < d; j += 32) {
-        const double t = (double)p[j];
+        const double t = (double)p[channels ? channels[j] : j];
         acc = fma(t, t, acc);
       }
     }
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) norms[v * out_stride] = (float)sqrt(acc);
+    if (lane == 0) norms[slots ? slots[v] : v * out_stride] = (float)sqrt(acc);
   }
 }
 
@@ -598,6 +598,15 @@ bool make_f16_map(CUtensorMap* m, const void* base, int64_t kext, int64_t rows) 
 
 bool quant_gen_supported(const tq_ctx* h) { return h->dev.gen_pi != nullptr; }
 
+int launch_gen_norms(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, float* norms,
+                     int64_t out_stride, void* stream, const int32_t* channels, const int64_t* slots) {
+  const int64_t blocks = (N + 7) / 8;  // 8 warps per block, one vector per warp
+  const int grid = (int)(blocks < (int64_t)h->sm_count * 16 ? blocks : (int64_t)h->sm_count * 16);
+  gen_norms_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, dtype == TQ_BF16 ? 1 : 0, x_stride, N, h->d, norms,
+                                                          out_stride, channels, slots);
+  return (int)cudaGetLastError();
+}
+
 // the residual path (stage 3) is used for prod when d_pad > 256
 bool quant_gen_needs_workspace(const tq_ctx* h) { return h->variant == TQ_PROD && h->gen_d_pad > 256; }
 
@@ -610,13 +619,7 @@ int launch_quant_gen(const tq_ctx* h, const void* x, int dtype, int64_t N, int64
   const bool prod = h->variant == TQ_PROD;
   const int xbf16 = dtype == TQ_BF16 ? 1 : 0;
   const int esz = xbf16 ? 2 : 4;
-  {
-    const int64_t blocks = (N + 7) / 8;  // 8 warps per block, one vector per warp
-    const int grid = (int)(blocks < (int64_t)h->sm_count * 16 ? blocks : (int64_t)h->sm_count * 16);
-    gen_norms_kernel<<<grid, 256, 0, s>>>(x, xbf16, x_stride, N, h->d, norms, out_stride);
-    int e = (int)cudaGetLastError();
-    if (e) return e;
-  }
+  if (int e = launch_gen_norms(h, x, dtype, N, x_stride, norms, out_stride, stream)) return e;
   const int dp = h->gen_d_pad;
   const bool resid = prod && quant_gen_needs_workspace(h);
   // rows per launch: all of them, or as many whole 128-row tiles as the workspace holds

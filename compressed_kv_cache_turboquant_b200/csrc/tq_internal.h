@@ -54,7 +54,16 @@ struct DevConsts {
   // [S | T] as [2 d_pad][2 d_pad]
   uint16_t* gen_pi = nullptr;
   uint16_t* gen_st = nullptr;
+  // fused quantizer operands (d <= 256): fp16 pieces (hi, and the remainder
+  // itself as lo) of kFusedPieceScale * Pi and (prod) of kFusedPieceScale * T,
+  // each [2][n16][k64] (row = output coordinate, column = input coordinate,
+  // n16 = d rounded up to 16, k64 = d rounded up to 64, zero padded)
+  uint16_t* fz_pi = nullptr;
+  uint16_t* fz_t = nullptr;
 };
+
+// scale of the fused quantizer's constant pieces: keeps their fp16 remainders normal
+constexpr float kFusedPieceScale = 1024.f;
 
 }  // namespace tqi
 
@@ -85,11 +94,23 @@ struct tq_ctx {
   //                         address run and find the window elsewhere
   //                         (TQ_STATUS_LAYOUT)
   uint64_t debug_stall_ns = 0;
+  int fz_n16 = 0, fz_k64 = 0;  // fused quantizer tile shape (0: not available)
   bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 
 namespace tqi {
+
+// A paged K/V cache (page > 0): token t of (batch, kv-head) bh is row
+// block_table[bh * max_pages + t / page] * page + t % page of every array;
+// page == 0 is the dense layout (row bh * kv_stride + t).  rn16: the residual
+// norms are stored as fp16.
+struct PagedCache {
+  const int32_t* block_table = nullptr;
+  int max_pages = 0;
+  int page = 0;
+  int rn16 = 0;
+};
 
 // number of context splits tq_attn_decode uses for a (B, Hq, T) problem
 int probe_dyn_smem_base(uint32_t* scratch, uint32_t* base);
@@ -108,6 +129,17 @@ int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, in
 int launch_query_prep_gather(const tq_ctx* h, const void* q, int q_dtype, int64_t nq, int dq,
                              const int32_t* channels, float* qrot, float* qproj, void* stream);
 bool quant_gen_supported(const tq_ctx* h);
+// n_i = ||x_i|| in float64 -> norms[out row of i] (channels / slots as for the fused quantizer)
+int launch_gen_norms(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, float* norms,
+                     int64_t out_stride, void* stream, const int32_t* channels = nullptr,
+                     const int64_t* slots = nullptr);
+bool quant_fused_supported(const tq_ctx* h);
+// d <= 256: norms, then one persistent tensor-core kernel for codes (and QJL bits, ||r||).
+// channels: optional gather of each row's d channels; slots: optional output row per
+// vector (else i * out_stride); rn_f16: rnorms is __half storage
+int launch_quant_fused(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
+                       uint32_t* signs, float* norms, void* rnorms, int64_t out_stride, void* stream,
+                       const int32_t* channels = nullptr, const int64_t* slots = nullptr, int rn_f16 = 0);
 bool quant_gen_needs_workspace(const tq_ctx* h);
 size_t quant_gen_workspace_rows_bytes(const tq_ctx* h);
 int launch_quant_gen(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
@@ -138,8 +170,10 @@ int launch_scores_simple(const tq_ctx* h, const float* qrot, const float* qproj,
                          const float* rnorms, int64_t N, float* scores, void* stream);
 int launch_topk_simple(const float* scores, int64_t nq, int64_t N, int k, int32_t* top_idx,
                        float* top_val, void* stream);
+// merge of decode partials: split s of row bh at partials + bh * row_stride + s * split_stride;
+// partial_out writes the merged (acc, m, l) record [BH][d + 2] instead of the rotated output
 int launch_decode_merge(const float* partials, int64_t BH, int splits, const tq_ctx* hv, float* out,
-                        void* stream);
+                        void* stream, int64_t split_stride, int64_t row_stride, int partial_out = 0);
 bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride);
 int decode_mma_grid(int B, int Hkv, int64_t T, int sm_count);
 int decode_mma_max_seg(int B, int Hkv, int64_t T, int sm_count);
@@ -147,17 +181,22 @@ int launch_qfrag(const float* qrot, const float* qproj, int64_t nq, void* qfrag,
 int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
                       int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
-                      const float* vnorms, float scale, float* partials, float* out, void* stream);
-// decode attention through whichever kernel fits; workspace layout owned here
+                      const float* vnorms, float scale, float* partials, float* out, void* stream,
+                      int partial_out = 0, PagedCache pg = PagedCache());
+// decode attention through whichever kernel fits; workspace layout owned here.
+// partial_out: write the (acc[d] in the rotated value frame, m, l) record of
+// every (batch, q-head) to out [B*Hq][d + 2] instead of the normalised output
 size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t T);
 int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
                     int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
                     const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
-                    float scale, float* out, void* workspace, void* stream);
+                    float scale, float* out, void* workspace, void* stream, int partial_out = 0,
+                    PagedCache pg = PagedCache());
 int launch_decode_simple(const tq_ctx* hk, const tq_ctx* hv, const float* qrot,
                          const float* qproj, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride,
                          const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
                          const float* krnorms, const uint32_t* vcodes, const float* vnorms,
-                         float scale, int splits, float* partials, float* out, void* stream);
+                         float scale, int splits, float* partials, float* out, void* stream, int partial_out = 0,
+                         PagedCache pg = PagedCache());
 
 }  // namespace tqi

@@ -73,6 +73,7 @@ extern "C" {
 /* element types */
 #define TQ_F32 0
 #define TQ_BF16 1
+#define TQ_F16 2  /* storage of residual norms only (tq_quant_paged, tq_attn_decode_paged) */
 
 /* variants */
 #define TQ_MSE 0  /* TurboQuant_mse: b bits per coordinate */
@@ -318,6 +319,104 @@ TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int 
                                  const uint32_t* ksigns, const float* knorms, const float* krnorms,
                                  const uint32_t* vcodes, const float* vnorms, float scale, float* out,
                                  void* stream);
+
+/* ---------------------------------------------------------------- a cache split across devices */
+
+/*
+ * tq_attn_decode_partial -- the decode step of tq_attn_decode over the slice of
+ * the context held here, stopped before normalisation so that slices held by
+ * other devices can be combined with it ([tq.net, "实现步骤草图", 集成到 attention];
+ * the split itself is not on the pages: one device's HBM is the limit of a
+ * single cache).  For every (batch b, query head j) it writes the record
+ *   partial[b*Hq + j] = (acc[0..d-1], m, l),  m = max_t logit_t (natural units),
+ *   l = sum_t e^(logit_t - m),  acc = sum_t e^(logit_t - m) n_t c_V[idx_t]
+ * with acc in the rotated value frame (Pi_V is not applied).  T = 0 (an empty
+ * slice) writes acc = 0, m = -FLT_MAX, l = 0.
+ *   arguments   as tq_attn_decode (T >= 0), with
+ *   partial     dev out, [B*Hq][d + 2] float32
+ *   workspace   dev scratch of at least tq_attn_decode_partial_workspace(...) bytes
+ * Errors: as tq_attn_decode.
+ */
+TQ_API int tq_attn_decode_partial(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                                  int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                                  const float* knorms, const float* krnorms, const uint32_t* vcodes,
+                                  const float* vnorms, float scale, float* partial, void* workspace, size_t ws_bytes,
+                                  void* stream);
+TQ_API size_t tq_attn_decode_partial_workspace(tq_handle hk, int B, int Hq, int Hkv, int64_t T);
+
+/*
+ * tq_attn_merge -- combine the records of R slices and rotate back once:
+ *   M = max_r m_r,  out = Pi_V^T (sum_r e^(m_r - M) acc_r) / (sum_r e^(m_r - M) l_r)
+ *   hv        the TQ_MSE value handle of the records
+ *   partials  dev in, [R][rows][d + 2] float32 (tq_attn_decode_partial's records
+ *             of R slices, e.g. the result of an all-gather across devices)
+ *   rows      B*Hq
+ *   out       dev out, [rows][d] float32
+ * A row whose slices are all empty has no softmax: its output is NaN.
+ * Errors: TQ_EINVAL, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_attn_merge(tq_handle hv, const float* partials, int R, int64_t rows, float* out, void* stream);
+
+/*
+ * tq_topk_merge -- the global top-k of nq queries from R slices' own top-k
+ * lists (the search of [admirer, "內存價格能下來嗎？"] over a database split across
+ * devices, each scoring its slice with tq_ip_scores).
+ *   val, idx    dev in, [R][nq][k] float32 scores and int32 indices local to each
+ *               slice; a local index of INT32_MAX marks an empty candidate
+ *   offsets     host in, [R]: the global index of each slice's first key
+ *   out_idx, out_val   dev out, [nq][k]: by score descending, ties to the lower
+ *               global index (INT32_MAX / -FLT_MAX where fewer than k candidates exist)
+ * Errors: TQ_EINVAL (R outside 1..TQ_MAX_SHARDS, k outside 1..TQ_MAX_TOPK), TQ_EALIGN, TQ_ECUDA.
+ */
+#define TQ_MAX_SHARDS 64
+TQ_API int tq_topk_merge(const float* val, const int32_t* idx, int R, int64_t nq, int k, const int64_t* offsets,
+                         int32_t* out_idx, float* out_val, void* stream);
+
+/* ---------------------------------------------------------------- a paged cache */
+
+/*
+ * tq_quant_paged -- quantize-on-write: quantize N vectors (tq_quant_mse /
+ * tq_quant_prod with the handle's variant) and write vector i's outputs into
+ * row slots[i] of the cache arrays, so a serving layer whose KV cache lives in
+ * pages (a block table per sequence) stores each arriving token straight into
+ * its page ([ttakun, "新旧量化方案深度权衡矩阵"]: each token is compressed as it
+ * arrives; [tmdm, "实测数据"]: only the KV store and load change).
+ *   x, dtype, N, x_stride   as tq_quant_mse (x_stride % 8 == 0 unless channels)
+ *   channels   dev in, [d] int32, or NULL: vector i is x_i[channels[0..d-1]]
+ *              (one channel group of a split cache, as tq_quant_gather)
+ *   slots      dev in, [N] int64: the cache row of each vector (rows need not be
+ *              distinct from earlier calls; two vectors of one call must not
+ *              share a row)
+ *   codes, signs, norms    dev out, cache arrays indexed by row as in tq_quant_prod
+ *   rnorms     dev out, [rows] of rn_dtype: TQ_F32, or TQ_F16 -- the residual
+ *              norm as one FP16 scalar per vector ([tq.net, "工程风险与应对",
+ *              残差范数存储]), the nearest fp16 of the float32 result
+ *   signs, rnorms are ignored for TQ_MSE handles (may be NULL)
+ * Supported for d <= 256 (TQ_EUNSUPPORTED otherwise).
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN (x and slots 16-byte aligned,
+ * the outputs 4-byte aligned), TQ_ECUDA.
+ */
+TQ_API int tq_quant_paged(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride, const int32_t* channels,
+                          const int64_t* slots, uint32_t* codes, uint32_t* signs, float* norms, void* rnorms,
+                          int rn_dtype, void* stream);
+
+/*
+ * tq_attn_decode_paged -- tq_attn_decode over a paged cache: token t of
+ * (batch b, kv-head h) is row block_table[(b*Hkv + h)*max_pages + t / page_size]
+ * * page_size + t % page_size of every cache array.
+ *   block_table   dev in, [B*Hkv][max_pages] int32 page ids (max_pages *
+ *                 page_size >= T)
+ *   page_size     tokens per page, a multiple of 8
+ *   krnorms       dev in, residual norms of rn_dtype (TQ_F32 or TQ_F16)
+ *   other arguments as tq_attn_decode (every sequence has context length T)
+ *   workspace     dev scratch of at least tq_attn_decode_workspace(hk, B, Hq, Hkv, T) bytes
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
+ */
+TQ_API int tq_attn_decode_paged(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                                int64_t T, const int32_t* block_table, int max_pages, int page_size,
+                                const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
+                                const void* krnorms, int rn_dtype, const uint32_t* vcodes, const float* vnorms,
+                                float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- channel groups */
 

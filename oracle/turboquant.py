@@ -95,7 +95,8 @@ def dequant_mse(idx: np.ndarray, norms: np.ndarray, Pi: np.ndarray, centroids: n
     return (y_hat @ Pi) * np.asarray(norms, dtype=np.float64)[:, None]
 
 
-def quant_prod(x: np.ndarray, b: int, Pi: np.ndarray, S: np.ndarray, mse_thresholds, mse_centroids):
+def quant_prod(x: np.ndarray, b: int, Pi: np.ndarray, S: np.ndarray, mse_thresholds, mse_centroids,
+               rn_dtype=np.float32):
     """TurboQuant_prod with b total bits per coordinate
     ([ttakun, "TurboQuant_mse vs TurboQuant_prod两个变体的精确分工"]: stage one is (b-1)-bit
     mse giving x_hat and the residual r; stage two keeps 1-bit QJL of r;
@@ -106,6 +107,9 @@ def quant_prod(x: np.ndarray, b: int, Pi: np.ndarray, S: np.ndarray, mse_thresho
     Readings: S is m x d with m = d (the estimator's sqrt(pi/2)/d factor implies
     m = d); both norms are float32 (one page stores the norm as float32, another
     says the residual norm costs one FP16 scalar -- float32 is taken for both).
+    ``rn_dtype=np.float16`` is that second page's storage of the residual norm
+    ([tq.net, "工程风险与应对", 残差范数存储]): ||r|| rounded once, from float64, to
+    the nearest fp16; the estimator then uses the stored value.
     b = 1 means zero mse bits: x_hat = 0 and r = x.
     """
     x = np.atleast_2d(np.asarray(x, dtype=np.float64))
@@ -120,7 +124,7 @@ def quant_prod(x: np.ndarray, b: int, Pi: np.ndarray, S: np.ndarray, mse_thresho
     r = x - x_hat
     v = r @ S.T
     signs = (v >= 0.0)
-    rn = np.sqrt(np.sum(r * r, axis=1)).astype(np.float32)
+    rn = np.sqrt(np.sum(r * r, axis=1)).astype(rn_dtype)
     return dict(idx=idx, norms=norms, signs=signs, rnorms=rn, y=y, x_hat=x_hat, r=r, Sr=v)
 
 
@@ -303,6 +307,48 @@ def attention_decode(q: np.ndarray, k_est_fn, v_hat: np.ndarray, Hkv: int, scale
             out[b, h * g:(h + 1) * g] = p @ v_hat(b, h)
             all_logits[(b, h)] = logits
     return out, all_logits
+
+
+def attention_partial(q: np.ndarray, k_est_fn, v_hat, Hkv: int, scale: float | None = None):
+    """The softmax state of one decode step over a slice of the context, to be
+    combined with the states of the other slices (the context split across
+    devices).  Same readings as ``attention_decode``; for every (batch, q-head):
+    m = max logit over the slice, l = sum_t exp(logit_t - m),
+    acc = sum_t exp(logit_t - m) v_hat_t.  An empty slice gives m = -inf, l = 0,
+    acc = 0.  Returns (m [B, Hq], l [B, Hq], acc [B, Hq, d]).  Pinned, through
+    ``merge_attention_partials``, by the softmax of the whole context."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    g = Hq // Hkv
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    m = np.full((B, Hq), -np.inf)
+    l = np.zeros((B, Hq))
+    acc = np.zeros((B, Hq, d))
+    for b in range(B):
+        for h in range(Hkv):
+            qs = q[b, h * g:(h + 1) * g]
+            logits = np.atleast_2d(k_est_fn(b, h, qs)) * scale
+            if logits.shape[1] == 0:
+                continue
+            mx = np.max(logits, axis=1)
+            p = np.exp(logits - mx[:, None])
+            m[b, h * g:(h + 1) * g] = mx
+            l[b, h * g:(h + 1) * g] = p.sum(axis=1)
+            acc[b, h * g:(h + 1) * g] = p @ v_hat(b, h)
+    return m, l, acc
+
+
+def merge_attention_partials(ms, ls, accs):
+    """Combine the softmax states of context slices: with M = max_s m_s,
+    out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s (the log-sum-exp
+    rescale).  ms, ls: [S, ...]; accs: [S, ..., d].  Returns out [..., d]."""
+    ms = np.asarray(ms, dtype=np.float64)
+    ls = np.asarray(ls, dtype=np.float64)
+    accs = np.asarray(accs, dtype=np.float64)
+    M = np.max(ms, axis=0)
+    w = np.exp(ms - M[None])                     # empty slices: exp(-inf) = 0
+    L = np.sum(w * ls, axis=0)
+    return np.sum(w[..., None] * accs, axis=0) / L[..., None]
 
 
 def topk(scores: np.ndarray, k: int):

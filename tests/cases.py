@@ -129,6 +129,51 @@ def sqrt_half_pi_over(d: int) -> float:
     return math.sqrt(math.pi / 2) / d
 
 
+def decode_cache(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
+    """A K (prod 4 bits) / V (mse 4 bits) cache [B*Hkv][T + stride_extra] on the
+    GPU: the sampled (batch, kv-head) slices hold the oracle's codes of seeded
+    synthetic keys and values, every other slot random valid words.  Returns
+    (key Instance, value Instance, cache dict, bf16-exact queries [B][Hq][d] as
+    float64, {(b, h): (oracle key record, oracle x_hat of the values)})."""
+    hk = Instance(d, 4, tq.TQ_PROD, seed=seed)
+    hv = Instance(d, 4, tq.TQ_MSE, seed=seed, rot_stream=synth.ROT_V)
+    S = T + stride_extra
+    rows = B * Hkv * S
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    rnd = lambda cols: torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, cols), dtype=torch.int32, device=DEV, generator=g)
+    c = dict(kcodes=rnd(hk.h.words), ksigns=rnd(tq.sign_words(d)), vcodes=rnd(hv.h.words))
+    c["knorms"] = torch.rand(rows, device=DEV, generator=g) * 10 + 1
+    c["krnorms"] = c["knorms"] * 0.2
+    c["vnorms"] = torch.rand(rows, device=DEV, generator=g) * 10 + 1
+    q64 = bf16_exact(synth.decode_queries(B, Hq, d, seed=seed))
+    refs = {}
+    for (b, h) in sample:
+        k64 = synth.kv_head_rows(T, d, 0, b, h, seed=seed)
+        v64 = synth.kv_head_rows(T, d, 1, b, h, seed=seed)
+        kst = hk.oracle_quant(k64)
+        vidx, vn, _ = oq.quant_mse(v64, hv.Pi_o, hv.t_o)
+        r0 = (b * Hkv + h) * S
+        c["kcodes"][r0:r0 + T] = upload_words(oq.pack_codes_vec(kst["idx"], 3))
+        c["ksigns"][r0:r0 + T] = upload_words(oq.pack_signs(kst["signs"]))
+        c["knorms"][r0:r0 + T] = torch.tensor(kst["norms"], device=DEV)
+        c["krnorms"][r0:r0 + T] = torch.tensor(kst["rnorms"], device=DEV)
+        c["vcodes"][r0:r0 + T] = upload_words(oq.pack_codes_vec(vidx, 4))
+        c["vnorms"][r0:r0 + T] = torch.tensor(vn, device=DEV)
+        refs[(b, h)] = (kst, oq.dequant_mse(vidx, vn, hv.Pi_o, hv.c_o))
+    return hk, hv, c, q64, refs
+
+
+def decode_tolerance(ref, logits, qs, kst, vhat, scale):
+    """Per-head bound on |out - ref| of a decode step: the score bound
+    1e-4 ||q|| ||k|| (scaled) propagated through the softmax, plus 1e-3
+    relative for the fp16 value table."""
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    eps = scale * 1e-4 * np.linalg.norm(qs, axis=1)[:, None] * (np.asarray(kst["norms"], dtype=np.float64)[None, :])
+    spread = np.linalg.norm(vhat[None, :, :] - ref[:, None, :], axis=2)
+    return 2 * np.sum(p * eps * spread, axis=1) + 1e-3 * np.linalg.norm(ref, axis=1)
+
+
 def assert_status_clean(*handles):
     """Every bounded wait of the calls made so far completed and every kernel
     found its shared-memory window where it was built to (reads and clears the

@@ -105,3 +105,20 @@ def test_hot_path_calls_reject_null_handle():
     assert L.tq_ip_scores_workspace(None, 1, 1, 0) == 0
     assert L.tq_attn_decode_workspace(None, 1, 1, 1, 1) == 0
     assert L.tq_destroy(None) == _lib.TQ_OK
+
+
+def test_shard_merge_calls_reject_bad_arguments_before_any_gpu_work():
+    L = _lib.lib
+    off = (ctypes.c_int64 * 2)(0, 10)
+    p = ctypes.c_void_p(16)
+    assert L.tq_topk_merge(p, p, 0, 4, 10, off, p, p, None) == _lib.TQ_EINVAL          # R = 0
+    assert L.tq_topk_merge(p, p, _lib.TQ_MAX_SHARDS + 1, 4, 10, off, p, p, None) == _lib.TQ_EINVAL
+    assert L.tq_topk_merge(p, p, 2, 4, 0, off, p, p, None) == _lib.TQ_EINVAL           # k = 0
+    assert L.tq_topk_merge(p, p, 2, 4, _lib.TQ_MAX_TOPK + 1, off, p, p, None) == _lib.TQ_EINVAL
+    assert L.tq_topk_merge(p, p, 2, 4, 10, None, p, p, None) == _lib.TQ_EINVAL         # no offsets
+    neg = (ctypes.c_int64 * 2)(0, -1)
+    assert L.tq_topk_merge(p, p, 2, 4, 10, neg, p, p, None) == _lib.TQ_EINVAL
+    assert L.tq_topk_merge(p, p, 2, 0, 10, off, p, p, None) == _lib.TQ_OK              # nothing to do
+    assert L.tq_attn_merge(None, p, 2, 4, p, None) == _lib.TQ_EINVAL
+    assert L.tq_attn_decode_partial(None, None, p, 0, 1, 4, 1, 10, 10, p, p, p, p, p, p, ctypes.c_float(0.1), p, p,
+                                    0, None) == _lib.TQ_EINVAL

@@ -16,8 +16,8 @@ import torch
 import synth
 from oracle import turboquant as oq
 
-from cases import (DEV, Instance, assert_status_clean, bf16_exact, compare_codes, compare_signs, rel_err,
-                   rel_l2_rows, to_device, upload_words, words_u32)
+from cases import (DEV, Instance, assert_status_clean, bf16_exact, compare_codes, compare_signs, decode_cache,
+                   decode_tolerance, rel_err, rel_l2_rows, to_device, upload_words, words_u32)
 
 import compressed_kv_cache_turboquant_b200 as tq
 
@@ -129,6 +129,39 @@ def test_zero_vectors_every_path(d, dtype, variant, b):
     torch.cuda.synchronize()
     _check_quant(inst, x64, out)
     assert np.all(out["norms"].cpu().numpy()[zero] == 0)
+
+
+@pytest.mark.parametrize("d", [8, 240, 256])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_tile_shape_edges(d, dtype):
+    """Dimensions at the edges of the fused tile shapes: one 16-wide K step (d = 8),
+    a partial last 32-group (d = 240) and the widest tile, whose operand ring
+    drops to two stages (d = 256); 700 rows = five tiles and a ragged tail."""
+    N = 700
+    for variant, b in [(tq.TQ_MSE, 2), (tq.TQ_PROD, 4), (tq.TQ_PROD, 3)]:
+        inst = Instance(d, b, variant, seed=d + 1)
+        x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=d)
+        if dtype == torch.bfloat16:
+            x64 = bf16_exact(x64)
+        out = inst.alloc_outputs(N)
+        inst.gpu_quant(to_device(x64, dtype), out)
+        torch.cuda.synchronize()
+        _check_quant(inst, x64, out)
+
+
+def test_search_quantize_d200_full_size_sampled():
+    """The search workload's quantize in the launch the bench times: 10^6 unit
+    fp32 vectors at d = 200, prod 4 bits; sampled rows, the first and the last
+    tiles checked against the oracle."""
+    d, N = 200, 1_000_000
+    inst = Instance(d, 4, tq.TQ_PROD, seed=0)
+    x64 = synth.unit_rows(N, d, 0)
+    out = inst.alloc_outputs(N)
+    inst.gpu_quant(to_device(x64, torch.float32), out)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([synth.rng(31, 1).choice(N, 4000, replace=False), np.arange(128),
+                                     np.arange(N - 300, N)]))
+    _check_quant(inst, x64, out, rows)
 
 
 def test_prod_many_row_tiles_per_cta():
@@ -296,36 +329,13 @@ def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
     """Quantize K (prod 4b) and V (mse 4b) with the oracle for the sampled
     (batch, kv-head) slices, random valid codes elsewhere; decode on the GPU
     and compare the sampled outputs with the oracle's attention."""
-    hk = Instance(d, 4, tq.TQ_PROD, seed=seed)
-    hv = Instance(d, 4, tq.TQ_MSE, seed=seed, rot_stream=synth.ROT_V)
+    hk, hv, c, q64, refs = decode_cache(B, Hq, Hkv, T, d, sample, seed, stride_extra)
     S = T + stride_extra
-    rows = B * Hkv * S
-    g = torch.Generator(device=DEV).manual_seed(seed)
-    kcodes = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, hk.h.words), dtype=torch.int32, device=DEV, generator=g)
-    ksigns = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, tq.sign_words(d)), dtype=torch.int32, device=DEV, generator=g)
-    vcodes = torch.randint(-2 ** 31, 2 ** 31 - 1, (rows, hv.h.words), dtype=torch.int32, device=DEV, generator=g)
-    knorms = torch.rand(rows, device=DEV, generator=g) * 10 + 1
-    krnorms = knorms * 0.2
-    vnorms = torch.rand(rows, device=DEV, generator=g) * 10 + 1
-    q64 = bf16_exact(synth.decode_queries(B, Hq, d, seed=seed))
-    refs = {}
-    for (b, h) in sample:
-        k64 = synth.kv_head_rows(T, d, 0, b, h, seed=seed)
-        v64 = synth.kv_head_rows(T, d, 1, b, h, seed=seed)
-        kst = hk.oracle_quant(k64)
-        vidx, vn, _ = oq.quant_mse(v64, hv.Pi_o, hv.t_o)
-        r0 = (b * Hkv + h) * S
-        kcodes[r0:r0 + T] = upload_words(oq.pack_codes_vec(kst["idx"], 3))
-        ksigns[r0:r0 + T] = upload_words(oq.pack_signs(kst["signs"]))
-        knorms[r0:r0 + T] = torch.tensor(kst["norms"], device=DEV)
-        krnorms[r0:r0 + T] = torch.tensor(kst["rnorms"], device=DEV)
-        vcodes[r0:r0 + T] = upload_words(oq.pack_codes_vec(vidx, 4))
-        vnorms[r0:r0 + T] = torch.tensor(vn, device=DEV)
-        refs[(b, h)] = (kst, oq.dequant_mse(vidx, vn, hv.Pi_o, hv.c_o))
     q = to_device(q64, torch.bfloat16)
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=DEV)
     scale = 1.0 / math.sqrt(d)
-    tq.tq_attn_decode(hk.h, hv.h, q, Hkv, T, S, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, scale, out)
+    tq.tq_attn_decode(hk.h, hv.h, q, Hkv, T, S, c["kcodes"], c["ksigns"], c["knorms"], c["krnorms"], c["vcodes"],
+                      c["vnorms"], scale, out)
     torch.cuda.synchronize()
     got = out.cpu().numpy()
     gsz = Hq // Hkv
@@ -336,13 +346,7 @@ def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
                                                     hk.Pi_o, hk.S, hk.c_o, 4)
         ref_out, ref_logits = oq.attention_decode(qs[None], est, lambda _b, _h: vhat, 1, scale=scale)
         ref = ref_out[0]
-        logits = ref_logits[(0, 0)]
-        p = np.exp(logits - logits.max(axis=1, keepdims=True))
-        p /= p.sum(axis=1, keepdims=True)
-        # logit tolerance of the score bound, propagated through the softmax
-        eps = scale * 1e-4 * np.linalg.norm(qs, axis=1)[:, None] * (np.asarray(kst["norms"], dtype=np.float64)[None, :])
-        spread = np.linalg.norm(vhat[None, :, :] - ref[:, None, :], axis=2)
-        tol = 2 * np.sum(p * eps * spread, axis=1) + 1e-3 * np.linalg.norm(ref, axis=1)
+        tol = decode_tolerance(ref, ref_logits[(0, 0)], qs, kst, vhat, scale)
         err = np.linalg.norm(got[b, h * gsz:(h + 1) * gsz] - ref, axis=1)
         assert np.all(err <= tol), (b, h, err, tol)
     assert_status_clean(hk, hv)

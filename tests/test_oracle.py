@@ -350,6 +350,24 @@ def _golden_packing():
     return cases
 
 
+def test_fp16_residual_norm_is_one_rounding_of_the_float64_norm():
+    # the stored fp16 norm is the nearest fp16 of ||x - x_hat|| (float64), so it
+    # is within half an fp16 ulp (2^-11 relative) of it; everything else equal
+    d, b = 64, 3
+    Pi = tq.haar_rotation(synth.gaussian_matrix(d, d, 3, synth.ROT_K))
+    S = synth.gaussian_matrix(d, d, 3, synth.QJL_K)
+    c, t = cb.lloyd_max(b - 1, d)
+    x = synth.rng(3, 3).standard_normal((400, d)) * 5
+    a = tq.quant_prod(x, b, Pi, S, t, c)
+    h = tq.quant_prod(x, b, Pi, S, t, c, rn_dtype=np.float16)
+    assert h["rnorms"].dtype == np.float16 and a["rnorms"].dtype == np.float32
+    exact = np.sqrt(np.sum((x - a["x_hat"]) ** 2, axis=1))
+    rel = np.abs(h["rnorms"].astype(np.float64) - exact) / exact
+    assert np.max(rel) <= 2.0 ** -11 and np.max(rel) > 2.0 ** -16
+    for k in ("idx", "norms", "signs"):
+        assert np.array_equal(a[k], h[k])
+
+
 @pytest.mark.parametrize("case", _golden_packing())
 def test_packing_matches_hand_built_words(case):
     b, idx, words = case
@@ -399,6 +417,37 @@ def test_attention_uniform_and_dominant_limits():
     out, lg = tq.attention_decode(q2, lambda b, h, qs: qs @ k[h].T, lambda b, h: v[h], Hkv)
     p = special.softmax(q2[0, 0] @ k[0].T / math.sqrt(d))
     assert np.allclose(out[0, 0], p @ v[0], atol=1e-13)
+
+
+def test_context_split_softmax_states_merge_to_the_full_softmax():
+    # Any split of the context into slices (an empty one included) merges back
+    # to scipy's softmax over the whole context; a single slice merges to its
+    # own normalised sum; slices of very different logit size still combine
+    B, Hq, Hkv, T, d = 2, 4, 2, 50, 6
+    r = synth.rng(4, 1)
+    k = r.standard_normal((B, Hkv, T, d))
+    v = r.standard_normal((B, Hkv, T, d))
+    q = r.standard_normal((B, Hq, d)) * 3
+    full = np.zeros((B, Hq, d))
+    for b in range(B):
+        for j in range(Hq):
+            p = special.softmax(q[b, j] @ k[b, j // 2].T / math.sqrt(d))
+            full[b, j] = p @ v[b, j // 2]
+    cuts = [0, 7, 7, 31, 50]   # slices [0,7), [7,7) (empty), [7,31), [31,50)
+    parts = [tq.attention_partial(q, lambda b, h, qs, a=a, e=e: qs @ k[b, h, a:e].T,
+                                  lambda b, h, a=a, e=e: v[b, h, a:e], Hkv)
+             for a, e in zip(cuts[:-1], cuts[1:])]
+    ms, ls, accs = (np.stack(x) for x in zip(*parts))
+    assert np.all(np.isneginf(ms[1])) and np.all(ls[1] == 0)
+    assert np.allclose(tq.merge_attention_partials(ms, ls, accs), full, atol=1e-12)
+    one = tq.attention_partial(q, lambda b, h, qs: qs @ k[b, h].T, lambda b, h: v[b, h], Hkv)
+    assert np.allclose(tq.merge_attention_partials(*(x[None] for x in one)), full, atol=1e-12)
+    out, _ = tq.attention_decode(q, lambda b, h, qs: qs @ k[b, h].T, lambda b, h: v[b, h], Hkv)
+    assert np.allclose(out, full, atol=1e-12)
+    # a slice whose logits are all far below the others' contributes ~nothing
+    ms2 = np.stack([ms[0], ms[2] - 800.0])
+    got = tq.merge_attention_partials(ms2, np.stack([ls[0], ls[2]]), np.stack([accs[0], accs[2]]))
+    assert np.allclose(got, accs[0] / ls[0][..., None], atol=1e-12)
 
 
 def test_topk_matches_sorting():
