@@ -508,10 +508,10 @@ class Stream:
         if record:
             e0, e1, e2 = E(), E(), E()
             e0.record(self.stream)
-        t = self.T - 1  # slot of the arriving token
-        for k, (h, c) in enumerate(zip(self.h, self.cache)):
-            tq.tq_quant_gather(h, self.token, self.channels[64 * k:64 * (k + 1)], c["codes"][t:], c["norms"][t:],
-                               signs=c["signs"][t:], rnorms=c["rnorms"][t:], out_stride=self.T)
+        t = self.T - 1  # slot of the arriving token: both channel groups of every kv-head in one launch
+        tq.tq_quant_gather_groups(self.h, self.token, self.channels, [c["codes"][t:] for c in self.cache],
+                                  [c["norms"][t:] for c in self.cache], signs=[c["signs"][t:] for c in self.cache],
+                                  rnorms=[c["rnorms"][t:] for c in self.cache], out_stride=self.T)
         if record:
             e1.record(self.stream)
         self.logits_only()

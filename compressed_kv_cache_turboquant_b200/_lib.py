@@ -64,6 +64,8 @@ SIGNATURES = {
                                   _p, _sz, _p]),
     "tq_device_status": (_i, [_p, ctypes.POINTER(_i)]),
     "tq_quant_gather": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _i64, _p]),
+    "tq_quant_gather_groups": (_i, [ctypes.POINTER(_p), _i, _p, _i, _i64, _i64, _p, ctypes.POINTER(_p),
+                                    ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), _i64, _p]),
     "tq_attn_logits": (_i, [ctypes.POINTER(_p), _i, _p, _p, _i, _i, _i, _i, _i, _i64, _i64, ctypes.POINTER(_p),
                             ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), _f, _p, _p, _sz, _p]),
     "tq_attn_logits_workspace": (_sz, [ctypes.POINTER(_p), _i, _i, _i]),

@@ -22,7 +22,7 @@ __all__ = [
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
     "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
     "tq_attn_decode_partial", "tq_attn_decode_partial_workspace", "tq_attn_merge", "tq_topk_merge",
-    "tq_quant_paged", "tq_attn_decode_paged",
+    "tq_quant_paged", "tq_attn_decode_paged", "tq_quant_gather_groups",
 ]
 
 
@@ -272,6 +272,19 @@ def tq_quant_gather(h: Handle, x: torch.Tensor, channels: torch.Tensor, codes: t
     check("tq_quant_gather", lib.tq_quant_gather(h.ptr, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1],
                                                  _ptr(channels), _ptr(codes), _ptr(signs), _ptr(norms),
                                                  _ptr(rnorms), out_stride, _stream(stream)))
+
+
+def tq_quant_gather_groups(handles, x: torch.Tensor, channels: torch.Tensor, codes, norms, signs=None, rnorms=None,
+                           out_stride: int = 1, stream=None) -> None:
+    """Every channel group of the rows of x in one launch; codes / norms /
+    signs / rnorms are lists with one tensor (or None) per group."""
+    n = len(handles)
+    hs = (ctypes.c_void_p * n)(*[h.ptr for h in handles])
+    signs = signs or [None] * n
+    rnorms = rnorms or [None] * n
+    check("tq_quant_gather_groups", lib.tq_quant_gather_groups(
+        hs, n, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1], _ptr(channels), _ptr_array(codes),
+        _ptr_array(signs), _ptr_array(norms), _ptr_array(rnorms), out_stride, _stream(stream)))
 
 
 def _ptr_array(items):

@@ -34,17 +34,23 @@ int clear_error() {
   return TQ_OK;
 }
 
+// The attribute is one value per (kernel, device), the largest dynamic window a
+// launch may ask for; it is raised once to the device's opt-in maximum, so
+// launches of one kernel with different window sizes (one per d) never lower it.
 int ensure_dyn_smem(const void* kernel, int bytes) {
   static std::mutex mu;
-  static std::set<std::tuple<const void*, int, int>> done;
+  static std::set<std::pair<const void*, int>> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return (int)e;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(kernel, dev, bytes);
-  if (done.count(key)) return (int)cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert(key);
+  if (done.count({kernel, dev})) return (int)cudaSuccess;
+  int maxb = 0;
+  e = cudaDeviceGetAttribute(&maxb, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return (int)e;
+  if (bytes > maxb) return (int)cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+  if (e == cudaSuccess) done.insert({kernel, dev});
   return (int)e;
 }
 
@@ -665,9 +671,54 @@ extern "C" int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N,
     if (reinterpret_cast<uintptr_t>(p) & 3u)
       return set_error(TQ_EALIGN, "tq_quant_gather: a device pointer is not 4-byte aligned");
   if (N == 0) return clear_error();
-  int e = launch_quant_simple(h, x, dtype, N, x_stride, codes, prod ? signs : nullptr, norms, prod ? rnorms : nullptr,
-                              out_stride, stream, channels);
+  // bulk gathers (a cache fill) on the tensor cores; a few arriving tokens in one short launch
+  const bool bulk = N >= 256 && quant_fused_supported(h) && !(reinterpret_cast<uintptr_t>(x) & 15u);
+  int e;
+  if (bulk) {
+    e = launch_quant_fused(h, x, dtype, N, x_stride, codes, prod ? signs : nullptr, norms, prod ? rnorms : nullptr,
+                           out_stride, stream, channels);
+  } else if (h->d <= 256 && N < 65536) {
+    uint32_t* sg = prod ? signs : nullptr;
+    float* rn = prod ? rnorms : nullptr;
+    e = launch_quant_small(&h, 1, x, dtype, N, x_stride, channels, &codes, &sg, &norms, &rn, out_stride, stream);
+  } else {
+    e = launch_quant_simple(h, x, dtype, N, x_stride, codes, prod ? signs : nullptr, norms, prod ? rnorms : nullptr,
+                            out_stride, stream, channels);
+  }
   return e ? cuda_error("tq_quant_gather", e) : clear_error();
+}
+
+extern "C" int tq_quant_gather_groups(const tq_handle* h, int ngroups, const void* x, int dtype, int64_t N,
+                                      int64_t x_stride, const int32_t* channels, uint32_t* const* codes,
+                                      uint32_t* const* signs, float* const* norms, float* const* rnorms,
+                                      int64_t out_stride, void* stream) {
+  const char* fn = "tq_quant_gather_groups";
+  if (!h || ngroups < 1 || ngroups > 2) return set_error(TQ_EINVAL, "%s: need 1 or 2 groups", fn);
+  if (N < 0 || N >= 65536) return set_error(TQ_EINVAL, "%s: N = %lld (need 0 <= N < 65536)", fn, (long long)N);
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return set_error(TQ_EUNSUPPORTED, "%s: dtype %d", fn, dtype);
+  if (x_stride < 1 || out_stride < 1) return set_error(TQ_EINVAL, "%s: stride < 1", fn);
+  if (!codes || !norms || (N > 0 && (!x || !channels))) return set_error(TQ_EINVAL, "%s: NULL pointer", fn);
+  for (int g = 0; g < ngroups; ++g) {
+    if (!h[g]) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
+    if (h[g]->d > 256) return set_error(TQ_EUNSUPPORTED, "%s: d = %d (need <= 256)", fn, h[g]->d);
+    const bool prod = h[g]->variant == TQ_PROD;
+    if (!codes[g] || !norms[g] || (prod && (!signs || !rnorms || !signs[g] || !rnorms[g])))
+      return set_error(TQ_EINVAL, "%s: NULL pointer of group %d", fn, g);
+    for (const void* p : {(const void*)codes[g], (const void*)norms[g], prod ? (const void*)signs[g] : nullptr,
+                          prod ? (const void*)rnorms[g] : nullptr})
+      if (reinterpret_cast<uintptr_t>(p) & 3u) return set_error(TQ_EALIGN, "%s: a pointer is not 4-byte aligned", fn);
+  }
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(channels)) & 3u)
+    return set_error(TQ_EALIGN, "%s: a pointer is not 4-byte aligned", fn);
+  if (N == 0) return clear_error();
+  uint32_t* sg[2] = {nullptr, nullptr};
+  float* rn[2] = {nullptr, nullptr};
+  for (int g = 0; g < ngroups; ++g)
+    if (h[g]->variant == TQ_PROD) sg[g] = signs[g], rn[g] = rnorms[g];
+  const tq_ctx* hs[2] = {h[0], ngroups > 1 ? h[1] : nullptr};
+  const int e = launch_quant_small(hs, ngroups, x, dtype, N, x_stride, channels, codes, sg, norms, rn, out_stride,
+                                   stream);
+  return e ? cuda_error(fn, e) : clear_error();
 }
 
 extern "C" size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, int Hq) {

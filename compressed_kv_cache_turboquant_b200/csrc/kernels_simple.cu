@@ -176,6 +176,105 @@ __global__ void __launch_bounds__(128) quant_simple_kernel(QuantArgs a) {
   }
 }
 
+// Small batches (one arriving token per kv-head): one launch quantizes every
+// channel group of every vector, CTA (vector, group), 256 threads.  Each
+// mat-vec (Pi x, then T u) splits the input coordinates into 256 / d parts
+// whose partial sums meet in shared memory, so a thread's dependent FMA chain
+// is d^2 / 256 long instead of d; the norm is summed in float64.
+struct SmallGroup {
+  const float* PiT;          // [i][j] = Pi[j][i]
+  const float* TT;           // [i][j] = T[j][i]
+  const float* centroids;
+  const float* thresholds;
+  const int32_t* channels;   // [d] channels of the input row
+  uint32_t* codes;
+  uint32_t* signs;
+  float* norms;
+  float* rnorms;
+  int d, bm, prod;
+};
+
+struct SmallArgs {
+  const void* x;
+  int64_t N, x_stride, out_stride;
+  SmallGroup g[2];
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(256) quant_small_kernel(SmallArgs a) {
+  const SmallGroup& G = a.g[blockIdx.y];
+  const int64_t v = blockIdx.x;
+  const int d = G.d, t = threadIdx.x;
+  __shared__ float xs[256], ys[256], us[256], part[256];
+  __shared__ uint8_t sidx[256];
+  __shared__ double redd[8];
+  __shared__ float red[8];
+  __shared__ float thr[16];
+  const int parts = 256 / d;            // d <= 256
+  const int j = t % d, p = t / d;       // output coordinate and input part of this thread
+  const int i0 = p * d / parts, i1 = (p + 1) * d / parts;
+  const TIn* x = static_cast<const TIn*>(a.x) + v * a.x_stride;
+  double ss = 0.0;
+  if (t < d) {
+    const float e = load_elem(x, G.channels ? G.channels[t] : t);
+    xs[t] = e;
+    ss = (double)e * e;
+  }
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((t & 31) == 0) redd[t >> 5] = ss;
+  __syncthreads();
+  double tot = 0.0;
+  for (int w = 0; w < 8; ++w) tot += redd[w];
+  const float n = (float)sqrt(tot);
+  const int K = 1 << G.bm;
+  if (t < K - 1) thr[t] = n * G.thresholds[t];
+  // y = Pi x, split over the input coordinates
+  float acc = 0.f;
+  if (p < parts) {
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) acc = fmaf(G.PiT[(int64_t)i * d + j], xs[i], acc);
+  }
+  part[t] = acc;
+  __syncthreads();
+  const int64_t slot = v * a.out_stride;
+  if (t < d) {
+    float y = 0.f;
+    for (int q = 0; q < parts; ++q) y += part[q * d + t];
+    int idx = 0;
+    for (int k = 0; k < K - 1; ++k) idx += (y >= thr[k]) ? 1 : 0;
+    sidx[t] = (uint8_t)idx;
+    us[t] = (G.prod && n > 0.f) ? (y / n - G.centroids[idx]) : 0.f;
+  }
+  __syncthreads();
+  const int Gw = (d + 31) >> 5, words = Gw * G.bm;
+  if (t < words) G.codes[slot * words + t] = pack_word(sidx, d, G.bm, t / G.bm, t % G.bm);
+  if (t == 0) G.norms[slot] = n;
+  if (!G.prod) return;
+  float uu = t < d ? us[t] * us[t] : 0.f;
+  for (int o = 16; o > 0; o >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, o);
+  if ((t & 31) == 0) red[t >> 5] = uu;
+  // V = T u, split the same way
+  acc = 0.f;
+  if (p < parts) {
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) acc = fmaf(G.TT[(int64_t)i * d + j], us[i], acc);
+  }
+  part[t] = acc;
+  __syncthreads();
+  if (t < d) {
+    float vv = 0.f;
+    for (int q = 0; q < parts; ++q) vv += part[q * d + t];
+    sidx[t] = vv >= 0.f ? 1 : 0;
+  }
+  __syncthreads();
+  if (t < Gw) G.signs[slot * Gw + t] = pack_word(sidx, d, 1, t, 0);
+  if (t == 0) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += red[w];
+    G.rnorms[slot] = n * sqrtf(s);
+  }
+}
+
 // One CTA per vector: y_hat_j = c[idx_j] (shared), x_hat_i = n sum_j Pi[j][i] y_hat_j.
 template <typename TOut>
 __global__ void __launch_bounds__(128) dequant_simple_kernel(const uint32_t* codes, const float* norms,
@@ -410,6 +509,32 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float* partials
 int grid_for(int64_t n, int cap) { return (int)((n < cap) ? (n > 0 ? n : 1) : cap); }
 
 }  // namespace
+
+int launch_quant_small(const tq_ctx* const* h, int ngroups, const void* x, int dtype, int64_t N, int64_t x_stride,
+                       const int32_t* channels, uint32_t* const* codes, uint32_t* const* signs, float* const* norms,
+                       float* const* rnorms, int64_t out_stride, void* stream) {
+  SmallArgs a;
+  a.x = x;
+  a.N = N;
+  a.x_stride = x_stride;
+  a.out_stride = out_stride;
+  int off = 0;
+  for (int g = 0; g < ngroups; ++g) {
+    const tq_ctx* hg = h[g];
+    const bool prod = hg->variant == TQ_PROD;
+    a.g[g] = SmallGroup{hg->dev.PiT, hg->dev.TT, hg->dev.centroids, hg->dev.thresholds,
+                        channels ? channels + off : nullptr, codes[g], prod ? signs[g] : nullptr, norms[g],
+                        prod ? rnorms[g] : nullptr, hg->d, hg->bm, prod ? 1 : 0};
+    off += hg->d;
+  }
+  const dim3 grid((unsigned)N, (unsigned)ngroups);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == TQ_BF16)
+    quant_small_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  else
+    quant_small_kernel<float><<<grid, 256, 0, s>>>(a);
+  return (int)cudaGetLastError();
+}
 
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,

@@ -12,10 +12,10 @@ namespace tqi {
 int set_error(int code, const char* fmt, ...);
 int clear_error();
 
-// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
-// device.  The setting belongs to the device that is current when it is made,
-// so it is applied once per (kernel, device); safe to call from several host
-// threads.  Returns a cudaError_t.
+// Let a kernel use a dynamic shared-memory window of `bytes` on the current
+// device: its limit is raised to the device's opt-in maximum once per
+// (kernel, device) -- the setting belongs to the device current when it is
+// made.  Safe to call from several host threads.  Returns a cudaError_t.
 int ensure_dyn_smem(const void* kernel, int bytes);
 
 constexpr int kMaxMseBits = 4;
@@ -126,6 +126,10 @@ int launch_quant_mse_tc(const tq_ctx* h, const void* x, int64_t N, int64_t x_str
 int launch_quant_simple(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride,
                         uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
                         int64_t out_stride, void* stream, const int32_t* channels = nullptr);
+// one launch for up to two channel groups of N vectors (d <= 256 each; N < 65536)
+int launch_quant_small(const tq_ctx* const* h, int ngroups, const void* x, int dtype, int64_t N, int64_t x_stride,
+                       const int32_t* channels, uint32_t* const* codes, uint32_t* const* signs, float* const* norms,
+                       float* const* rnorms, int64_t out_stride, void* stream);
 int launch_query_prep_gather(const tq_ctx* h, const void* q, int q_dtype, int64_t nq, int dq,
                              const int32_t* channels, float* qrot, float* qproj, void* stream);
 bool quant_gen_supported(const tq_ctx* h);

@@ -439,6 +439,24 @@ TQ_API int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N, int
                            int64_t out_stride, void* stream);
 
 /*
+ * tq_quant_gather_groups -- tq_quant_gather for every channel group of a few
+ * arriving tokens in one launch (the append of a split cache, [ttakun,
+ * "新旧量化方案深度权衡矩阵"]: each token is compressed as it arrives).
+ *   h          host array [ngroups] of handles (ngroups 1 or 2; d <= 256 each)
+ *   channels   dev in, [sum d_g] int32: group g's channels at offset sum_{g'<g} d_g'
+ *   codes, signs, norms, rnorms   host arrays [ngroups] of dev pointers, each
+ *              as tq_quant_gather for that group (signs / rnorms entries may be
+ *              NULL for TQ_MSE groups)
+ *   N          vectors (0 <= N < 65536), x_stride, out_stride as tq_quant_gather
+ * Pointers need only be 4-byte aligned.
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_quant_gather_groups(const tq_handle* h, int ngroups, const void* x, int dtype, int64_t N,
+                                  int64_t x_stride, const int32_t* channels, uint32_t* const* codes,
+                                  uint32_t* const* signs, float* const* norms, float* const* rnorms,
+                                  int64_t out_stride, void* stream);
+
+/*
  * tq_attn_logits -- attention logits over a TurboQuant_prod key cache whose
  * channels may be split into groups (the pages' outlier channels kept at
  * higher precision, [tq.net, "TurboQuant 最近的进展和外溢影响"]; logits over a

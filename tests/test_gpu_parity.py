@@ -423,6 +423,49 @@ def test_streaming_append_gathers_channel_groups():
         _check_quant(inst, x64, sub)
 
 
+def test_streaming_append_both_groups_in_one_launch():
+    """The same append as above through tq_quant_gather_groups: one launch per
+    arriving token covers both channel groups of all 8 kv-heads; the words
+    equal those of the per-group calls, and both match the oracle."""
+    Hkv, cap, steps = 8, 40, 5
+    scales, hi, lo, ia, ib, channels = _split_instances()
+    keys = [_split_keys(steps, h, scales, 8) for h in range(Hkv)]
+    one = {n: inst.alloc_outputs(Hkv * cap) for inst, n in ((ia, "a"), (ib, "b"))}
+    per = {n: inst.alloc_outputs(Hkv * cap) for inst, n in ((ia, "a"), (ib, "b"))}
+    for t in range(steps):
+        x = to_device(np.stack([keys[h][t] for h in range(Hkv)]), torch.bfloat16)
+        tq.tq_quant_gather_groups([ia.h, ib.h], x, channels, [one[n]["codes"][t:] for n in "ab"],
+                                  [one[n]["norms"][t:] for n in "ab"], signs=[one[n]["signs"][t:] for n in "ab"],
+                                  rnorms=[one[n]["rnorms"][t:] for n in "ab"], out_stride=cap)
+        for inst, n, off in ((ia, "a", 0), (ib, "b", 64)):
+            c = per[n]
+            tq.tq_quant_gather(inst.h, x, channels[off:off + 64], c["codes"][t:], c["norms"][t:],
+                               signs=c["signs"][t:], rnorms=c["rnorms"][t:], out_stride=cap)
+    torch.cuda.synchronize()
+    for inst, n, chans in ((ia, "a", hi), (ib, "b", lo)):
+        for k in one[n]:
+            assert torch.equal(one[n][k], per[n][k]), (n, k)
+        rows = np.array([h * cap + t for h in range(Hkv) for t in range(steps)])
+        x64 = np.stack([keys[h][t][chans] for h in range(Hkv) for t in range(steps)])
+        sub = {k: v[torch.tensor(rows, device=DEV)] for k, v in one[n].items()}
+        _check_quant(inst, x64, sub)
+
+
+def test_bulk_gather_on_the_tensor_cores():
+    """A cache fill through tq_quant_gather (N >= 256 takes the tensor-core
+    quantizer with the channel gather in its producers): 3000 tokens, both groups."""
+    N = 3000
+    scales, hi, lo, ia, ib, channels = _split_instances(seed=4)
+    k64 = _split_keys(N, 0, scales, 4)
+    x = to_device(k64, torch.bfloat16)
+    for inst, chans, off in ((ia, hi, 0), (ib, lo, 64)):
+        out = inst.alloc_outputs(N)
+        tq.tq_quant_gather(inst.h, x, channels[off:off + 64], out["codes"], out["norms"], signs=out["signs"],
+                           rnorms=out["rnorms"])
+        torch.cuda.synchronize()
+        _check_quant(inst, k64[:, chans], out)
+
+
 def _logits_case(B, Hq, Hkv, T, sample, seed=0):
     scales, hi, lo, ia, ib, channels = _split_instances(seed=seed)
     rows = B * Hkv * T
