@@ -460,6 +460,40 @@ class Decode:
         return self.B * self.Hkv * self.T
 
 
+class Prefill:
+    """Prefill over the decode configuration's cache: B = 8, Hq = 32, Hkv = 8,
+    d = 128, T = 131072 (K prod 4b, V mse 4b); a block of nq = 512 new tokens
+    at the end of the context attends causally.  One step = one
+    tq_attn_prefill call (query prep, the tensor-core kernel, the merge)."""
+
+    def __init__(self, tq, torch, dec, nq=512):
+        self.tq, self.torch, self.dec, self.nq = tq, torch, dec, nq
+        g = torch.Generator(device=dec.dev).manual_seed(5000)
+        sq = torch.tensor(synth.lognormal_channel_scales(D, 1.0, 0, 21), dtype=torch.float32, device=dec.dev)
+        self.q = (torch.randn((dec.B, nq, dec.Hq, D), generator=g, device=dec.dev) * sq).to(torch.bfloat16)
+        self.out = torch.empty((dec.B, nq, dec.Hq, D), dtype=torch.float32, device=dec.dev)
+        self.ws = torch.empty(max(1, tq.tq_attn_prefill_workspace(dec.hk, dec.B, nq, dec.Hq, dec.Hkv, dec.T)),
+                              dtype=torch.uint8, device=dec.dev)
+        self.ev = []
+
+    def step(self, record=False):
+        d = self.dec
+        if record:
+            e0, e1 = self.torch.cuda.Event(enable_timing=True), self.torch.cuda.Event(enable_timing=True)
+            e0.record(d.stream)
+        self.tq.tq_attn_prefill(d.hk, d.hv, self.q, d.Hkv, d.T, d.T, d.kcodes, d.ksigns, d.knorms, d.krnorms,
+                                d.vcodes, d.vnorms, d.scale, self.out, self.ws)
+        if record:
+            e1.record(d.stream)
+            self.ev.append((e0, e1))
+
+    def flops(self):
+        # 6 d FLOP per (query row, visible key): the two logit products and the value product
+        d = self.dec
+        vis = sum(d.T - self.nq + i + 1 for i in range(self.nq))
+        return 6.0 * D * d.B * d.Hq * vis
+
+
 class Stream:
     """Config: batch 1, 32 q-heads / 8 kv-heads, d = 128, context 2^20; keys split
     into the 64 largest-scale channels at prod 4 bits and 64 at prod 3 bits
@@ -756,6 +790,22 @@ def run_ours(args):
                             "ms_per_step": dms, "GBps": gbs, "frac_hbm": gbs / hbm,
                             "bytes_per_step": dl.bytes_per_step(),
                             "config": "B=8, Hq=32, Hkv=8, d=128, T=131072, K prod 4b, V mse 4b"}
+        try:
+            pf = Prefill(tq, torch, dl)
+            for _ in range(args.warmup):
+                pf.step()
+            for _ in range(max(1, args.steps // 2)):
+                pf.step(record=True)
+            torch.cuda.synchronize()
+            pms = max_over_ranks(sum(a.elapsed_time(b) for a, b in pf.ev) / len(pf.ev))
+            tfl = pf.flops() / (pms / 1e3) / 1e12
+            result["prefill"] = {"ms_per_step": pms, "tokens_per_s": dl.B * pf.nq * world / (pms / 1e3),
+                                 "TFLOPs": tfl, "frac_tensor": tfl / bf16,
+                                 "config": "decode cache (B=8, Hq=32, Hkv=8, d=128, T=131072), a causal block of "
+                                           f"nq={pf.nq} new tokens; 6 d FLOP per (query row, visible key)"}
+            del pf
+        except Exception as exc:  # a sub-result must not cost the bench line
+            result["prefill"] = {"error": repr(exc)}
 
     if args.workload == "sweep" and not args.no_decode:
         torch.cuda.empty_cache()

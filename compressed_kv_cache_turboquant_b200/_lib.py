@@ -62,6 +62,9 @@ SIGNATURES = {
     "tq_quant_paged": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _i, _p]),
     "tq_attn_decode_paged": (_i, [_p, _p, _p, _i, _i, _i, _i, _i64, _p, _i, _i, _p, _p, _p, _p, _i, _p, _p, _f, _p,
                                   _p, _sz, _p]),
+    "tq_attn_prefill": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f, _p, _p, _sz,
+                             _p]),
+    "tq_attn_prefill_workspace": (_sz, [_p, _i, _i, _i, _i, _i64]),
     "tq_device_status": (_i, [_p, ctypes.POINTER(_i)]),
     "tq_quant_gather": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _i64, _p]),
     "tq_quant_gather_groups": (_i, [ctypes.POINTER(_p), _i, _p, _i, _i64, _i64, _p, ctypes.POINTER(_p),

@@ -22,7 +22,8 @@ __all__ = [
     "tq_ip_scores", "tq_ip_scores_workspace", "tq_attn_decode", "tq_attn_decode_workspace", "tq_version",
     "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
     "tq_attn_decode_partial", "tq_attn_decode_partial_workspace", "tq_attn_merge", "tq_topk_merge",
-    "tq_quant_paged", "tq_attn_decode_paged", "tq_quant_gather_groups",
+    "tq_quant_paged", "tq_attn_decode_paged", "tq_quant_gather_groups", "tq_attn_prefill",
+    "tq_attn_prefill_workspace",
 ]
 
 
@@ -258,6 +259,25 @@ def tq_attn_decode_paged(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: i
         hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, Hq, Hkv, T, _ptr(block_table), block_table.shape[1], page_size,
         _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _rn_code(krnorms), _ptr(vcodes), _ptr(vnorms),
         float(scale), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def tq_attn_prefill_workspace(hk: Handle, B: int, nq: int, Hq: int, Hkv: int, T: int) -> int:
+    return int(lib.tq_attn_prefill_workspace(hk.ptr, B, nq, Hq, Hkv, T))
+
+
+def tq_attn_prefill(hk: Handle, hv: Handle, q: torch.Tensor, Hkv: int, T: int, kv_stride: int, kcodes, ksigns,
+                    knorms, krnorms, vcodes, vnorms, scale: float, out: torch.Tensor, workspace=None,
+                    stream=None) -> None:
+    """Causal attention of a block of nq new tokens, q [B][nq][Hq][d], over a
+    cache of T tokens that ends with them; out [B][nq][Hq][d] float32."""
+    B, nq, Hq, _ = q.shape
+    if workspace is None:
+        workspace = torch.empty(max(1, tq_attn_prefill_workspace(hk, B, nq, Hq, Hkv, T)), dtype=torch.uint8,
+                                device=q.device)
+    check("tq_attn_prefill", lib.tq_attn_prefill(
+        hk.ptr, hv.ptr, _ptr(q), _dtype_code(q), B, nq, Hq, Hkv, T, kv_stride, _ptr(kcodes), _ptr(ksigns),
+        _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms), float(scale), _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
 
 
 def tq_device_status(h: Handle) -> int:

@@ -373,6 +373,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
     const char* ev = getenv("TQ_RUNTIME_TABLE_ADDRESSES");
     if (e == cudaSuccess && !(ev && ev[0] == '1'))
       e = (cudaError_t)probe_dyn_smem_base((uint32_t*)(h->dev.status + 16), &h->dyn_base);
+    const char* fr = getenv("TQ_FUSED_REGISTER_LOADS");
+    h->fused_register_loads = fr && fr[0] == '1';
     const char* st = getenv("TQ_DEBUG_STALL_MS");
     if (st && atof(st) > 0) h->debug_stall_ns = (uint64_t)(atof(st) * 1e6);
     const char* db = getenv("TQ_DEBUG_DYN_BASE");

@@ -581,10 +581,12 @@ __global__ void __launch_bounds__(128) decode_merge_persistent_kernel(const floa
     }
     orot[j] = partial_out ? v : v * invL;
   }
-  if (partial_out) {  // the merged record (acc, m, l) in the rotated frame
+  if (partial_out) {  // the merged record (acc, m, l) in the rotated frame, at true scale:
+    // the kernel's sums carry the fp16 weight scaling kPScale, which cancels in
+    // its own quotient but not against records of other slices
     float* o = out + bq * (D + 2);
-    for (int j = threadIdx.x; j < D; j += blockDim.x) o[j] = orot[j];
-    if (threadIdx.x == 0) o[D] = M, o[D + 1] = ML[1];
+    for (int j = threadIdx.x; j < D; j += blockDim.x) o[j] = orot[j] * (1.f / kPScale);
+    if (threadIdx.x == 0) o[D] = M, o[D + 1] = ML[1] * (1.f / kPScale);
     return;
   }
   __syncthreads();

@@ -16,13 +16,10 @@
 //          128B-swizzled K-major A tiles (double-buffered)
 //   5..12  epilogue, two warps per TMEM lane quarter taking half of the column
 //          chunks each: one thread per vector reads both accumulators from TMEM,
-//          combines and scales by n, and writes its row's 128-byte chunk into
-//          the warp's own shared-memory box (16-byte units XOR-swizzled by row,
-//          so neither the writes nor the reads below meet in a bank); the warp
-//          then reads the box back four rows per instruction and stores it
-//          with 16-byte global stores, each instruction covering four whole
-//          128-byte lines.  No store waits on an earlier one, so the warp moves
-//          straight on to its next chunk.
+//          combines and scales by n; each warp stages its 32 rows x 128 B
+//          column chunk in 128B-swizzled shared memory (two buffers) and
+//          writes it with one TMA tensor store, so global writes are whole
+//          128-byte lines instead of 32 scattered 16-byte pieces per store
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -60,23 +57,11 @@ struct DqArgs {
   const uint8_t* pit_f16;  // 2 pieces x [slab][row i][128 B swizzled] of Pi^T (B[i][j] = Pi[j][i])
   const uint32_t* lut;     // [16]: fp16 hi | fp16 lo' << 16 of c_k
   int out_bf16;
-  void* out;               // [N][D] of fp32 (or bf16 with out_bf16)
   int* status;
 };
 
-// 16 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane = thread)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
-  uint32_t* u = reinterpret_cast<uint32_t*>(r);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
-        "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
-      : "r"(taddr));
-}
-
 template <int D, int BM>
-__global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_constant__ CUtensorMap omap, DqArgs a) {
   using S = DqShape<D>;
   constexpr int W = (D / 32) * BM;
   extern __shared__ uint8_t smem_raw[];
@@ -234,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
     const int part = (warp - 5) >> 2;
     const int r = quarter * 32 + lane;
     uint8_t* buf = o_s + (warp - 5) * S::kStageOut;
-    const int row_bytes = a.out_bf16 ? 2 * D : 4 * D;   // one output row in global memory
+    constexpr int kCols = 32;  // fp32 columns per 128-byte chunk (bf16: 64)
+    int nst = 0;
     int i = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = i & 1;
@@ -250,64 +236,51 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(DqArgs a) {
       const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 2 * D);
       const int nchunks = a.out_bf16 ? D / 64 : D / 32;
       const int c_lo = part * (nchunks / 2), c_hi = (nchunks == 1) ? (part == 0 ? 1 : 0) : c_lo + nchunks / 2;
-      for (int c = c_lo; c < c_hi; ++c) {
-        // the row's 128 bytes in pieces of 16 TMEM columns; row `lane` of the
-        // box: 16-byte unit j at lane * 128 + (j ^ (lane & 7)) * 16
+      for (int c = c_lo; c < c_hi; ++c, ++nst) {
+        // the previous store from this warp's buffer must have read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        uint32_t pk[32];
         if (a.out_bf16) {
 #pragma unroll
-          for (int qt = 0; qt < 4; ++qt) {  // 16 columns -> 32 bytes = units 2 qt, 2 qt + 1
-            float v0[16], v1[16];
-            tmem_ld16(t0 + c * 64 + qt * 16, v0);
-            tmem_ld16(t0 + D + c * 64 + qt * 16, v1);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            float v0[32], v1[32];
+            tmem_ld32(t0 + c * 64 + hlf * 32, v0);
+            tmem_ld32(t0 + D + c * 64 + hlf * 32, v1);
             tmem_wait_ld();
-            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 16; ++e) {
               const float y0 = n * fmaf(v1[2 * e], 4.8828125e-4f, v0[2 * e]);
               const float y1 = n * fmaf(v1[2 * e + 1], 4.8828125e-4f, v0[2 * e + 1]);
               __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-              pk[e] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const int j = 2 * qt + jj;
-              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-                  make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+              pk[16 * hlf + e] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
         } else {
+          float v0[32], v1[32];
+          tmem_ld32(t0 + c * kCols, v0);
+          tmem_ld32(t0 + D + c * kCols, v1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {  // 16 columns -> 64 bytes = units 4 hf .. 4 hf + 3
-            float v0[16], v1[16];
-            tmem_ld16(t0 + c * 32 + hf * 16, v0);
-            tmem_ld16(t0 + D + c * 32 + hf * 16, v1);
-            tmem_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const int j = 4 * hf + jj;
-              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-                  make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-            }
-          }
+          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
         }
-        __syncwarp();
-        // back out four rows per instruction: lane -> row 4 it + lane / 8, unit lane % 8
-        uint8_t* gout = static_cast<uint8_t*>(a.out) + row0 * row_bytes + c * 128;
+        // row `lane` of the 128B-swizzled box: 16-byte unit j lands at j ^ (lane & 7)
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int rr = 4 * it + (lane >> 3), j = lane & 7;
-          const uint4 v = *reinterpret_cast<const uint4*>(buf + rr * 128 + ((j ^ (rr & 7)) * 16));
-          if (row0 + rr < a.N) *reinterpret_cast<uint4*>(gout + (int64_t)rr * row_bytes + j * 16) = v;
-        }
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        fence_async_smem();
         __syncwarp();
+        if (lane == 0 && row0 < a.N) {
+          tma_store_2d(&omap, buf, c * (a.out_bf16 ? 64 : kCols), (int)row0);
+          bulk_commit();
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[s]);
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -322,12 +295,25 @@ template <int D, int BM>
 int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_t N, void* out, int out_bf16,
               cudaStream_t stream) {
   using S = DqShape<D>;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return (int)cudaErrorNotSupported;
+  // output as a [N][D] tensor, boxes of 32 rows x 128 bytes
+  CUtensorMap omap;
+  const int esz = out_bf16 ? 2 : 4;
+  const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)N};
+  const cuuint64_t gstride[1] = {(cuuint64_t)D * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  const cuuint32_t estride[2] = {1, 1};
+  if (enc(&omap, out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, gdim, gstride,
+          box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return (int)cudaErrorInvalidValue;
   auto kern = dequant_tc_kernel<D, BM>;
   if (int e = ensure_dyn_smem((const void*)kern, S::kSmemBytes)) return e;
-  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, out, h->dev.status};
+  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, h->dev.status};
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);
-  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(a);
+  kern<<<grid, kThreads, S::kSmemBytes, stream>>>(omap, a);
   return (int)cudaGetLastError();
 }
 

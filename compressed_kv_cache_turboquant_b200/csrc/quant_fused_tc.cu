@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 
 #include "sm100_common.cuh"
 #include "tq_internal.h"
@@ -579,6 +580,11 @@ bool quant_fused_supported(const tq_ctx* h) { return h->dev.fz_pi != nullptr; }
 int launch_quant_fused(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
                        uint32_t* signs, float* norms, void* rnorms, int64_t out_stride, void* stream,
                        const int32_t* channels, const int64_t* slots, int rn_f16) {
+  // contiguous rows: the TMA-staged kernel; a channel gather stays on this one
+  const int esz = dtype == TQ_BF16 ? 2 : 4;
+  if (!channels && !(reinterpret_cast<uintptr_t>(x) & 15u) && (x_stride * esz) % 16 == 0 && !h->fused_register_loads)
+    return launch_quant_fused2(h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride, stream, slots,
+                               rn_f16);
   cudaStream_t s = (cudaStream_t)stream;
   const bool prod = h->variant == TQ_PROD;
   if (int e = launch_gen_norms(h, x, dtype, N, x_stride, norms, out_stride, stream, channels, slots)) return e;

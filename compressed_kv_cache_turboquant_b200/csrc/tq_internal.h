@@ -95,6 +95,10 @@ struct tq_ctx {
   //                         (TQ_STATUS_LAYOUT)
   uint64_t debug_stall_ns = 0;
   int fz_n16 = 0, fz_k64 = 0;  // fused quantizer tile shape (0: not available)
+  // TQ_FUSED_REGISTER_LOADS=1 at creation: contiguous inputs take the fused
+  // quantizer whose producer threads load x themselves (the one a channel
+  // gather always takes) instead of the TMA-staged one
+  bool fused_register_loads = false;
   bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
@@ -138,6 +142,11 @@ int launch_gen_norms(const tq_ctx* h, const void* x, int dtype, int64_t N, int64
                      int64_t out_stride, void* stream, const int32_t* channels = nullptr,
                      const int64_t* slots = nullptr);
 bool quant_fused_supported(const tq_ctx* h);
+// the fused quantizer with the input staged by TMA and the residual in tensor
+// memory (rows of x start 16-byte aligned; no channel gather)
+int launch_quant_fused2(const tq_ctx* h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
+                        uint32_t* signs, float* norms, void* rnorms, int64_t out_stride, void* stream,
+                        const int64_t* slots, int rn_f16);
 // d <= 256: norms, then one persistent tensor-core kernel for codes (and QJL bits, ||r||).
 // channels: optional gather of each row's d channels; slots: optional output row per
 // vector (else i * out_stride); rn_f16: rnorms is __half storage
@@ -187,6 +196,14 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
                       const float* vnorms, float scale, float* partials, float* out, void* stream,
                       int partial_out = 0, PagedCache pg = PagedCache());
+// prefill (multi-query) attention on the tensor cores
+bool prefill_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride);
+int prefill_splits(int B, int nq, int Hq, int Hkv, int64_t T, int sm_count);
+size_t prefill_partials_bytes(int B, int nq, int Hq, int Hkv, int64_t T, int sm_count);
+int launch_prefill(const tq_ctx* hk, const tq_ctx* hv, const float* qrot, const float* qproj, int B, int nq, int Hq,
+                   int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                   const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms, float scale,
+                   float* partials, float* out, void* stream);
 // decode attention through whichever kernel fits; workspace layout owned here.
 // partial_out: write the (acc[d] in the rotated value frame, m, l) record of
 // every (batch, q-head) to out [B*Hq][d + 2] instead of the normalised output

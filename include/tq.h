@@ -146,6 +146,10 @@ TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
  *   TQ_DEBUG_DYN_BASE=a  record `a` as the measured shared-window address, so
  *                        the decode and logits kernels built for the usual
  *                        address report TQ_STATUS_LAYOUT and write nothing
+ * and one that selects between two implementations of the same arithmetic:
+ *   TQ_FUSED_REGISTER_LOADS=1  quantization at d <= 256 takes the kernel whose
+ *                        producer threads load x themselves (the one a channel
+ *                        gather always takes) instead of the TMA-staged one
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
  */
 TQ_API int tq_create(tq_handle* h, int d, int b, int variant, const double* Pi, const double* S,
@@ -319,6 +323,31 @@ TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int 
                                  const uint32_t* ksigns, const float* knorms, const float* krnorms,
                                  const uint32_t* vcodes, const float* vnorms, float scale, float* out,
                                  void* stream);
+
+/*
+ * tq_attn_prefill -- attention of a block of nq new tokens (a prompt chunk)
+ * over a TurboQuant K/V cache that already holds them ([tq.net, "实现步骤草图",
+ * 集成到 attention]; [tmdm, "实测数据"]: logits over a 4-bit cache).  Token i of
+ * the block sits at position T - nq + i and attends keys t <= T - nq + i
+ * (causal); for batch b, token i, query head j (kv-head h = j / (Hq/Hkv)):
+ *   out[b][i][j] = sum_{t <= T-nq+i} softmax(scale * est(q_bij, k_t)) n_t Pi_V^T c_V[idx_t]
+ * The products run on the tensor cores (decoded keys and values as fp16
+ * operands, fp32 accumulation); the value sum stays in the rotated frame and
+ * Pi_V^T is applied once per output row.
+ *   q         dev in, [B][nq][Hq][d] of q_dtype (TQ_F32 or TQ_BF16)
+ *   T         context length including the block (nq <= T)
+ *   kv_stride, cache arrays   as tq_attn_decode
+ *   out       dev out, [B][nq][Hq][d] float32
+ *   workspace dev scratch of at least tq_attn_prefill_workspace(...) bytes
+ * Supported: d = 128, keys TQ_PROD b = 4, values TQ_MSE b = 4, Hq / Hkv a
+ * divisor of 128, kv_stride % 4 == 0 (TQ_EUNSUPPORTED otherwise).
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
+ */
+TQ_API int tq_attn_prefill(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int nq, int Hq, int Hkv,
+                           int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
+                           const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                           float scale, float* out, void* workspace, size_t ws_bytes, void* stream);
+TQ_API size_t tq_attn_prefill_workspace(tq_handle hk, int B, int nq, int Hq, int Hkv, int64_t T);
 
 /* ---------------------------------------------------------------- a cache split across devices */
 

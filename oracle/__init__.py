@@ -26,14 +26,14 @@ from .codebook import (coord_pdf, coord_cdf, bin_first_moment, lloyd_max, lloyd_
 from .turboquant import (haar_rotation, quantize_indices, nearest_centroid_bruteforce,
                          quant_mse, dequant_mse, quant_prod, prod_estimate, mse_estimate,
                          pack_codes, pack_codes_vec, unpack_codes, pack_signs, unpack_signs, code_words,
-                         attention_decode, attention_partial, merge_attention_partials, topk, channel_split,
+                         attention_decode, attention_prefill, attention_partial, merge_attention_partials, topk, channel_split,
                          near_threshold_mask)
 
 __all__ = [
     "coord_pdf", "coord_cdf", "bin_first_moment", "lloyd_max", "lloyd_max_quadrature", "distortion",
     "b1_centroid", "haar_rotation", "quantize_indices", "nearest_centroid_bruteforce", "quant_mse",
     "dequant_mse", "quant_prod", "prod_estimate", "mse_estimate", "pack_codes", "pack_codes_vec", "unpack_codes",
-    "pack_signs", "unpack_signs", "code_words", "attention_decode", "attention_partial",
+    "pack_signs", "unpack_signs", "code_words", "attention_decode", "attention_prefill", "attention_partial",
     "merge_attention_partials", "topk", "channel_split",
     "near_threshold_mask",
 ]

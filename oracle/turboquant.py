@@ -309,6 +309,32 @@ def attention_decode(q: np.ndarray, k_est_fn, v_hat: np.ndarray, Hkv: int, scale
     return out, all_logits
 
 
+def attention_prefill(q: np.ndarray, k_est_fn, v_hat, Hkv: int, T: int, scale: float | None = None):
+    """Attention of a block of nq new tokens (a prompt chunk) over a TurboQuant
+    K/V cache that already holds them: query token i sits at position
+    T - nq + i and attends the keys t <= T - nq + i (causal).  Same readings as
+    ``attention_decode`` ([tq.net, "实现步骤草图", 集成到 attention]).
+    q: [B, nq, Hq, d]; k_est_fn(b, h, q_rows [r, d]) -> [r, T]; v_hat(b, h) -> [T, d].
+    Returns out [B, nq, Hq, d].  Pinned by scipy's softmax over each query's
+    visible keys and, for nq = 1, by ``attention_decode``."""
+    q = np.asarray(q, dtype=np.float64)
+    B, nq, Hq, d = q.shape
+    g = Hq // Hkv
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = np.zeros((B, nq, Hq, d))
+    for b in range(B):
+        for h in range(Hkv):
+            rows = q[b, :, h * g:(h + 1) * g].reshape(nq * g, d)      # row = (token i, head j)
+            logits = np.atleast_2d(k_est_fn(b, h, rows)) * scale     # [nq * g, T]
+            pos = T - nq + np.repeat(np.arange(nq), g)               # position of each row's token
+            logits = np.where(np.arange(T)[None, :] <= pos[:, None], logits, -np.inf)
+            mx = np.max(logits, axis=1, keepdims=True)
+            p = np.exp(logits - mx)
+            p /= np.sum(p, axis=1, keepdims=True)
+            out[b, :, h * g:(h + 1) * g] = (p @ v_hat(b, h)).reshape(nq, g, d)
+    return out
+
+
 def attention_partial(q: np.ndarray, k_est_fn, v_hat, Hkv: int, scale: float | None = None):
     """The softmax state of one decode step over a slice of the context, to be
     combined with the states of the other slices (the context split across

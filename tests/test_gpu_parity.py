@@ -131,13 +131,18 @@ def test_zero_vectors_every_path(d, dtype, variant, b):
     assert np.all(out["norms"].cpu().numpy()[zero] == 0)
 
 
-@pytest.mark.parametrize("d", [8, 240, 256])
+@pytest.mark.parametrize("d", [8, 200, 240, 256])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_quantize_tile_shape_edges(d, dtype):
+@pytest.mark.parametrize("register_loads", [False, True])
+def test_quantize_tile_shape_edges(d, dtype, register_loads, monkeypatch):
     """Dimensions at the edges of the fused tile shapes: one 16-wide K step (d = 8),
-    a partial last 32-group (d = 240) and the widest tile, whose operand ring
-    drops to two stages (d = 256); 700 rows = five tiles and a ragged tail."""
+    a half-filled last 32-group (d = 200, 240) and the widest tile, whose rings
+    are shallower (d = 256); 700 rows = five tiles and a ragged tail.  Both fused
+    kernels: the TMA-staged one and (register_loads) the one whose producer
+    threads load x themselves."""
     N = 700
+    if register_loads:
+        monkeypatch.setenv("TQ_FUSED_REGISTER_LOADS", "1")
     for variant, b in [(tq.TQ_MSE, 2), (tq.TQ_PROD, 4), (tq.TQ_PROD, 3)]:
         inst = Instance(d, b, variant, seed=d + 1)
         x64 = synth.scaled_gaussian_rows(N, d, 1.0, seed=d)

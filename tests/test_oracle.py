@@ -419,6 +419,33 @@ def test_attention_uniform_and_dominant_limits():
     assert np.allclose(out[0, 0], p @ v[0], atol=1e-13)
 
 
+def test_prefill_is_causal_softmax_over_each_tokens_visible_keys():
+    # every new token's output is scipy's softmax over the keys at or before its
+    # position; the last token sees everything (= the decode step), the first
+    # one T - nq + 1 keys; a key after a token's position never contributes
+    B, nq, Hq, Hkv, T, d = 2, 5, 4, 2, 23, 6
+    r = synth.rng(5, 1)
+    k = r.standard_normal((B, Hkv, T, d))
+    v = r.standard_normal((B, Hkv, T, d))
+    q = r.standard_normal((B, nq, Hq, d)) * 2
+    est = lambda b, h, rows: rows @ k[b, h].T
+    out = tq.attention_prefill(q, est, lambda b, h: v[b, h], Hkv, T)
+    for b in range(B):
+        for i in range(nq):
+            vis = T - nq + i + 1
+            for j in range(Hq):
+                p = special.softmax(q[b, i, j] @ k[b, j // 2, :vis].T / math.sqrt(d))
+                assert np.allclose(out[b, i, j], p @ v[b, j // 2, :vis], atol=1e-13)
+    dec, _ = tq.attention_decode(q[:, -1], est, lambda b, h: v[b, h], Hkv)
+    assert np.allclose(out[:, -1], dec, atol=1e-13)
+    # changing a key after the first token's position leaves that token's output alone
+    k2 = k.copy()
+    k2[:, :, T - nq + 1:] += 5.0
+    out2 = tq.attention_prefill(q, lambda b, h, rows: rows @ k2[b, h].T, lambda b, h: v[b, h], Hkv, T)
+    assert np.allclose(out2[:, 0], out[:, 0], atol=1e-13)
+    assert not np.allclose(out2[:, -1], out[:, -1])
+
+
 def test_context_split_softmax_states_merge_to_the_full_softmax():
     # Any split of the context into slices (an empty one included) merges back
     # to scipy's softmax over the whole context; a single slice merges to its
