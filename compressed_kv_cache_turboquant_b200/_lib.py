@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA, TQ_ENOMEM, TQ_EWORKSPACE = range(7)
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
-TQ_MSE, TQ_PROD = 0, 1
+TQ_MSE, TQ_PROD, TQ_POLAR = 0, 1, 2
 TQ_MAX_DIM = 4096
 TQ_MAX_TOPK = 64
 TQ_STATUS_TIMEOUT, TQ_STATUS_LAYOUT = 1, 2
@@ -65,6 +65,10 @@ SIGNATURES = {
     "tq_attn_prefill": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i64, _i64, _p, _p, _p, _p, _p, _p, _f, _p, _p, _sz,
                              _p]),
     "tq_attn_prefill_workspace": (_sz, [_p, _i, _i, _i, _i, _i64]),
+    "tq_polar_codebook": (_i, [_i, _i, _dp, _dp]),
+    "tq_create_polar": (_i, [ctypes.POINTER(_p), _i, _i, _i, _dp]),
+    "tq_quant_polar": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _i64, _p]),
+    "tq_dequant_polar": (_i, [_p, _p, _p, _i64, _p, _i, _p]),
     "tq_device_status": (_i, [_p, ctypes.POINTER(_i)]),
     "tq_quant_gather": (_i, [_p, _p, _i, _i64, _i64, _p, _p, _p, _p, _p, _i64, _p]),
     "tq_quant_gather_groups": (_i, [ctypes.POINTER(_p), _i, _p, _i, _i64, _i64, _p, ctypes.POINTER(_p),

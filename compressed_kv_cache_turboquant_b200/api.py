@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (TQ_BF16, TQ_F16, TQ_F32, TQ_MAX_TOPK, TQ_MSE, TQ_PROD, TQ_STATUS_LAYOUT, TQ_STATUS_TIMEOUT, TQError,
+from ._lib import (TQ_BF16, TQ_F16, TQ_F32, TQ_MAX_TOPK, TQ_POLAR, TQ_MSE, TQ_PROD, TQ_STATUS_LAYOUT, TQ_STATUS_TIMEOUT, TQError,
                    check, lib)
 
 __all__ = [
@@ -23,7 +23,8 @@ __all__ = [
     "tq_attn_decode_static", "tq_quant_gather", "tq_attn_logits", "tq_attn_logits_workspace", "tq_device_status",
     "tq_attn_decode_partial", "tq_attn_decode_partial_workspace", "tq_attn_merge", "tq_topk_merge",
     "tq_quant_paged", "tq_attn_decode_paged", "tq_quant_gather_groups", "tq_attn_prefill",
-    "tq_attn_prefill_workspace",
+    "tq_attn_prefill_workspace", "TQ_POLAR", "tq_polar_codebook", "tq_create_polar", "tq_quant_polar",
+    "tq_dequant_polar",
 ]
 
 
@@ -87,13 +88,15 @@ def tq_make_rotation(G: np.ndarray) -> np.ndarray:
 class Handle:
     """Owns a tq_handle (device constants); destroyed with the object."""
 
-    def __init__(self, ptr: int, d: int, b: int, variant: int):
+    def __init__(self, ptr: int, d: int, b: int, variant: int, bh: int = 0):
         self.ptr = ptr
-        self.d, self.b, self.variant = d, b, variant
-        self.bm = b if variant == TQ_MSE else b - 1
+        self.d, self.b, self.variant, self.bh = d, b, variant, bh
+        self.bm = b if variant in (TQ_MSE, TQ_POLAR) else b - 1
 
     @property
     def words(self) -> int:
+        if self.variant == TQ_POLAR:
+            return code_words(self.b, self.d // 2) + code_words(self.bh, self.d // 2 - 1)
         return code_words(self.bm, self.d)
 
     def close(self):
@@ -117,6 +120,32 @@ def tq_create(d: int, b: int, variant: int, Pi: np.ndarray, S: np.ndarray | None
     check("tq_create", lib.tq_create(ctypes.byref(h), d, b, variant, _dptr(Pi),
                                      None if Sa is None else _dptr(Sa), None if ca is None else _dptr(ca)))
     return Handle(h.value, d, b, variant)
+
+
+def tq_polar_codebook(b: int, level: int) -> tuple[np.ndarray, np.ndarray]:
+    c = np.zeros(2 ** b)
+    t = np.zeros(2 ** b - 1)
+    check("tq_polar_codebook", lib.tq_polar_codebook(b, level, _dptr(c), _dptr(t)))
+    return c, t
+
+
+def tq_create_polar(d: int, b1: int, bh: int, Pi: np.ndarray) -> Handle:
+    """A PolarQuant instance: b1 bits for level-1 angles, bh for the others."""
+    Pi = np.ascontiguousarray(Pi, dtype=np.float64)
+    h = ctypes.c_void_p()
+    check("tq_create_polar", lib.tq_create_polar(ctypes.byref(h), d, b1, bh, _dptr(Pi)))
+    return Handle(h.value, d, b1, TQ_POLAR, bh)
+
+
+def tq_quant_polar(h: Handle, x: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor, out_stride: int = 1,
+                   stream=None) -> None:
+    check("tq_quant_polar", lib.tq_quant_polar(h.ptr, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1], _ptr(codes),
+                                               _ptr(norms), out_stride, _stream(stream)))
+
+
+def tq_dequant_polar(h: Handle, codes: torch.Tensor, norms: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    check("tq_dequant_polar", lib.tq_dequant_polar(h.ptr, _ptr(codes), _ptr(norms), codes.shape[0], _ptr(out),
+                                                   _dtype_code(out), _stream(stream)))
 
 
 def tq_quant_mse(h: Handle, x: torch.Tensor, codes: torch.Tensor, norms: torch.Tensor,

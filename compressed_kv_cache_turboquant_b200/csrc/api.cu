@@ -410,9 +410,50 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   return clear_error();
 }
 
+extern "C" int tq_create_polar(tq_handle* out, int d, int b1, int bh, const double* Pi) {
+  if (!out || !Pi) return set_error(TQ_EINVAL, "tq_create_polar: NULL handle or rotation");
+  *out = nullptr;
+  if (d != 64 && d != 128) return set_error(TQ_EUNSUPPORTED, "tq_create_polar: d = %d (need 64 or 128)", d);
+  if ((b1 != 2 && b1 != 4) || (bh != 1 && bh != 2))
+    return set_error(TQ_EUNSUPPORTED, "tq_create_polar: b1 = %d, bh = %d (need b1 in {2, 4}, bh in {1, 2})", b1, bh);
+  // the rotation operands of an mse instance, then the polar constants
+  int rc = tq_create(out, d, b1, TQ_MSE, Pi, nullptr, nullptr);
+  if (rc) return rc;
+  tq_ctx* h = *out;
+  h->variant = TQ_POLAR;
+  h->polar_b1 = b1;
+  h->polar_bh = bh;
+  int L = 0;
+  while ((1 << L) < d) ++L;
+  std::vector<float> cs(2 * 8 * 16, 0.f);
+  double c[16], t[15];
+  rc = tq_polar_codebook(b1, 1, c, nullptr);
+  for (int k = 0; rc == TQ_OK && k < (1 << b1); ++k) {
+    cs[0 * 128 + 1 * 16 + k] = (float)std::cos(c[k]);
+    cs[1 * 128 + 1 * 16 + k] = (float)std::sin(c[k]);
+  }
+  for (int l = 2; rc == TQ_OK && l <= L; ++l) {
+    rc = tq_polar_codebook(bh, l, c, t);
+    for (int k = 0; rc == TQ_OK && k < (1 << bh); ++k) {
+      cs[0 * 128 + l * 16 + k] = (float)std::cos(c[k]);
+      cs[1 * 128 + l * 16 + k] = (float)std::sin(c[k]);
+      if (k + 1 < (1 << bh)) h->polar_tan2[l][k] = (float)(std::tan(t[k]) * std::tan(t[k]));
+    }
+  }
+  int e = rc == TQ_OK ? (int)cudaMalloc(&h->polar_cs, cs.size() * 4) : 0;
+  if (rc == TQ_OK && e == cudaSuccess) e = cudaMemcpy(h->polar_cs, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice);
+  if (rc != TQ_OK || e != cudaSuccess) {
+    tq_destroy(h);
+    *out = nullptr;
+    return rc != TQ_OK ? rc : cuda_error("tq_create_polar", e);
+  }
+  return clear_error();
+}
+
 extern "C" int tq_destroy(tq_handle h) {
   if (!h) return clear_error();
   int e = cudaDeviceSynchronize();
+  if (h->polar_cs) cudaFree(h->polar_cs);
   int e2 = cudaFree(h->block);
   delete h;
   if (e != cudaSuccess) return cuda_error("tq_destroy", e);
@@ -519,6 +560,7 @@ extern "C" size_t tq_quant_prod_workspace(tq_handle h, int64_t N) {
 extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* norms, int64_t N,
                               void* out, int out_dtype, void* stream) {
   if (!h) return set_error(TQ_EINVAL, "tq_dequant_mse: NULL handle");
+  if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_dequant_mse: a TQ_POLAR handle (use tq_dequant_polar)");
   if (N < 0) return set_error(TQ_EINVAL, "tq_dequant_mse: N < 0");
   if (out_dtype != TQ_F32 && out_dtype != TQ_BF16)
     return set_error(TQ_EUNSUPPORTED, "tq_dequant_mse: out_dtype %d", out_dtype);
@@ -547,6 +589,7 @@ extern "C" int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint3
                             int64_t N, float* scores, int topk, int32_t* top_idx, float* top_val,
                             void* workspace, size_t ws_bytes, void* stream) {
   if (!h) return set_error(TQ_EINVAL, "tq_ip_scores: NULL handle");
+  if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_ip_scores: a TQ_POLAR handle");
   if (nq < 0 || N < 0) return set_error(TQ_EINVAL, "tq_ip_scores: negative size");
   if (topk < 0 || topk > TQ_MAX_TOPK || (topk > 0 && topk > N && N > 0))
     return set_error(TQ_EINVAL, "tq_ip_scores: topk %d (need 0..min(N, %d))", topk, TQ_MAX_TOPK);
@@ -657,10 +700,38 @@ extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_d
   return e ? cuda_error("tq_attn_decode", e) : clear_error();
 }
 
+extern "C" int tq_quant_polar(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
+                              float* norms, int64_t out_stride, void* stream) {
+  int rc = check_quant_args("tq_quant_polar", h, TQ_POLAR, x, dtype, N, x_stride, codes, norms, out_stride);
+  if (rc) return rc;
+  if (N == 0) return clear_error();
+  if (reinterpret_cast<uintptr_t>(x) & 15u) return set_error(TQ_EALIGN, "tq_quant_polar: x is not 16-byte aligned");
+  const int e = launch_quant_fused2(h, x, dtype, N, x_stride, codes, nullptr, norms, nullptr, out_stride, stream,
+                                    nullptr, 0);
+  return e ? cuda_error("tq_quant_polar", e) : clear_error();
+}
+
+extern "C" int tq_dequant_polar(tq_handle h, const uint32_t* codes, const float* norms, int64_t N, void* out,
+                                int out_dtype, void* stream) {
+  if (!h) return set_error(TQ_EINVAL, "tq_dequant_polar: NULL handle");
+  if (h->variant != TQ_POLAR) return set_error(TQ_EINVAL, "tq_dequant_polar: need a TQ_POLAR handle");
+  if (N < 0) return set_error(TQ_EINVAL, "tq_dequant_polar: N < 0");
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16)
+    return set_error(TQ_EUNSUPPORTED, "tq_dequant_polar: out_dtype %d", out_dtype);
+  if (N > 0 && (!codes || !norms || !out)) return set_error(TQ_EINVAL, "tq_dequant_polar: NULL pointer");
+  TQ_CHECK_ALIGN(codes, "codes");
+  TQ_CHECK_ALIGN(norms, "norms");
+  TQ_CHECK_ALIGN(out, "out");
+  if (N == 0) return clear_error();
+  const int e = launch_dequant_tc(h, codes, norms, N, out, out_dtype, stream);
+  return e ? cuda_error("tq_dequant_polar", e) : clear_error();
+}
+
 extern "C" int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                                const int32_t* channels, uint32_t* codes, uint32_t* signs, float* norms,
                                float* rnorms, int64_t out_stride, void* stream) {
   if (!h) return set_error(TQ_EINVAL, "tq_quant_gather: NULL handle");
+  if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_quant_gather: a TQ_POLAR handle");
   if (N < 0) return set_error(TQ_EINVAL, "tq_quant_gather: N < 0");
   if (dtype != TQ_F32 && dtype != TQ_BF16) return set_error(TQ_EUNSUPPORTED, "tq_quant_gather: dtype %d", dtype);
   if (x_stride < 1 || out_stride < 1) return set_error(TQ_EINVAL, "tq_quant_gather: stride < 1");
@@ -702,6 +773,7 @@ extern "C" int tq_quant_gather_groups(const tq_handle* h, int ngroups, const voi
   if (!codes || !norms || (N > 0 && (!x || !channels))) return set_error(TQ_EINVAL, "%s: NULL pointer", fn);
   for (int g = 0; g < ngroups; ++g) {
     if (!h[g]) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
+    if (h[g]->variant == TQ_POLAR) return set_error(TQ_EINVAL, "%s: a TQ_POLAR handle", fn);
     if (h[g]->d > 256) return set_error(TQ_EUNSUPPORTED, "%s: d = %d (need <= 256)", fn, h[g]->d);
     const bool prod = h[g]->variant == TQ_PROD;
     if (!codes[g] || !norms[g] || (prod && (!signs || !rnorms || !signs[g] || !rnorms[g])))

@@ -44,7 +44,7 @@ struct DqShape {
   static constexpr int kBBytes = kSlabs * kSlabBytesB;  // one piece of Pi (as B, K-major)
   static constexpr int kStages = 2;
   static constexpr int kTmemCols = (4 * D <= 256) ? 256 : 512;  // 2 buffers x 2 accumulators
-  static constexpr int kMiscBytes = 1024;
+  static constexpr int kMiscBytes = 2048;
   static constexpr int kStageOut = 32 * 128;  // one warp's output chunk: 32 rows x 128 B
   static constexpr int kOutBytes = 8 * kStageOut;  // one staging box per epilogue warp
   static constexpr int kSmemBytes = 2 * kBBytes + kStages * 2 * kABytes + kOutBytes + kMiscBytes + 1024;
@@ -58,12 +58,24 @@ struct DqArgs {
   const uint32_t* lut;     // [16]: fp16 hi | fp16 lo' << 16 of c_k
   int out_bf16;
   int* status;
+  // PolarQuant codes (BM = 0): words per row, bits of level 1 / levels >= 2,
+  // first entry of each level among the codes of levels >= 2, and the cos /
+  // sin of every level's centroids ([2][8 levels][16])
+  int polar_w, b1, bh, w1;
+  int base[9];
+  const float* polar_cs;
 };
+
+// the polar code of entry e (level 1) or of entry e of the levels >= 2
+__device__ __forceinline__ uint32_t polar_code(const uint32_t* w, int word0, int e, int bits) {
+  const int pos = e * bits;
+  return (w[word0 + (pos >> 5)] >> (pos & 31)) & ((1u << bits) - 1u);
+}
 
 template <int D, int BM>
 __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_constant__ CUtensorMap omap, DqArgs a) {
   using S = DqShape<D>;
-  constexpr int W = (D / 32) * BM;
+  constexpr int W = BM ? (D / 32) * BM : 12;  // BM = 0: PolarQuant codes, at most 12 words
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* b_s = smem;                      // [2 pieces][kBBytes]
@@ -78,6 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
   uint64_t* done_bar = bars + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
   uint32_t* lut_s = tmem_slot + 4;      // [16]
+  float* pcs = reinterpret_cast<float*>(lut_s + 16);  // [2][8][16] (PolarQuant)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = (a.N + kTileM - 1) / kTileM;
@@ -94,6 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
     fence_mbar_init();
   }
   if (threadIdx.x < 16) lut_s[threadIdx.x] = a.lut[threadIdx.x];
+  if (BM == 0)
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) pcs[e] = a.polar_cs[e];
   if (warp == 0) tmem_alloc(tmem_slot, S::kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -142,7 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
     const int r = threadIdx.x - 32;
     auto load_codes = [&](int64_t tile, uint32_t (&w)[W]) {
       const int64_t vec = tile * kTileM + r;
-      if (tile < ntiles && vec < a.N) {
+      if (BM == 0) {
+#pragma unroll
+        for (int q = 0; q < W; ++q) w[q] = (tile < ntiles && vec < a.N && q < a.polar_w) ? a.codes[vec * a.polar_w + q] : 0u;
+      } else if (tile < ntiles && vec < a.N) {
         if constexpr (W % 4 == 0) {
           const uint4* src = reinterpret_cast<const uint4*>(a.codes + vec * W);
 #pragma unroll
@@ -175,6 +193,69 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       }
       uint8_t* hi_tile = a_s + s * 2 * S::kABytes;
       uint8_t* lo_tile = hi_tile + S::kABytes;
+      if constexpr (BM == 0) {
+        // the unit angle tree run back down: radii of the top levels, then one
+        // 32-coordinate group at a time
+        constexpr int G = D / 32;
+        const float* cosl = pcs;
+        const float* sinl = pcs + 128;
+        float rg[G];
+        if (D == 128) {
+          const uint32_t c7 = polar_code(w, a.w1, a.base[7], a.bh);
+          const float r6[2] = {cosl[7 * 16 + c7], sinl[7 * 16 + c7]};
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint32_t c6 = polar_code(w, a.w1, a.base[6] + i, a.bh);
+            rg[2 * i] = r6[i] * cosl[6 * 16 + c6];
+            rg[2 * i + 1] = r6[i] * sinl[6 * 16 + c6];
+          }
+        } else {
+          const uint32_t c6 = polar_code(w, a.w1, a.base[6], a.bh);
+          rg[0] = cosl[6 * 16 + c6];
+          rg[1] = sinl[6 * 16 + c6];
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float rr[16];
+          rr[0] = rg[g];
+          // levels 5 .. 2 inside the group: 1, 2, 4, 8 angles
+#pragma unroll
+          for (int lev = 5, cnt = 1; lev >= 2; --lev, cnt <<= 1) {
+#pragma unroll
+            for (int i = cnt - 1; i >= 0; --i) {
+              const uint32_t c = polar_code(w, a.w1, a.base[lev] + cnt * g + i, a.bh);
+              const float r = rr[i];
+              rr[2 * i] = r * cosl[lev * 16 + c];
+              rr[2 * i + 1] = r * sinl[lev * 16 + c];
+            }
+          }
+          float y[32];
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const uint32_t c = polar_code(w, 0, 16 * g + p, a.b1);
+            y[2 * p] = rr[p] * cosl[16 + c];
+            y[2 * p + 1] = rr[p] * sinl[16 + c];
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int kglob = 32 * g + 8 * c4;
+            const int slab = kglob / 64, chunk = (kglob % 64) / 8;
+            uint32_t hv[4], lv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float v0 = y[8 * c4 + 2 * e], v1 = y[8 * c4 + 2 * e + 1];
+              const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+              const __half l0 = __float2half_rn((v0 - __half2float(h0)) * 2048.f);
+              const __half l1 = __float2half_rn((v1 - __half2float(h1)) * 2048.f);
+              hv[e] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+              lv[e] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+            }
+            const int off = slab * S::kSlabBytesA + r * 128 + ((chunk ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+          }
+        }
+      } else {
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {
         uint32_t idx[32];
@@ -208,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
           *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
           *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
+      }
       }
       // generic-proxy writes must be visible to the tensor core's async proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -311,6 +393,15 @@ int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_
   auto kern = dequant_tc_kernel<D, BM>;
   if (int e = ensure_dyn_smem((const void*)kern, S::kSmemBytes)) return e;
   DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, h->dev.status};
+  if (BM == 0) {
+    a.b1 = h->polar_b1;
+    a.bh = h->polar_bh;
+    a.polar_w = TQ_POLAR_WORDS(a.b1, a.bh, D);
+    a.w1 = TQ_CODE_WORDS(a.b1, D / 2);
+    a.base[2] = 0;
+    for (int l = 2; l < 8; ++l) a.base[l + 1] = a.base[l] + (D >> l);
+    a.polar_cs = h->polar_cs;
+  }
   const int64_t ntiles = (N + kTileM - 1) / kTileM;
   const int grid = (int)(ntiles < h->sm_count ? ntiles : h->sm_count);
   kern<<<grid, kThreads, S::kSmemBytes, stream>>>(omap, a);
@@ -327,6 +418,8 @@ int launch_dequant_tc(const tq_ctx* h, const uint32_t* codes, const float* norms
                       int out_dtype, void* stream) {
   cudaStream_t s = (cudaStream_t)stream;
   const int bf = out_dtype == TQ_BF16;
+  if (h->variant == TQ_POLAR)
+    return h->d == 128 ? launch_dq<128, 0>(h, codes, norms, N, out, bf, s) : launch_dq<64, 0>(h, codes, norms, N, out, bf, s);
   if (h->d == 128) {
     switch (h->bm) {
       case 1: return launch_dq<128, 1>(h, codes, norms, N, out, bf, s);

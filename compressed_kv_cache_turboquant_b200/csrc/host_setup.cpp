@@ -238,3 +238,72 @@ extern "C" int tq_make_rotation(int d, const double* G, double* Pi) {
   }
   return clear_error();
 }
+
+namespace tqi {
+
+// Law of a level-l angle of the polar tree of a uniform point on the sphere
+// (l >= 2): sin^2(theta) ~ Beta(m/2, m/2) with m = 2^(l-1) coordinates on each
+// side of the pair, i.e. f(theta) proportional to (sin theta cos theta)^(m-1)
+// on [0, pi/2].  Cell mass and first moment by composite Gauss-Legendre in
+// theta (the normalising constant cancels in the Lloyd-Max centroids).
+struct AngleLaw {
+  int m;
+  const GaussLegendre* gl;
+  void integrals(double a, double b, double* mass, double* mom) const {
+    *mass = 0.0;
+    *mom = 0.0;
+    if (b <= a) return;
+    const int pieces = std::max(1, (int)std::ceil((b - a) / 0.01));
+    const double h = (b - a) / pieces;
+    for (int p = 0; p < pieces; ++p) {
+      const double mid = a + (p + 0.5) * h;
+      for (size_t i = 0; i < gl->x.size(); ++i) {
+        const double th = mid + 0.5 * h * gl->x[i];
+        const double f = std::pow(0.5 * std::sin(2.0 * th), m - 1);
+        *mass += 0.5 * h * gl->w[i] * f;
+        *mom += 0.5 * h * gl->w[i] * f * th;
+      }
+    }
+  }
+};
+
+}  // namespace tqi
+
+extern "C" int tq_polar_codebook(int b, int level, double* centroids, double* thresholds) {
+  if (!centroids) return set_error(TQ_EINVAL, "tq_polar_codebook: NULL centroids");
+  if (b < 1 || b > 8 || level < 1 || level > 12)
+    return set_error(TQ_EUNSUPPORTED, "tq_polar_codebook: b = %d, level = %d", b, level);
+  const int K = 1 << b;
+  std::vector<double> c(K);
+  if (level == 1) {
+    // the uniform law on the circle: cells [k, k+1) 2 pi / K, centroids in the middle
+    for (int k = 0; k < K; ++k) c[k] = (k + 0.5) * 2.0 * M_PI / K;
+  } else {
+    static const GaussLegendre gl(16);
+    const AngleLaw law{1 << (level - 1), &gl};
+    const double sd = 0.5 / std::sqrt((double)law.m);
+    for (int k = 0; k < K; ++k) {
+      const double q = K > 1 ? -2.0 + 4.0 * k / (K - 1) : 0.0;
+      c[k] = std::min(M_PI / 2 - 1e-6, std::max(1e-6, M_PI / 4 + sd * q));
+    }
+    for (int it = 0; it < 2000; ++it) {
+      double change = 0.0;
+      std::vector<double> next(K);
+      for (int k = 0; k < K; ++k) {
+        const double lo = k == 0 ? 0.0 : 0.5 * (c[k - 1] + c[k]);
+        const double hi = k == K - 1 ? M_PI / 2 : 0.5 * (c[k] + c[k + 1]);
+        double mass, mom;
+        law.integrals(lo, hi, &mass, &mom);
+        next[k] = mass > 0.0 ? mom / mass : 0.5 * (lo + hi);
+        change = std::max(change, std::fabs(next[k] - c[k]));
+      }
+      c = next;
+      if (change < 1e-15) break;
+    }
+  }
+  for (int k = 0; k < K; ++k) centroids[k] = c[k];
+  if (thresholds)
+    for (int k = 0; k + 1 < K; ++k)
+      thresholds[k] = level == 1 ? (k + 1) * 2.0 * M_PI / K : 0.5 * (c[k] + c[k + 1]);
+  return clear_error();
+}

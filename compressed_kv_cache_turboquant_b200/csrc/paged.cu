@@ -20,6 +20,7 @@ extern "C" int tq_quant_paged(tq_handle h, const void* x, int dtype, int64_t N, 
                               float* norms, void* rnorms, int rn_dtype, void* stream) {
   const char* fn = "tq_quant_paged";
   if (!h) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
+  if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "%s: a TQ_POLAR handle", fn);
   if (N < 0) return set_error(TQ_EINVAL, "%s: N < 0", fn);
   if (dtype != TQ_F32 && dtype != TQ_BF16) return set_error(TQ_EUNSUPPORTED, "%s: dtype %d", fn, dtype);
   if (rn_dtype != TQ_F32 && rn_dtype != TQ_F16) return set_error(TQ_EUNSUPPORTED, "%s: rn_dtype %d", fn, rn_dtype);

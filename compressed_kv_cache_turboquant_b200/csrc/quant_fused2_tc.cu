@@ -44,6 +44,8 @@
 
 #include <cmath>
 
+#include "tq.h"
+
 #include "sm100_common.cuh"
 #include "tq_internal.h"
 
@@ -59,6 +61,17 @@ constexpr int kAStage = 2 * kAPiece;       // hi + lo
 constexpr int kYCol = 0, kVCol = 256;
 constexpr float kUScale = 4096.f;
 constexpr int kMisc = 4096;
+
+// PolarQuant decisions (variant TQ_POLAR): level-1 sectors by quadrant and
+// tangent comparisons, levels >= 2 by squared radii against tan^2 of the
+// thresholds (theta >= t <=> r_b^2 >= tan^2(t) r_a^2 for radii r >= 0)
+struct PolarDec {
+  float t1[3];      // b1 = 4: tan(pi/8), 1, tan(3 pi/8)
+  float T[8][3];    // [level][k]: tan^2 of level-l threshold k (l = 2..L)
+  int b1, bh, L;
+  int base[9];      // first entry of level l among the packed codes of levels >= 2
+  int w1;           // words of the level-1 codes
+};
 
 struct F2Args {
   int64_t N;
@@ -77,6 +90,7 @@ struct F2Args {
   int xs, as, bs;           // stage counts of the three rings
   int x_stage_bytes, b_stage_bytes;
   int64_t row_tiles;
+  PolarDec pol;
   int* status;
 };
 
@@ -188,7 +202,82 @@ __device__ __forceinline__ void pack32(const uint32_t (&c)[32], uint32_t (&w)[BM
   }
 }
 
-template <int BM>
+// level-1 cell of the angle of (a, b) on the uniform grid of 2^b1 cells over [0, 2 pi)
+__device__ __forceinline__ uint32_t polar_sector(float a, float b, const PolarDec& P) {
+  if (a == 0.f && b == 0.f) return 0u;
+  uint32_t q;
+  float ap, bp;  // (a, b) rotated by -q quarter turns into [0, pi/2)
+  if (a > 0.f && b >= 0.f) q = 0u, ap = a, bp = b;
+  else if (a <= 0.f && b > 0.f) q = 1u, ap = b, bp = -a;
+  else if (a < 0.f && b <= 0.f) q = 2u, ap = -a, bp = -b;
+  else q = 3u, ap = -b, bp = a;
+  if (P.b1 == 2) return q;
+  const uint32_t sub = (bp >= P.t1[0] * ap ? 1u : 0u) + (bp >= P.t1[1] * ap ? 1u : 0u) + (bp >= P.t1[2] * ap ? 1u : 0u);
+  return 4u * q + sub;
+}
+
+// level-l (l >= 2) cell of atan2(r_b, r_a) from the squared radii
+__device__ __forceinline__ uint32_t polar_cell(float sa, float sb, const float (&T)[3], int bh) {
+  if (sa == 0.f && sb == 0.f) return 0u;
+  uint32_t c = sb >= T[0] * sa ? 1u : 0u;
+  if (bh == 2) c += (sb >= T[1] * sa ? 1u : 0u) + (sb >= T[2] * sa ? 1u : 0u);
+  return c;
+}
+
+__device__ __forceinline__ void put_bits(uint32_t* w, int e, uint32_t code, int bits) {
+  w[(e * bits) >> 5] |= code << ((e * bits) & 31);
+}
+
+// PolarQuant codes of one row whose rotated coordinates are the TMEM columns
+// [0, D) of this thread's lane
+template <int D>
+__device__ __forceinline__ void polar_row(uint32_t taddr, const PolarDec& P, uint32_t* dst, bool live) {
+  constexpr int G = D / 32;
+  uint32_t w1[8], wh[4];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) w1[q] = 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) wh[q] = 0u;
+  float sg[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float v[32];
+    tmem_ld32(taddr + (uint32_t)(32 * g), v);
+    tmem_wait_ld();
+    float s[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      put_bits(w1, 16 * g + p, polar_sector(v[2 * p], v[2 * p + 1], P), P.b1);
+      s[p] = fmaf(v[2 * p], v[2 * p], v[2 * p + 1] * v[2 * p + 1]);
+    }
+    // levels 2..5 inside the group: 8, 4, 2, 1 entries
+#pragma unroll
+    for (int lev = 2, cnt = 8; cnt >= 1; ++lev, cnt >>= 1) {
+#pragma unroll
+      for (int p = 0; p < cnt; ++p) {
+        put_bits(wh, P.base[lev] + cnt * g + p, polar_cell(s[2 * p], s[2 * p + 1], P.T[lev], P.bh), P.bh);
+        s[p] = s[2 * p] + s[2 * p + 1];
+      }
+    }
+    sg[g] = s[0];
+  }
+  // levels above the groups: pairs of group radii
+#pragma unroll
+  for (int lev = 6, cnt = G / 2; cnt >= 1; ++lev, cnt >>= 1) {
+#pragma unroll
+    for (int p = 0; p < cnt; ++p) {
+      put_bits(wh, P.base[lev] + p, polar_cell(sg[2 * p], sg[2 * p + 1], P.T[lev], P.bh), P.bh);
+      sg[p] = sg[2 * p] + sg[2 * p + 1];
+    }
+  }
+  if (live) {
+    for (int q = 0; q < P.w1; ++q) dst[q] = w1[q];
+    const int wn = ((D / 2 - 1 + 31) / 32) * P.bh;
+    for (int q = 0; q < wn; ++q) dst[P.w1 + q] = wh[q];
+  }
+}
+
+template <int BM, int POLAR_D>
 __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                    const __grid_constant__ CUtensorMap pimap,
                                                                    const __grid_constant__ CUtensorMap tmap,
@@ -457,6 +546,14 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_
         break;
       }
       tc_fence_after();
+      if constexpr (POLAR_D > 0) {
+        // one thread per row walks the whole angle tree; the other half idles
+        if (half == 0) polar_row<POLAR_D>(tmem_base + lane_base + kYCol, a.pol, a.codes + orow * a.W, live);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(y_empty);
+        continue;
+      }
       for (int g = half; g < a.G; g += 2) {
         const int jg = 32 * g;
         float v[32];
@@ -623,11 +720,29 @@ int launch_quant_fused2(const tq_ctx* h, const void* x, int dtype, int64_t N, in
     kern<<<grid, kThreads, smem, s>>>(xm, pm, tm, a);
     return (int)cudaGetLastError();
   };
+  if (h->variant == TQ_POLAR) {
+    a.prod = 0;
+    a.W = TQ_POLAR_WORDS(h->polar_b1, h->polar_bh, h->d);
+    PolarDec& P = a.pol;
+    P.b1 = h->polar_b1;
+    P.bh = h->polar_bh;
+    P.L = 0;
+    while ((1 << P.L) < h->d) ++P.L;
+    P.t1[0] = (float)std::tan(M_PI / 8);
+    P.t1[1] = 1.f;
+    P.t1[2] = (float)std::tan(3 * M_PI / 8);
+    P.base[2] = 0;
+    for (int l = 2; l < 8; ++l) P.base[l + 1] = P.base[l] + (h->d >> l);
+    for (int l = 0; l < 8; ++l)
+      for (int k = 0; k < 3; ++k) P.T[l][k] = (l >= 2 && l <= P.L) ? h->polar_tan2[l][k] : 0.f;
+    P.w1 = TQ_CODE_WORDS(P.b1, h->d / 2);
+    return h->d == 64 ? go(quant_fused2_kernel<1, 64>) : go(quant_fused2_kernel<1, 128>);
+  }
   switch (h->bm) {
-    case 1: return go(quant_fused2_kernel<1>);
-    case 2: return go(quant_fused2_kernel<2>);
-    case 3: return go(quant_fused2_kernel<3>);
-    default: return go(quant_fused2_kernel<4>);
+    case 1: return go(quant_fused2_kernel<1, 0>);
+    case 2: return go(quant_fused2_kernel<2, 0>);
+    case 3: return go(quant_fused2_kernel<3, 0>);
+    default: return go(quant_fused2_kernel<4, 0>);
   }
 }
 

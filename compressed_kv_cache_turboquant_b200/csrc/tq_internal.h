@@ -99,6 +99,11 @@ struct tq_ctx {
   // quantizer whose producer threads load x themselves (the one a channel
   // gather always takes) instead of the TMA-staged one
   bool fused_register_loads = false;
+  // PolarQuant (variant TQ_POLAR): level-1 bits, bits of levels >= 2, tan^2 of
+  // the thresholds of levels 2..7 and the cos / sin of every level's centroids
+  int polar_b1 = 0, polar_bh = 0;
+  float polar_tan2[8][3] = {};
+  float* polar_cs = nullptr;  // device [2][8 levels][16]: cos, sin of centroid k of level l (level 1 at l = 1)
   bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };

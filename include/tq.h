@@ -513,6 +513,70 @@ TQ_API int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* chann
                           void* workspace, size_t ws_bytes, void* stream);
 TQ_API size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int B, int Hq);
 
+/* ---------------------------------------------------------------- PolarQuant */
+
+/*
+ * PolarQuant, the polar stage-one variant ([tmdm, "双剑合璧：PolarQuant + QJL",
+ * ✦ PolarQuant]: after the random rotation the Cartesian coordinates become a
+ * radius and a chain of bounded angles, so no normalisation constants are
+ * stored; [admirer, "第一階段"]: coordinates are paired and mapped to polar
+ * form, the pair radii are transformed the same way, recursively, down to one
+ * final radius and a set of angles, each quantized with its own scalar
+ * quantizer).  Readings (the pages give no grid or bit allocation): d a power
+ * of two, L = log2 d levels; level-1 angles atan2(y_2i+1, y_2i) in [0, 2 pi)
+ * take b1 bits on the uniform grid (cells [k, k+1) 2 pi / 2^b1, centroid in
+ * the middle); an angle of level l >= 2, atan2(r_2i+1, r_2i) in [0, pi/2] of
+ * the level below's radii, takes bh bits of the Lloyd-Max quantizer of its law
+ * f_l ~ (sin t cos t)^(m-1), m = 2^(l-1) (sin^2 t ~ Beta(m/2, m/2) for a
+ * uniform point on the sphere); the final radius is ||x|| (float32).  Values
+ * on a threshold take the upper cell.  b1 = 4, bh = 2 spends about 3 bits per
+ * coordinate.
+ * Packed words per vector: TQ_POLAR_WORDS(b1, bh, d) = the d/2 level-1 codes in
+ * the b1-bit layout of the code words above (as if they were d/2
+ * coordinates), then the d/2 - 1 codes of levels 2..L (level 2 first, each
+ * level in order) in the bh-bit layout.
+ */
+#define TQ_POLAR 2
+#define TQ_POLAR_WORDS(b1, bh, d) (TQ_CODE_WORDS(b1, (d) / 2) + TQ_CODE_WORDS(bh, (d) / 2 - 1))
+
+/*
+ * tq_polar_codebook -- the scalar quantizer of one level's angles (host).
+ *   b           bits, 1..8;  level  1..12
+ *   centroids   host out [2^b] ascending; thresholds host out [2^b - 1] (may be NULL)
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED.
+ */
+TQ_API int tq_polar_codebook(int b, int level, double* centroids, double* thresholds);
+
+/*
+ * tq_create_polar -- a PolarQuant instance (variant TQ_POLAR).
+ *   d    64 or 128;  b1   2 or 4 (level-1 bits);  bh   1 or 2 (bits of levels >= 2)
+ *   Pi   host in [d*d] row-major float64 rotation (y = Pi x)
+ * Allocates the handle's constants on the current device.
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
+ */
+TQ_API int tq_create_polar(tq_handle* h, int d, int b1, int bh, const double* Pi);
+
+/*
+ * tq_quant_polar -- PolarQuant codes of N vectors: n = ||x||, y = Pi x on the
+ * tensor cores, the angle tree of y and each angle's cell (decided from the
+ * squared radii and tangents, no trigonometry).
+ *   x, dtype, N, x_stride, out_stride   as tq_quant_mse
+ *   codes   dev out, row i at codes + i*out_stride*TQ_POLAR_WORDS(b1, bh, d)
+ *   norms   dev out, float32, norms[i*out_stride]
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_quant_polar(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
+                          float* norms, int64_t out_stride, void* stream);
+
+/*
+ * tq_dequant_polar -- x_hat = n Pi^T y_hat, y_hat the unit tree rebuilt from
+ * the centroid angles (cos / sin products down the levels), on the tensor cores.
+ *   codes [N][TQ_POLAR_WORDS(b1, bh, d)], norms [N]; out [N][d] of out_dtype
+ * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_ECUDA.
+ */
+TQ_API int tq_dequant_polar(tq_handle h, const uint32_t* codes, const float* norms, int64_t N, void* out,
+                            int out_dtype, void* stream);
+
 /* ---------------------------------------------------------------- diagnostics */
 
 /*

@@ -122,3 +122,24 @@ def test_shard_merge_calls_reject_bad_arguments_before_any_gpu_work():
     assert L.tq_attn_merge(None, p, 2, 4, p, None) == _lib.TQ_EINVAL
     assert L.tq_attn_decode_partial(None, None, p, 0, 1, 4, 1, 10, 10, p, p, p, p, p, p, ctypes.c_float(0.1), p, p,
                                     0, None) == _lib.TQ_EINVAL
+
+
+@pytest.mark.parametrize("b,level", [(4, 1), (2, 1), (1, 2), (2, 2), (2, 5), (2, 7), (1, 6)])
+def test_host_polar_codebook_matches_oracle(b, level):
+    from oracle import polar as opq
+    c, t = tqmod.tq_polar_codebook(b, level)
+    co, to = opq.angle_codebook(b, level)
+    assert np.max(np.abs(c - co)) < 1e-12 and np.max(np.abs(t - to)) < 1e-12
+
+
+def test_polar_calls_reject_bad_arguments():
+    L = _lib.lib
+    h = ctypes.c_void_p()
+    Pi = np.eye(64)
+    dp = Pi.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    assert L.tq_create_polar(ctypes.byref(h), 96, 4, 2, dp) == _lib.TQ_EUNSUPPORTED     # not 64 / 128
+    assert L.tq_create_polar(ctypes.byref(h), 64, 3, 2, dp) == _lib.TQ_EUNSUPPORTED     # b1 3
+    assert L.tq_create_polar(ctypes.byref(h), 64, 4, 3, dp) == _lib.TQ_EUNSUPPORTED     # bh 3
+    assert L.tq_create_polar(None, 64, 4, 2, dp) == _lib.TQ_EINVAL
+    c = np.zeros(4)
+    assert L.tq_polar_codebook(2, 0, c.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), None) == _lib.TQ_EUNSUPPORTED
