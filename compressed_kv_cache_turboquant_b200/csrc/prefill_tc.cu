@@ -491,6 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
     if (ok && nkt > 0 && !mbar_wait(pv_done, (uint32_t)((nkt - 1) & 1))) ok = false;
     if (!ok) atomicOr(a.status, kStatusTimeout);
     tc_fence_after();
+    // records are d + 2 = 130 floats apart, so a record starts on an 8-byte
+    // (not always a 16-byte) boundary: two-float stores
     float* rec = a.partials + (grow * a.splits + split) * (D + 2);
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -504,8 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       }
       if (live)
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(rec + c0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        for (int e = 0; e < 32; e += 2) *reinterpret_cast<float2*>(rec + c0 + e) = make_float2(o[e], o[e + 1]);
     }
     if (live) {
       rec[D] = m_run > -FLT_MAX ? m_run / kLog2e : -FLT_MAX;
