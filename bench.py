@@ -299,15 +299,21 @@ class Sweep:
                 self.kern["quant_mse"].append((e0, e1, b))
                 self.kern["dequant_mse"].append((e1, e2, b))
 
+    def launch_bytes(self, name, b):
+        """Algorithmic bytes of one launch: quantize reads bf16 x and writes codes
+        and norms, dequantize reads codes and norms and writes fp32 x_hat."""
+        return self.N * (D * 2 + 16 * b + 4) if name == "quant_mse" else self.N * (16 * b + 4 + D * 4)
+
     def kernel_stats(self):
         out = {}
         for name, evs in self.kern.items():
             ms = [a.elapsed_time(bb) for a, bb, _ in evs]
-            if name == "quant_mse":
-                bytes_ = [self.N * (D * 2 + 16 * b + 4) for _, _, b in evs]
-            else:
-                bytes_ = [self.N * (16 * b + 4 + D * 4) for _, _, b in evs]
-            out[name] = dict(ms_total=sum(ms), launches=len(ms), bytes_total=sum(bytes_))
+            bytes_ = [self.launch_bytes(name, b) for _, _, b in evs]
+            per_b = {}
+            for (_, _, b), t in zip(evs, ms):
+                per_b.setdefault(b, []).append(t)
+            out[name] = dict(ms_total=sum(ms), launches=len(ms), bytes_total=sum(bytes_),
+                             per_b={b: (sum(v) / len(v), self.launch_bytes(name, b)) for b, v in per_b.items()})
         return out
 
     def units_per_step(self):
@@ -749,6 +755,10 @@ def run_ours(args):
     kernels = {k: {"avg_ms": v["ms_total"] / v["launches"],
                    "GBps": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9,
                    "frac_hbm": v["bytes_total"] / (v["ms_total"] / 1e3) / 1e9 / hbm} for k, v in ks.items()}
+    for k, v in ks.items():
+        if "per_b" in v:  # each bit width on its own: average launch time and its fraction of the peak
+            kernels[k]["per_b"] = {f"b{b}": {"us": round(t * 1e3, 2), "frac_hbm": round(by / (t / 1e3) / 1e9 / hbm, 4)}
+                                   for b, (t, by) in sorted(v["per_b"].items())}
 
     e2e = None
     if args.workload == "sweep" and not args.no_e2e:

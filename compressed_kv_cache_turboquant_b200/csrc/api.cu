@@ -140,19 +140,20 @@ static void scaled_half_codebook(tq_ctx* h) {
   h->sc_rel_err = best;
 }
 
-// Pi^T as fp16 pieces (hi, (Pi - hi) * 2^11) in the swizzled K-major layout:
-// B[i][j] = Pi[j][i], row i, K index j
+// 2^6 Pi^T as fp16 pieces (hi, 2^6 Pi - hi: the low piece true-valued, so
+// subnormal where small) in the swizzled K-major layout: B[i][j] = Pi[j][i],
+// row i, K index j
 static void split_rotation_t_f16(const double* Pi, int d, std::vector<uint16_t>& out) {
   const size_t piece = (size_t)d * d;
   out.assign(2 * piece, 0);
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) {
-      const double v = Pi[(size_t)j * d + i];
+      const double v = 64.0 * Pi[(size_t)j * d + i];
       const int slab = j / 64, c = (j % 64) / 8, e = j % 8;
       const size_t off = (size_t)slab * d * 64 + (size_t)i * 64 + (size_t)((c ^ (i & 7)) * 8 + e);
       const uint16_t hi = half_bits(v);
       out[off] = hi;
-      out[piece + off] = half_bits((v - half_value(hi)) * 2048.0);
+      out[piece + off] = half_bits(v - half_value(hi));
     }
 }
 
@@ -331,6 +332,7 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
   for (int k = 0; has_vtab && k < 16; ++k)
     if (h->host_centroids[15 - k] != -h->host_centroids[k]) has_vtab = false;  // needs c[15-i] = -c[i]
   if (has_ktab) byte_table(h->host_centroids, ktab);
+  for (int k = 0; k < 4; ++k) h->host_ktab[k] = ktab[k];
   if (has_vtab) byte_table(h->host_centroids + 8, vtab);
   const size_t oTabs = take(8 * 4);
   const size_t oGenPi = take(gpi.size() * 2);
@@ -375,6 +377,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
       e = (cudaError_t)probe_dyn_smem_base((uint32_t*)(h->dev.status + 16), &h->dyn_base);
     const char* fr = getenv("TQ_FUSED_REGISTER_LOADS");
     h->fused_register_loads = fr && fr[0] == '1';
+    const char* dl = getenv("TQ_LEGACY_MMA_SYNC");
+    h->legacy_mma = dl && dl[0] == '1';
     const char* st = getenv("TQ_DEBUG_STALL_MS");
     if (st && atof(st) > 0) h->debug_stall_ns = (uint64_t)(atof(st) * 1e6);
     const char* db = getenv("TQ_DEBUG_DYN_BASE");
@@ -631,11 +635,15 @@ size_t decode_workspace_bytes(const tq_ctx* hk, int B, int Hq, int Hkv, int64_t 
   const size_t simple = nq * decode_splits(B, Hq, T, hk->sm_count) * (hk->d + 2) * 4;
   const size_t fast = (size_t)decode_mma_grid(B, Hkv, T, hk->sm_count) * decode_mma_max_seg(B, Hkv, T, hk->sm_count) *
                       4 * (hk->d + 2) * 4;
-  return 2 * align_up(nq * hk->d * 4, 256) + align_up(nq * 2 * hk->d * 2, 256) + align_up(nq * 2 * 4, 256) +
-         align_up(std::max(simple, fast), 256);
+  const size_t tc = (size_t)decode_tc_grid(B, Hkv, T, hk->sm_count) * decode_tc_max_seg(B, Hkv, T, hk->sm_count) * 4 *
+                    (hk->d + 2) * 4;
+  const size_t qops = std::max(nq * 2 * hk->d * 2, decode_tc_qtile_bytes(B, Hkv));
+  return 2 * align_up(nq * hk->d * 4, 256) + align_up(qops, 256) + align_up(nq * 2 * 4, 256) +
+         align_up(std::max(simple, std::max(fast, tc)), 256);
 }
 
-// workspace: rotated queries | projected queries (fp32) | fp16 query operands | their scales | partials
+// workspace: rotated queries | projected queries (fp32) | fp16 query operands (fragments, or the
+// tcgen05 kernel's query tiles) | their scales | partials
 int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
                     int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
                     const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
@@ -646,10 +654,14 @@ int decode_dispatch(const tq_ctx* hk, const tq_ctx* hv, const void* q, int q_dty
   float* qrot = (float*)ws;
   float* qproj = (float*)(ws + q32);
   void* qfrag = ws + 2 * q32;
-  float* qscale = (float*)(ws + 2 * q32 + align_up(nq * 2 * hk->d * 2, 256));
+  const size_t qops = std::max(nq * 2 * hk->d * 2, decode_tc_qtile_bytes(B, Hkv));
+  float* qscale = (float*)(ws + 2 * q32 + align_up(qops, 256));
   float* partials = (float*)((char*)qscale + align_up(nq * 2 * 4, 256));
   int e = launch_query_prep(hk, (const float*)q, q_dtype, (int64_t)nq, qrot, qproj, stream);
   if (e) return e;
+  if (!pg.page && decode_tc_supported(hk, hv, Hq, Hkv, kv_stride, pg.rn16))
+    return launch_decode_tc(hk, hv, qrot, qproj, (uint8_t*)qfrag, qscale, B, Hq, Hkv, T, kv_stride, kcodes, ksigns,
+                            knorms, krnorms, vcodes, vnorms, scale, partials, out, stream, partial_out, pg.rn16);
   const bool mma = pg.page ? decode_mma_supported(hk, hv, Hq, Hkv, 4) && pg.page % 8 == 0
                             : decode_mma_supported(hk, hv, Hq, Hkv, kv_stride) && (!pg.rn16 || kv_stride % 8 == 0);
   if (mma) {
@@ -802,8 +814,8 @@ extern "C" size_t tq_attn_logits_workspace(const tq_handle* hk, int ngroups, int
     if (!hk[g]) return 0;
     bytes += 2 * align_up((size_t)B * Hq * hk[g]->d * 4, 256);
   }
-  // fp16 query fragments of the tensor-core path
-  if (ngroups == 2) bytes += logits_mma_workspace((int64_t)B * Hq);
+  // fp16 query operands of the tensor-core paths (fragments, or query tiles)
+  if (ngroups == 2) bytes += std::max(logits_mma_workspace((int64_t)B * Hq), logits_tc_workspace(B, (Hq + 3) / 4));
   return bytes;
 }
 
@@ -860,7 +872,10 @@ extern "C" int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* c
     off += hk[g]->d;
   }
   if (!e) {
-    if (logits_mma_supported(hk, ngroups, kv_stride))
+    if (logits_tc_supported(hk, ngroups, kv_stride))
+      e = launch_logits_tc(hk, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale, logits, ws,
+                           stream);
+    else if (logits_mma_supported(hk, ngroups, kv_stride))
       e = launch_logits_mma(hk, qr, qp, B, Hq, Hkv, T, kv_stride, kcodes, ksigns, knorms, krnorms, scale, logits, ws,
                             stream);
     else

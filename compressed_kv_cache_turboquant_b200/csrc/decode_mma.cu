@@ -663,8 +663,13 @@ int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag,
   kern<<<G, kThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  decode_merge_persistent_kernel<<<B * Hq, 128, 0, s>>>(partials, G, a.max_seg, a.nblk, a.total, Hq, Hkv,
-                                                        hv->dev.Pi, out, partial_out);
+  return launch_decode_merge_records(partials, G, a.max_seg, a.nblk, a.total, B, Hq, Hkv, hv, out, partial_out, s);
+}
+
+int launch_decode_merge_records(const float* partials, int64_t G, int max_seg, int64_t nblk, int64_t total, int B,
+                                int Hq, int Hkv, const tq_ctx* hv, float* out, int partial_out, void* stream) {
+  decode_merge_persistent_kernel<<<B * Hq, 128, 0, (cudaStream_t)stream>>>(partials, G, max_seg, nblk, total, Hq,
+                                                                           Hkv, hv->dev.Pi, out, partial_out);
   return (int)cudaGetLastError();
 }
 

@@ -96,26 +96,6 @@ struct PfArgs {
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-__device__ __forceinline__ void mma_ta(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
-      ::"r"(d), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
   uint32_t* u = reinterpret_cast<uint32_t*>(r);
   asm volatile(
@@ -238,8 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t boff = (uint32_t)((ks >> 2) * kTK * 128 + (ks & 3) * 32);
-          mma_ta(tmem + kColS1, tmem + kColQ1 + 8 * ks, sw128_kmajor_desc(cbase + boff), idesc, ks ? 1u : 0u);
-          mma_ta(tmem + kColS2, tmem + kColQ2 + 8 * ks, sw128_kmajor_desc(sbase + boff), idesc, ks ? 1u : 0u);
+          mma_f16_ta(tmem + kColS1, tmem + kColQ1 + 8 * ks, sw128_kmajor_desc(cbase + boff), idesc, ks ? 1u : 0u);
+          mma_f16_ta(tmem + kColS2, tmem + kColQ2 + 8 * ks, sw128_kmajor_desc(sbase + boff), idesc, ks ? 1u : 0u);
         }
         mma_commit(s_full);
         mma_commit(cs_free);
@@ -252,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t boff = (uint32_t)((ks >> 2) * kTK * 128 + (ks & 3) * 32);
-          mma_ta(tmem + kColO, tmem + kColS1 + 8 * ks, sw128_kmajor_desc(vbase + boff), idesc,
+          mma_f16_ta(tmem + kColO, tmem + kColS1 + 8 * ks, sw128_kmajor_desc(vbase + boff), idesc,
                  (it | ks) ? 1u : 0u);
         }
         mma_commit(pv_done);
@@ -392,10 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
           u1[c] = live ? h2u(__floats2half2_rn(q1[j1] * s1, q1[j1 + 1] * s1)) : 0u;
           u2[c] = live ? h2u(__floats2half2_rn(q2[j2a] * s2, q2[j2b] * s2)) : 0u;
         }
-        st16(tmem + lb + kColQ1 + c0, u1);
-        st16(tmem + lb + kColQ2 + c0, u2);
+        tmem_st16(tmem + lb + kColQ1 + c0, u1);
+        tmem_st16(tmem + lb + kColQ2 + c0, u2);
       }
-      wait_st();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
@@ -454,10 +434,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
             for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(o[16 * hh + e] * alpha);
-              st16(tmem + lb + kColO + c0 + 16 * hh, ou);
+              tmem_st16(tmem + lb + kColO + c0 + 16 * hh, ou);
             }
           }
-          wait_st();
+          tmem_wait_st();
         }
         l_run *= (it > 0) ? exp2f(m_run - mn) : 0.f;
         m_run = mn;
@@ -480,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
           l_run += __low2float(ph) + __high2float(ph);
           pu[e] = h2u(ph);
         }
-        st16(tmem + lb + kColS1 + c0 / 2, pu);
-        wait_st();
+        tmem_st16(tmem + lb + kColS1 + c0 / 2, pu);
+        tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();

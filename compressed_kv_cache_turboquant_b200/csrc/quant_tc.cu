@@ -13,11 +13,14 @@
 //   warp 1      TMEM allocation and the single-thread MMA issuer:
 //               Y[128 x d] = X[128 x d] . (Pi_hi + Pi_mid + Pi_lo)^T, three
 //               bf16 passes accumulated in fp32 in TMEM (double-buffered)
-//   warps 2..    epilogue, 4 warps per 32-coordinate group (d / 8 warps): one
-//               thread per vector (TMEM lane) and group; n = ||y|| (= ||x||,
-//               Pi orthogonal) from the groups' partial sums, the cell of every
-//               coordinate against n * t_k, packing, stores.  Four warps per
-//               SM sub-partition keep the issue slots busy.
+//   warps 2-13  epilogue: three sets of four warps (one per TMEM lane
+//               quarter) take the tiles in turn, each set with its own
+//               accumulator buffer, so three tiles are in flight; one thread
+//               per vector (TMEM lane) reads the vector's columns twice: once
+//               for n = ||y|| (= ||x||, Pi orthogonal), once for the cell of
+//               every coordinate against n * t_k, packing and stores.  Even
+//               32-coordinate groups search the thresholds on the ALU pipe,
+//               odd ones count them on the FMA pipe.
 //
 // Precision: x is exact in bf16; Pi = hi + mid + lo carries ~24 significant
 // bits, so every product is exact in fp32 and y has fp32-level error (far
@@ -37,9 +40,10 @@ using namespace sm100;
 
 constexpr int kPieces = 3;
 constexpr int kTileM = 128;
-// warps: TMA producer, MMA issuer, 4 epilogue warps per 32-coordinate group
+constexpr int kSets = 3;                  // epilogue warp sets = accumulator buffers
+// warps: TMA producer, MMA issuer, kSets sets of 4 epilogue warps
 template <int D>
-constexpr int threads_for() { return 32 * (2 + 4 * (D / 32)); }
+constexpr int threads_for() { return 32 * (2 + 4 * kSets); }
 
 template <int D>
 struct TcShape {
@@ -49,7 +53,7 @@ struct TcShape {
   static constexpr int kSlabBytesPi = D * 128;               // one slab of a D-row piece
   static constexpr int kPieceBytes = kSlabs * kSlabBytesPi;  // = D * D * 2
   static constexpr int kStages = (D == 128) ? 3 : 4;
-  static constexpr int kTmemCols = 2 * D;                    // two accumulators
+  static constexpr int kTmemCols = (kSets * D <= 256) ? 256 : 512;  // kSets accumulators
   static constexpr int kMiscBytes = 8192;  // barriers, TMEM slot, thresholds, norm partials
   static constexpr int kSmemBytes = kPieces * kPieceBytes + kStages * kStageBytes + kMiscBytes +
                                     1024 /*alignment*/;
@@ -204,15 +208,13 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(x_s + S::kStages * S::kStageBytes);
   uint64_t* full = bars;                       // [kStages]
   uint64_t* empty = bars + S::kStages;         // [kStages]
-  uint64_t* acc_full = bars + 2 * S::kStages;  // [2]
-  uint64_t* acc_empty = acc_full + 2;          // [2]
-  uint64_t* pi_bar = acc_empty + 2;
+  uint64_t* acc_full = bars + 2 * S::kStages;  // [kSets]
+  uint64_t* acc_empty = acc_full + kSets;      // [kSets]
+  uint64_t* pi_bar = acc_empty + kSets;
   uint64_t* done_bar = pi_bar + 1;
-  uint64_t* npart_bar = done_bar + 1;          // [2] norm partials of every group written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(npart_bar + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   float* thr_s = reinterpret_cast<float*>(tmem_slot + 4);  // [16]
-  float* npart = thr_s + 16;                               // [2 parity][d / 32 groups][128]
-  constexpr int kGroups = D / 32, kEpiWarps = 4 * kGroups;
+  constexpr int kGroups = D / 32;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = (a.N + kTileM - 1) / kTileM;
@@ -222,14 +224,12 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSets; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], 4);
     }
     mbar_init(pi_bar, 1);
     mbar_init(done_bar, 1);
-    mbar_init(&npart_bar[0], 32 * kEpiWarps);
-    mbar_init(&npart_bar[1], 32 * kEpiWarps);
     fence_mbar_init();
   }
   if (threadIdx.x < K - 1) thr_s[threadIdx.x] = a.thresholds[threadIdx.x];
@@ -268,8 +268,8 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
         const int s = i % S::kStages;
         const uint32_t u = (uint32_t)(i / S::kStages);
-        const int ab = i & 1;
-        const uint32_t ua = (uint32_t)(i >> 1);
+        const int ab = i % kSets;
+        const uint32_t ua = (uint32_t)(i / kSets);
         if (!mbar_wait(&full[s], u & 1u) || !mbar_wait(&acc_empty[ab], (ua & 1u) ^ 1u)) {
           ok = false;
           break;
@@ -293,65 +293,69 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       mma_commit(done_bar);  // arrives once everything issued above has completed
     }
   } else {
-    // epilogue: warp % 4 selects the TMEM lane quarter, (warp - 2) / 4 the 32-coordinate group
-    const int ew = warp - 2;
-    const int grp = ew >> 2;
+    // epilogue: set (warp - 2) / 4 takes tiles i = set (mod kSets) from its
+    // accumulator buffer; warp % 4 selects the TMEM lane quarter
+    const int set = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    float P[8];
+    constexpr int H = 1 << (BM - 1);
+    // positive thresholds t_m (m = 1 .. H - 1) and the constants of the FMA-pipe count
+    float tp[8], Cf[8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) P[m] = 0.f;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-      const int ab = i & 1;
-      const uint32_t ua = (uint32_t)(i >> 1);
+    for (int m = 0; m < 8; ++m) {
+      tp[m] = (m >= 1 && m < H) ? thr_s[H - 1 + m] : 0.f;
+      Cf[m] = (m >= 1 && m < H) ? 1.f - 4294967296.f * tp[m] : -1.f;
+    }
+    const uint32_t lb = (uint32_t)(quarter * 32) << 16;
+    int i = set;
+    for (int64_t tile = blockIdx.x + (int64_t)set * gridDim.x; tile < ntiles; tile += (int64_t)kSets * gridDim.x,
+                 i += kSets) {
+      const int ab = set;
+      const uint32_t ua = (uint32_t)(i / kSets);
       if (!mbar_wait(&acc_full[ab], ua & 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      float v[32];
-      tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * D + grp * 32), v);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      const uint32_t t0 = tmem_base + lb + (uint32_t)(ab * D);
+      // n = ||y|| from all of the vector's columns
       float ss = 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) ss = fmaf(v[c], v[c], ss);
-      // exchange the groups' partial sums of squares (bounded wait)
-      float* np = npart + (i & 1) * kGroups * 128;
-      np[grp * 128 + row] = ss;
-      mbar_arrive(&npart_bar[i & 1]);
-      if (!mbar_wait(&npart_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
-        atomicOr(a.status, kStatusTimeout);
-        break;
-      }
-      float sq = 0.f;
+      for (int g = 0; g < kGroups; ++g) {
+        float v[32];
+        tmem_ld32(t0 + 32 * g, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < kGroups; ++k) sq += np[k * 128 + row];
-      const float n = sqrtf(sq);
+        for (int c = 0; c < 32; ++c) ss = fmaf(v[c], v[c], ss);
+      }
+      const float n = sqrtf(ss);
       // a zero vector has y = 0, which lies below every positive threshold
+      float P[8], Cz[8];
 #pragma unroll
-      for (int m = 1; m < (1 << (BM - 1)); ++m) P[m] = n > 0.f ? n * thr_s[(1 << (BM - 1)) - 1 + m] : INFINITY;
-      const int64_t vec = tile * kTileM + row;
-      if (vec < a.N) {
-        uint32_t w[BM];
-        // odd groups count thresholds on the FMA pipe, even ones search on the ALU pipe
-        if (BM >= 2 && (grp & 1)) {
-          const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
-          float Cf[8];
-#pragma unroll
-          for (int m = 0; m < 8; ++m)
-            Cf[m] = (n > 0.f && m >= 1 && m < (1 << (BM - 1))) ? 1.f - 4294967296.f * thr_s[(1 << (BM - 1)) - 1 + m]
-                                                                : -1.f;
-          pack_group_fma<BM>(v, P, Bf, Cf, w);
-        } else {
-          pack_group<BM>(v, P, w);
-        }
-        store_words<BM>(a.codes + vec * a.out_stride * W + grp * BM, w);
-        if (grp == 0) a.norms[vec * a.out_stride] = n;
+      for (int m = 0; m < 8; ++m) {
+        P[m] = n > 0.f ? n * tp[m] : INFINITY;
+        Cz[m] = n > 0.f ? Cf[m] : -1.f;
       }
+      const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
+      const int64_t vec = tile * kTileM + row;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) {
+        float v[32];
+        tmem_ld32(t0 + 32 * g, v);
+        tmem_wait_ld();
+        if (g + 1 == kGroups) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+        if (vec < a.N) {
+          uint32_t w[BM];
+          if (BM >= 2 && (g & 1)) pack_group_fma<BM>(v, P, Bf, Cz, w);
+          else pack_group<BM>(v, P, w);
+          store_words<BM>(a.codes + vec * a.out_stride * W + g * BM, w);
+        }
+      }
+      if (vec < a.N) a.norms[vec * a.out_stride] = n;
     }
   }
 

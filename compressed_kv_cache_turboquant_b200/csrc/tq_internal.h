@@ -105,6 +105,13 @@ struct tq_ctx {
   float polar_tan2[8][3] = {};
   float* polar_cs = nullptr;  // device [2][8 levels][16]: cos, sin of centroid k of level l (level 1 at l = 1)
   bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
+  // TQ_LEGACY_MMA_SYNC=1 at creation: decode and split-cache logits take the
+  // mma.sync kernels instead of the tcgen05 ones (both stay covered by the
+  // parity tests)
+  bool legacy_mma = false;
+  // 3-bit codebook as fp16 byte tables (register decoding): lo bytes of c0-3,
+  // c4-7, hi bytes of c0-3, c4-7 (zero unless b = 3 mse bits)
+  uint32_t host_ktab[4] = {0, 0, 0, 0};
   double sc_rel_err = 0.0;  // max |fp16(alpha c) / alpha - c| / |c|
 };
 
@@ -196,6 +203,28 @@ bool decode_mma_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, i
 int decode_mma_grid(int B, int Hkv, int64_t T, int sm_count);
 int decode_mma_max_seg(int B, int Hkv, int64_t T, int sm_count);
 int launch_qfrag(const float* qrot, const float* qproj, int64_t nq, void* qfrag, float* qscale, void* stream);
+// combine the per-CTA softmax records of a persistent decode kernel (block
+// partition of `total` blocks, nblk per (batch, kv-head), max_seg records per
+// CTA and head) and rotate back once
+int launch_decode_merge_records(const float* partials, int64_t G, int max_seg, int64_t nblk, int64_t total, int B,
+                                int Hq, int Hkv, const tq_ctx* hv, float* out, int partial_out, void* stream);
+// split-cache logits on tcgen05
+bool logits_tc_supported(const tq_ctx* const* hk, int ngroups, int64_t kv_stride);
+size_t logits_tc_workspace(int B, int Hkv);
+int launch_logits_tc(const tq_ctx* const* hk, const float* const* qrot, const float* const* qproj, int B, int Hq,
+                     int Hkv, int64_t T, int64_t kv_stride, const uint32_t* const* kcodes,
+                     const uint32_t* const* ksigns, const float* const* knorms, const float* const* krnorms,
+                     float scale, float* logits, void* workspace, void* stream);
+// decode attention on tcgen05 (dense cache)
+bool decode_tc_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride, int rn16);
+int decode_tc_grid(int B, int Hkv, int64_t T, int sm_count);
+int decode_tc_max_seg(int B, int Hkv, int64_t T, int sm_count);
+size_t decode_tc_qtile_bytes(int B, int Hkv);
+int launch_decode_tc(const tq_ctx* hk, const tq_ctx* hv, const float* qrot, const float* qproj, uint8_t* qtiles,
+                     float* qscale, int B, int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
+                     const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,
+                     const float* vnorms, float scale, float* partials, float* out, void* stream, int partial_out,
+                     int rn16);
 int launch_decode_mma(const tq_ctx* hk, const tq_ctx* hv, const uint32_t* qfrag, const float* qscale, int B,
                       int Hq, int Hkv, int64_t T, int64_t kv_stride, const uint32_t* kcodes,
                       const uint32_t* ksigns, const float* knorms, const float* krnorms, const uint32_t* vcodes,

@@ -144,12 +144,16 @@ TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
  *                        of that kernel gives up after m ms: the call reports
  *                        TQ_STATUS_TIMEOUT and its output is undefined
  *   TQ_DEBUG_DYN_BASE=a  record `a` as the measured shared-window address, so
- *                        the decode and logits kernels built for the usual
- *                        address report TQ_STATUS_LAYOUT and write nothing
- * and one that selects between two implementations of the same arithmetic:
+ *                        the decode (mma.sync) and logits kernels built for the
+ *                        usual address report TQ_STATUS_LAYOUT and write nothing
+ * and two that select between implementations of the same arithmetic:
  *   TQ_FUSED_REGISTER_LOADS=1  quantization at d <= 256 takes the kernel whose
  *                        producer threads load x themselves (the one a channel
  *                        gather always takes) instead of the TMA-staged one
+ *   TQ_LEGACY_MMA_SYNC=1  tq_attn_decode on a dense cache and the two-group
+ *                        tq_attn_logits take the mma.sync kernels instead of
+ *                        the tcgen05 ones (a paged cache always takes the
+ *                        mma.sync decode kernel)
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
  */
 TQ_API int tq_create(tq_handle* h, int d, int b, int variant, const double* Pi, const double* S,

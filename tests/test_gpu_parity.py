@@ -357,20 +357,48 @@ def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
     assert_status_clean(hk, hv)
 
 
-def test_decode_small_ragged():
+# The dense 4-heads-per-kv-head decode and the two-group logits run on the
+# tcgen05 kernels; handles created with TQ_LEGACY_MMA_SYNC=1 take the mma.sync
+# kernels instead.
+DECODE_KERNELS = ["tcgen05", "mma_sync"]
+
+
+def _pick_decode_kernel(monkeypatch, kernel):
+    if kernel == "mma_sync":
+        monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
+    else:
+        monkeypatch.delenv("TQ_LEGACY_MMA_SYNC", raising=False)
+
+
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_decode_small_ragged(monkeypatch, kernel):
+    _pick_decode_kernel(monkeypatch, kernel)
     _decode_case(B=2, Hq=8, Hkv=2, T=1531, d=128, sample=[(0, 0), (0, 1), (1, 0), (1, 1)], seed=1,
                  stride_extra=5)
 
 
-def test_decode_cfg4_full_size_sampled():
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_decode_cfg4_full_size_sampled(monkeypatch, kernel):
     """B = 8, Hq = 32, Hkv = 8, d = 128, T = 131072: full launch, sampled slices."""
+    _pick_decode_kernel(monkeypatch, kernel)
     _decode_case(B=8, Hq=32, Hkv=8, T=131072, d=128, sample=[(0, 0), (7, 7), (3, 5)], seed=0)
 
 
-def test_decode_one_kv_head_long_context():
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_decode_one_kv_head_long_context(monkeypatch, kernel):
     """A single (batch, kv-head): every CTA of the persistent grid works on it and the
     merge combines hundreds of partials."""
+    _pick_decode_kernel(monkeypatch, kernel)
     _decode_case(B=1, Hq=4, Hkv=1, T=70001, d=128, sample=[(0, 0)], seed=2)
+
+
+def test_decode_tc_short_contexts():
+    """Contexts of one partial block, of a block and one token, and of many
+    (batch, kv-head) pairs per CTA: segment starts and ends inside the
+    tcgen05 kernel's pipeline, records of single-block segments."""
+    _decode_case(B=3, Hq=8, Hkv=2, T=37, d=128, sample=[(0, 0), (2, 1)], seed=6, stride_extra=3)
+    _decode_case(B=2, Hq=4, Hkv=1, T=129, d=128, sample=[(1, 0)], seed=7, stride_extra=3)
+    _decode_case(B=64, Hq=16, Hkv=4, T=300, d=128, sample=[(0, 0), (31, 2), (63, 3)], seed=8)
 
 
 def test_decode_fallback_shapes():
@@ -384,6 +412,7 @@ def test_decode_runtime_table_addresses(monkeypatch):
     """The decode kernel instance that adds its table addresses at run time (taken when the
     dynamic shared window is not where the library expects it) agrees just the same."""
     monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
+    monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
     _decode_case(B=2, Hq=8, Hkv=2, T=1531, d=128, sample=[(0, 1), (1, 0)], seed=5, stride_extra=5)
 
 
@@ -471,9 +500,10 @@ def test_bulk_gather_on_the_tensor_cores():
         _check_quant(inst, k64[:, chans], out)
 
 
-def _logits_case(B, Hq, Hkv, T, sample, seed=0):
+def _logits_case(B, Hq, Hkv, T, sample, seed=0, stride_extra=0):
     scales, hi, lo, ia, ib, channels = _split_instances(seed=seed)
-    rows = B * Hkv * T
+    S = T + stride_extra
+    rows = B * Hkv * S
     g = torch.Generator(device=DEV).manual_seed(seed)
     cache = {}
     for inst, name in ((ia, "a"), (ib, "b")):
@@ -486,7 +516,7 @@ def _logits_case(B, Hq, Hkv, T, sample, seed=0):
     refs = {}
     for (b, h) in sample:
         k64 = _split_keys(T, b * Hkv + h, scales, seed)
-        r0 = (b * Hkv + h) * T
+        r0 = (b * Hkv + h) * S
         st = {}
         for inst, name, chans in ((ia, "a", hi), (ib, "b", lo)):
             s_ = inst.oracle_quant(k64[:, chans])
@@ -500,7 +530,7 @@ def _logits_case(B, Hq, Hkv, T, sample, seed=0):
     q = to_device(q64, torch.bfloat16)
     logits = torch.empty((B, Hq, T), dtype=torch.float32, device=DEV)
     scale = 1.0 / math.sqrt(128)
-    tq.tq_attn_logits([ia.h, ib.h], channels, q, Hkv, T, T, [cache["a"]["codes"], cache["b"]["codes"]],
+    tq.tq_attn_logits([ia.h, ib.h], channels, q, Hkv, T, S, [cache["a"]["codes"], cache["b"]["codes"]],
                       [cache["a"]["signs"], cache["b"]["signs"]], [cache["a"]["norms"], cache["b"]["norms"]],
                       [cache["a"]["rnorms"], cache["b"]["rnorms"]], scale, logits)
     torch.cuda.synchronize()
@@ -521,16 +551,29 @@ def _logits_case(B, Hq, Hkv, T, sample, seed=0):
 
 
 def test_split_group_logits_small_ragged():
+    """Context 1001 with a cache stride of 1001: the general kernel."""
     _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 0), (1, 1)], seed=1)
+
+
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_split_group_logits_ragged_tensor_core(monkeypatch, kernel):
+    """Context 1001 (a 3-token tail past the last whole group of 4) with a cache
+    stride of 1004, and a context shorter than one block: the tensor-core kernels."""
+    _pick_decode_kernel(monkeypatch, kernel)
+    _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 0), (1, 1)], seed=1, stride_extra=3)
+    _logits_case(B=3, Hq=4, Hkv=1, T=70, sample=[(2, 0)], seed=3, stride_extra=2)
 
 
 def test_split_group_logits_runtime_table_addresses(monkeypatch):
     monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
-    _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 1), (1, 0)], seed=2)
+    monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
+    _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 1), (1, 0)], seed=2, stride_extra=3)
 
 
-def test_split_group_logits_full_context_sampled():
+@pytest.mark.parametrize("kernel", DECODE_KERNELS)
+def test_split_group_logits_full_context_sampled(monkeypatch, kernel):
     """Batch 1, 32 q-heads / 8 kv-heads, context 2^20: the full launch, one kv-head checked."""
+    _pick_decode_kernel(monkeypatch, kernel)
     _logits_case(B=1, Hq=32, Hkv=8, T=1 << 20, sample=[(0, 5)], seed=0)
 
 
