@@ -801,6 +801,8 @@ def run_ours(args):
                             "bytes_per_step": dl.bytes_per_step(),
                             "config": "B=8, Hq=32, Hkv=8, d=128, T=131072, K prod 4b, V mse 4b"}
         try:
+            if args.no_prefill:
+                raise RuntimeError("prefill not run (--no-prefill)")
             pf = Prefill(tq, torch, dl)
             for _ in range(args.warmup):
                 pf.step()
@@ -979,6 +981,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-search", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--search-d", type=int, default=200)
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
                     help="run a small case of one workload for an ncu capture instead of the bench")

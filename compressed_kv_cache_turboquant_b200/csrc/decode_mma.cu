@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
         }
       }
       mbar_arrive(pub);
-      if (!mbar_wait_ns(pub, 0u, a.wait_ns)) {
+      if (!mbar_wait_warp(pub, 0u, a.wait_ns)) {
         ok = false;
         return;
       }
@@ -344,10 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecArgs a) {
       }
       // second phase: everyone has read the merge buffer before it is written again
       mbar_arrive(pub);
-      if (!mbar_wait_ns(pub, 1u, a.wait_ns)) ok = false;
+      if (!mbar_wait_warp(pub, 1u, a.wait_ns)) ok = false;
     };
 
-    if (a.stall && !mbar_wait_ns(never, 0u, a.wait_ns)) ok = false;
+    if (a.stall && !mbar_wait_warp(never, 0u, a.wait_ns)) ok = false;
     BlockCursor cur;
     cur.init(gb_lo, a.nblk);
     const int nblocks = (int)(gb_hi - gb_lo);

@@ -368,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
     for (int i = 0; i < nb; ++i) {
       const int r = i % kStages, s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
-      if (!mbar_wait_ns(&full[r], (uint32_t)((i / kStages) & 1), wl) ||
-          !mbar_wait_ns(&qk_done[s], (u & 1u) ^ 1u, wl)) {
+      if (!mbar_wait_warp(&full[r], (uint32_t)((i / kStages) & 1), wl) ||
+          !mbar_wait_warp(&qk_done[s], (u & 1u) ^ 1u, wl)) {
         ok = false;
         break;
       }
@@ -426,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
     for (int i = 0; i < nb; ++i) {
       const int r = i % kStages, s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
-      if (!mbar_wait_ns(&full[r], (uint32_t)((i / kStages) & 1), wl) ||
-          !mbar_wait_ns(&pv_done[s], (u & 1u) ^ 1u, wl)) {
+      if (!mbar_wait_warp(&full[r], (uint32_t)((i / kStages) & 1), wl) ||
+          !mbar_wait_warp(&pv_done[s], (u & 1u) ^ 1u, wl)) {
         ok = false;
         break;
       }
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
     const int tid = threadIdx.x - 320;
     const int group = a.Hq / a.Hkv;            // 4
     bool ok = true;
-    if (a.stall && !mbar_wait_ns(never, 0u, wl)) ok = false;
+    if (a.stall && !mbar_wait_warp(never, 0u, wl)) ok = false;
     float inv1[4] = {0.f, 0.f, 0.f, 0.f}, inv2[4] = {0.f, 0.f, 0.f, 0.f};
     float m_run[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX}, lsum[4] = {0.f, 0.f, 0.f, 0.f};
     float oreg[4] = {0.f, 0.f, 0.f, 0.f}, alpha_prev[4] = {1.f, 1.f, 1.f, 1.f};
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
         for (int h = 0; h < 4; ++h) rl[sw_idx * 4 + h] = lsum[h];
         mbar_arrive(fbar);
       }
-      if (!mbar_wait_ns(fbar, (uint32_t)(nflush & 1), wl)) return false;
+      if (!mbar_wait_warp(fbar, (uint32_t)(nflush & 1), wl)) return false;
       ++nflush;
       float* dst = a.partials + ((int64_t)blockIdx.x * a.max_seg + sg) * 4 * (D + 2);
 #pragma unroll
@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
       }
       const int64_t t0 = cur.blk * kTok;
       const int n = (int)min((int64_t)kTok, a.T - t0);
-      if (!mbar_wait_ns(&s_full[s], u & 1u, wl)) {
+      if (!mbar_wait_warp(&s_full[s], u & 1u, wl)) {
         ok = false;
         break;
       }
@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
         for (int h = 0; h < 4; ++h) rx[sw_idx * 4 + h] = mx[h];
         mbar_arrive(&xbar[s]);
       }
-      if (!mbar_wait_ns(&xbar[s], u & 1u, wl)) {
+      if (!mbar_wait_warp(&xbar[s], u & 1u, wl)) {
         ok = false;
         break;
       }
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
         lsum[h] = fmaf(lsum[h], alpha[h], p[h] * kPScale);
       }
       // weights p |v| / 16 into row h of the weight tile (K-major, keys as K)
-      if (!mbar_wait_ns(&pv_done[s], (u & 1u) ^ 1u, wl)) {
+      if (!mbar_wait_warp(&pv_done[s], (u & 1u) ^ 1u, wl)) {
         ok = false;
         break;
       }
@@ -607,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(TcDecArgs a) {
       // fold the previous tile's O (same segment) into the registers: lane = coordinate t
       auto absorb = [&](int j, const float (&al)[4]) -> bool {
         const int sj = j & 1;
-        if (!mbar_wait_ns(&o_full[sj], (uint32_t)((j >> 1) & 1), wl)) return false;
+        if (!mbar_wait_warp(&o_full[sj], (uint32_t)((j >> 1) & 1), wl)) return false;
         tc_fence_after();
         float o[4];
         tmem_ld4(tmem + lb + kColO + 16u * sj, o);

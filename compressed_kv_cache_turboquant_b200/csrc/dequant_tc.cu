@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
-      if (!mbar_wait(&a_empty[s], (u & 1u) ^ 1u)) {
+      if (!mbar_wait_warp(&a_empty[s], (u & 1u) ^ 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       const int64_t vec = tile * kTileM + r;
       const int64_t row0 = tile * kTileM + quarter * 32;
       const float n = ((vec < a.N) ? a.norms[vec] : 0.f) * kInvScale2;  // issued before the wait
-      if (!mbar_wait(&acc_full[s], u & 1u)) {
+      if (!mbar_wait_warp(&acc_full[s], u & 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }

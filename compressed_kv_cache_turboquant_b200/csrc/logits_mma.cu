@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_mma_kernel(LgArgs a) {
       const int s = stg;
       const uint32_t ph = phase;
       if (++stg == kStages) stg = 0, phase ^= 1u;
-      if (!mbar_wait(&full[s], ph)) {
+      if (!mbar_wait_warp(&full[s], ph)) {
         ok = false;
         break;
       }

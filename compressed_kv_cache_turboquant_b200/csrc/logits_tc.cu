@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_tc_kernel(LtArgs a) {
     for (int i = 0; i < nb; ++i, cur.next(a.nblk)) {
       const int r = i % kStages, s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
-      if (!mbar_wait(&full[r], (uint32_t)((i / kStages) & 1)) || !mbar_wait(&qk_done[s], (u & 1u) ^ 1u)) {
+      if (!mbar_wait_warp(&full[r], (uint32_t)((i / kStages) & 1)) || !mbar_wait_warp(&qk_done[s], (u & 1u) ^ 1u)) {
         ok = false;
         break;
       }
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) logits_tc_kernel(LtArgs a) {
             c2[g][h] = qs[1] * kQjl64 * a.scale;
           }
       }
-      if (!mbar_wait(&s_full[s], u & 1u)) {
+      if (!mbar_wait_warp(&s_full[s], u & 1u)) {
         ok = false;
         break;
       }

@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       const int64_t t0 = (kt_lo + it) * kTK;
       const int n = (int)min((int64_t)kTK, a.T - t0);
       const int64_t row0 = bh * a.kv_stride + t0;
-      if (!mbar_wait(&full[s], (uint32_t)((it >> 1) & 1)) ||
-          (it > 0 && !mbar_wait(cs_free, (uint32_t)((it - 1) & 1)))) {
+      if (!mbar_wait_warp(&full[s], (uint32_t)((it >> 1) & 1)) ||
+          (it > 0 && !mbar_wait_warp(cs_free, (uint32_t)((it - 1) & 1)))) {
         ok = false;
         break;
       }
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       if (lane == 0) mbar_arrive(cs_ready);
       // transposed value tile: row = coordinate, K = keys; thread (m, ch) writes
       // the words (v[2m][c], v[2m+1][c]) for coordinates c of half ch
-      if (it > 0 && !mbar_wait(pv_done, (uint32_t)((it - 1) & 1))) {
+      if (it > 0 && !mbar_wait_warp(pv_done, (uint32_t)((it - 1) & 1))) {
         ok = false;
         break;
       }
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
     bool ok = true;
     for (int it = 0; ok && it < nkt; ++it) {
       const int64_t t0 = (kt_lo + it) * kTK;
-      if (!mbar_wait(s_full, (uint32_t)(it & 1))) {
+      if (!mbar_wait_warp(s_full, (uint32_t)(it & 1))) {
         ok = false;
         break;
       }
@@ -414,31 +414,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) mx = fmaxf(mx, x[e]);
       }
-      // lazy rescale: the reference max moves only when a logit passes it by kLazy
-      if (mx > m_run + kLazy || (it == 0 && mx > -FLT_MAX)) {
-        const float mn = mx;
-        if (it > 0) {
-          const float alpha = exp2f(m_run - mn);
-          if (!mbar_wait(pv_done, (uint32_t)((it - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            float o[32];
-            tmem_ld32(tmem + lb + kColO + c0, o);
-            tmem_wait_ld();
-            uint32_t ou[16];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(o[16 * hh + e] * alpha);
-              tmem_st16(tmem + lb + kColO + c0 + 16 * hh, ou);
-            }
-          }
-          tmem_wait_st();
+      // lazy rescale: a row's reference max moves only when one of its logits
+      // passes it by kLazy.  The O rescale goes through warp-collective tensor
+      // memory loads and stores, so the whole warp takes it when any row needs
+      // it (rows that do not rescale by 1).
+      const bool grow = mx > m_run + kLazy || (it == 0 && mx > -FLT_MAX);
+      const float mn = grow ? mx : m_run;
+      if (it > 0 && __any_sync(0xffffffffu, grow)) {
+        const float alpha = grow ? exp2f(m_run - mn) : 1.f;
+        if (!mbar_wait_warp(pv_done, (uint32_t)((it - 1) & 1))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float o[32];
+          tmem_ld32(tmem + lb + kColO + c0, o);
+          tmem_wait_ld();
+          uint32_t ou[16];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(o[16 * hh + e] * alpha);
+            tmem_st16(tmem + lb + kColO + c0 + 16 * hh, ou);
+          }
+        }
+        tmem_wait_st();
+      }
+      if (grow) {
         l_run *= (it > 0) ? exp2f(m_run - mn) : 0.f;
         m_run = mn;
       }
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       if (lane == 0) mbar_arrive(p_ready);
     }
     // the record of this row: acc (rotated frame), m (natural units), l
-    if (ok && nkt > 0 && !mbar_wait(pv_done, (uint32_t)((nkt - 1) & 1))) ok = false;
+    if (ok && nkt > 0 && !mbar_wait_warp(pv_done, (uint32_t)((nkt - 1) & 1))) ok = false;
     if (!ok) atomicOr(a.status, kStatusTimeout);
     tc_fence_after();
     // records are d + 2 = 130 floats apart, so a record starts on an 8-byte

@@ -449,8 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_
       const float sc = v < a.N ? vscale(a.norms[out_row2(a, v)]) : 0.f;
       for (int k = 0; k < kc; ++k, ++seq) {
         const int sx = (int)(seq % a.xs), sa = (int)(seq % a.as);
-        if (!mbar_wait(&x_full[sx], (uint32_t)((seq / a.xs) & 1)) ||
-            !mbar_wait(&a_empty[sa], (uint32_t)(((seq / a.as) & 1) ^ 1))) {
+        if (!mbar_wait_warp(&x_full[sx], (uint32_t)((seq / a.xs) & 1)) ||
+            !mbar_wait_warp(&a_empty[sa], (uint32_t)(((seq / a.as) & 1) ^ 1))) {
           ok = false;
           break;
         }
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_
       for (int m = 1; m < 8; ++m)
         if (m < (1 << (BM - 1))) P[m] = n > 0.f ? ns * thr_s[(1 << (BM - 1)) - 1 + m] : INFINITY;
       float u2 = 0.f;
-      if (!mbar_wait(y_full, (uint32_t)(i & 1))) {
+      if (!mbar_wait_warp(y_full, (uint32_t)(i & 1))) {
         ok = false;
         break;
       }
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_
       float* rs = rn_s + (i & 1) * 256;
       rs[half * 128 + row] = u2;
       mbar_arrive(&rn_bar[i & 1]);
-      if (!mbar_wait(&rn_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
+      if (!mbar_wait_warp(&rn_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
         ok = false;
         break;
       }
@@ -591,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused2_kernel(const __grid_
         else
           a.rnorms[orow] = rn;
       }
-      if (!mbar_wait(v_full, (uint32_t)(i & 1))) {
+      if (!mbar_wait_warp(v_full, (uint32_t)(i & 1))) {
         ok = false;
         break;
       }

@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused_kernel(const __grid_c
       }
       for (int k = 0; k < kc; ++k, ++seq) {
         const int s = (int)(seq % AS);
-        if (!mbar_wait(&a_empty[s], (uint32_t)(((seq / AS) & 1) ^ 1))) {
+        if (!mbar_wait_warp(&a_empty[s], (uint32_t)(((seq / AS) & 1) ^ 1))) {
           ok = false;
           break;
         }
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused_kernel(const __grid_c
       for (int m = 1; m < 8; ++m)
         if (m < (1 << (BM - 1))) P[m] = n > 0.f ? ns * thr_s[(1 << (BM - 1)) - 1 + m] : INFINITY;
       float u2 = 0.f;
-      if (!mbar_wait(y_full, (uint32_t)(i & 1))) {
+      if (!mbar_wait_warp(y_full, (uint32_t)(i & 1))) {
         ok = false;
         break;
       }
@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused_kernel(const __grid_c
         if (a.prod) {
           // the residual chunk k of this tile into the operand ring
           const int s = (int)(seq % AS);
-          if (!mbar_wait(&a_empty[s], (uint32_t)(((seq / AS) & 1) ^ 1))) {
+          if (!mbar_wait_warp(&a_empty[s], (uint32_t)(((seq / AS) & 1) ^ 1))) {
             ok = false;
             break;
           }
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused_kernel(const __grid_c
       float* rs = rn_s + (i & 1) * 256;
       rs[half * 128 + row] = u2;
       mbar_arrive(&rn_bar[i & 1]);
-      if (!mbar_wait(&rn_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
+      if (!mbar_wait_warp(&rn_bar[i & 1], (uint32_t)((i >> 1) & 1))) {
         ok = false;
         break;
       }
@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_fused_kernel(const __grid_c
           a.rnorms[orow] = rn;
       }
       // QJL bits from the projection
-      if (!mbar_wait(v_full, (uint32_t)(i & 1))) {
+      if (!mbar_wait_warp(v_full, (uint32_t)(i & 1))) {
         ok = false;
         break;
       }

@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_gen_kernel(const __grid_con
       }
       for (int kc = 0; kc < KC; ++kc, ++ch) {
         const int s = (int)(ch % kStages);
-        if (!mbar_wait(&a_empty[s], (uint32_t)(((ch / kStages) & 1) ^ 1))) {
+        if (!mbar_wait_warp(&a_empty[s], (uint32_t)(((ch / kStages) & 1) ^ 1))) {
           ok = false;
           break;
         }
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_gen_kernel(const __grid_con
         u2 = 0.f;
       }
       const int ab = i & 1;
-      if (!mbar_wait(&acc_full[ab], (uint32_t)((i >> 1) & 1))) {
+      if (!mbar_wait_warp(&acc_full[ab], (uint32_t)((i >> 1) & 1))) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
@@ -548,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_gen_kernel(const __grid_con
         float* rs = rn_s + (nrt & 1) * 256;
         rs[half * 128 + row] = u2;
         mbar_arrive(&rn_bar[nrt & 1]);
-        if (!mbar_wait(&rn_bar[nrt & 1], (uint32_t)((nrt >> 1) & 1))) {
+        if (!mbar_wait_warp(&rn_bar[nrt & 1], (uint32_t)((nrt >> 1) & 1))) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }

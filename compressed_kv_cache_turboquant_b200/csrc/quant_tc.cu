@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
                  i += kSets) {
       const int ab = set;
       const uint32_t ua = (uint32_t)(i / kSets);
-      if (!mbar_wait(&acc_full[ab], ua & 1u)) {
+      if (!mbar_wait_warp(&acc_full[ab], ua & 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }

@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
           else qk[kr] = valid ? __uint_as_float(slot[7]) * a.qjl_coef : 0.f;
         }
         const int sb = (int)(ch % kBStages);
-        if (!mbar_wait(&b_empty[sb], (uint32_t)(((ch / kBStages) & 1) ^ 1))) {
+        if (!mbar_wait_warp(&b_empty[sb], (uint32_t)(((ch / kBStages) & 1) ^ 1))) {
           ok = false;
           break;
         }
@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         kth = -FLT_MAX;
       }
       const int ab = i & 1;
-      if (!mbar_wait(&acc_full[ab], (uint32_t)((i >> 1) & 1))) {
+      if (!mbar_wait_warp(&acc_full[ab], (uint32_t)((i >> 1) & 1))) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }

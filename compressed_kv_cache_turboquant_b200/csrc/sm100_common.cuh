@@ -93,6 +93,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_ns(bar, parity, kWaitLimitNs);
 }
 
+// The same wait made by all 32 lanes of a warp, whose result every lane
+// shares: a warp that goes on to warp-collective instructions (tcgen05.ld /
+// st, shuffles, __syncwarp) must not split into lanes that gave up and lanes
+// that did not.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait_ns(bar, parity, limit_ns));
+}
+
 // 2D tiled TMA load into shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int y) {
   asm volatile(
