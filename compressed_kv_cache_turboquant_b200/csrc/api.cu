@@ -140,20 +140,19 @@ static void scaled_half_codebook(tq_ctx* h) {
   h->sc_rel_err = best;
 }
 
-// 2^6 Pi^T as fp16 pieces (hi, 2^6 Pi - hi: the low piece true-valued, so
-// subnormal where small) in the swizzled K-major layout: B[i][j] = Pi[j][i],
-// row i, K index j
+// Pi^T as fp16 pieces (hi, (Pi - hi) * 2^11) in the swizzled K-major layout:
+// B[i][j] = Pi[j][i], row i, K index j
 static void split_rotation_t_f16(const double* Pi, int d, std::vector<uint16_t>& out) {
   const size_t piece = (size_t)d * d;
   out.assign(2 * piece, 0);
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) {
-      const double v = 64.0 * Pi[(size_t)j * d + i];
+      const double v = Pi[(size_t)j * d + i];
       const int slab = j / 64, c = (j % 64) / 8, e = j % 8;
       const size_t off = (size_t)slab * d * 64 + (size_t)i * 64 + (size_t)((c ^ (i & 7)) * 8 + e);
       const uint16_t hi = half_bits(v);
       out[off] = hi;
-      out[piece + off] = half_bits(v - half_value(hi));
+      out[piece + off] = half_bits((v - half_value(hi)) * 2048.0);
     }
 }
 
@@ -175,6 +174,7 @@ extern "C" const char* tq_version(void) { return "tq-b200 0.1 (sm_100a)"; }
 
 extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double* Pi,
                          const double* S, const double* centroids) {
+  TQ_TRACE("tq_create");
   if (!out || !Pi) return set_error(TQ_EINVAL, "tq_create: NULL handle or rotation");
   *out = nullptr;
   if (variant != TQ_MSE && variant != TQ_PROD)
@@ -377,8 +377,8 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
       e = (cudaError_t)probe_dyn_smem_base((uint32_t*)(h->dev.status + 16), &h->dyn_base);
     const char* fr = getenv("TQ_FUSED_REGISTER_LOADS");
     h->fused_register_loads = fr && fr[0] == '1';
-    const char* dl = getenv("TQ_LEGACY_MMA_SYNC");
-    h->legacy_mma = dl && dl[0] == '1';
+    const char* dl = getenv("TQ_TCGEN05_ATTN");
+    h->tc_attn = dl && dl[0] == '1';
     const char* st = getenv("TQ_DEBUG_STALL_MS");
     if (st && atof(st) > 0) h->debug_stall_ns = (uint64_t)(atof(st) * 1e6);
     const char* db = getenv("TQ_DEBUG_DYN_BASE");
@@ -415,6 +415,7 @@ extern "C" int tq_create(tq_handle* out, int d, int b, int variant, const double
 }
 
 extern "C" int tq_create_polar(tq_handle* out, int d, int b1, int bh, const double* Pi) {
+  TQ_TRACE("tq_create_polar");
   if (!out || !Pi) return set_error(TQ_EINVAL, "tq_create_polar: NULL handle or rotation");
   *out = nullptr;
   if (d != 64 && d != 128) return set_error(TQ_EUNSUPPORTED, "tq_create_polar: d = %d (need 64 or 128)", d);
@@ -455,6 +456,7 @@ extern "C" int tq_create_polar(tq_handle* out, int d, int b1, int bh, const doub
 }
 
 extern "C" int tq_destroy(tq_handle h) {
+  TQ_TRACE("tq_destroy");
   if (!h) return clear_error();
   int e = cudaDeviceSynchronize();
   if (h->polar_cs) cudaFree(h->polar_cs);
@@ -473,6 +475,7 @@ extern "C" int tq_device_status(tq_handle h, int* status) {
 }
 
 extern "C" int tq_handle_info(tq_handle h, int* d, int* b, int* variant, int* mse_bits) {
+  TQ_TRACE("tq_handle_info");
   if (!h) return set_error(TQ_EINVAL, "tq_handle_info: NULL handle");
   if (d) *d = h->d;
   if (b) *b = h->b;
@@ -501,6 +504,7 @@ static int check_quant_args(const char* fn, tq_handle h, int want_variant, const
 
 extern "C" int tq_quant_mse(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                             uint32_t* codes, float* norms, int64_t out_stride, void* stream) {
+  TQ_TRACE("tq_quant_mse");
   int rc = check_quant_args("tq_quant_mse", h, TQ_MSE, x, dtype, N, x_stride, codes, norms, out_stride);
   if (rc) return rc;
   if (N == 0) return clear_error();
@@ -542,6 +546,7 @@ static int quant_prod_impl(const char* fn, tq_handle h, const void* x, int dtype
 extern "C" int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                              uint32_t* codes, uint32_t* signs, float* norms, float* rnorms,
                              int64_t out_stride, void* stream) {
+  TQ_TRACE("tq_quant_prod");
   return quant_prod_impl("tq_quant_prod", h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride,
                          nullptr, 0, stream);
 }
@@ -549,6 +554,7 @@ extern "C" int tq_quant_prod(tq_handle h, const void* x, int dtype, int64_t N, i
 extern "C" int tq_quant_prod_ws(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                                 uint32_t* codes, uint32_t* signs, float* norms, float* rnorms, int64_t out_stride,
                                 void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_quant_prod_ws");
   return quant_prod_impl("tq_quant_prod_ws", h, x, dtype, N, x_stride, codes, signs, norms, rnorms, out_stride,
                          workspace, ws_bytes, stream);
 }
@@ -563,6 +569,7 @@ extern "C" size_t tq_quant_prod_workspace(tq_handle h, int64_t N) {
 
 extern "C" int tq_dequant_mse(tq_handle h, const uint32_t* codes, const float* norms, int64_t N,
                               void* out, int out_dtype, void* stream) {
+  TQ_TRACE("tq_dequant_mse");
   if (!h) return set_error(TQ_EINVAL, "tq_dequant_mse: NULL handle");
   if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_dequant_mse: a TQ_POLAR handle (use tq_dequant_polar)");
   if (N < 0) return set_error(TQ_EINVAL, "tq_dequant_mse: N < 0");
@@ -592,6 +599,7 @@ extern "C" int tq_ip_scores(tq_handle h, const float* q, int64_t nq, const uint3
                             const uint32_t* signs, const float* norms, const float* rnorms,
                             int64_t N, float* scores, int topk, int32_t* top_idx, float* top_val,
                             void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_ip_scores");
   if (!h) return set_error(TQ_EINVAL, "tq_ip_scores: NULL handle");
   if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_ip_scores: a TQ_POLAR handle");
   if (nq < 0 || N < 0) return set_error(TQ_EINVAL, "tq_ip_scores: negative size");
@@ -687,6 +695,7 @@ extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_d
                               const uint32_t* ksigns, const float* knorms, const float* krnorms,
                               const uint32_t* vcodes, const float* vnorms, float scale, float* out,
                               void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_attn_decode");
   if (!hk || !hv) return set_error(TQ_EINVAL, "tq_attn_decode: NULL handle");
   if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)
     return set_error(TQ_EINVAL, "tq_attn_decode: need a TQ_PROD key handle and a TQ_MSE value handle");
@@ -714,6 +723,7 @@ extern "C" int tq_attn_decode(tq_handle hk, tq_handle hv, const void* q, int q_d
 
 extern "C" int tq_quant_polar(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride, uint32_t* codes,
                               float* norms, int64_t out_stride, void* stream) {
+  TQ_TRACE("tq_quant_polar");
   int rc = check_quant_args("tq_quant_polar", h, TQ_POLAR, x, dtype, N, x_stride, codes, norms, out_stride);
   if (rc) return rc;
   if (N == 0) return clear_error();
@@ -725,6 +735,7 @@ extern "C" int tq_quant_polar(tq_handle h, const void* x, int dtype, int64_t N, 
 
 extern "C" int tq_dequant_polar(tq_handle h, const uint32_t* codes, const float* norms, int64_t N, void* out,
                                 int out_dtype, void* stream) {
+  TQ_TRACE("tq_dequant_polar");
   if (!h) return set_error(TQ_EINVAL, "tq_dequant_polar: NULL handle");
   if (h->variant != TQ_POLAR) return set_error(TQ_EINVAL, "tq_dequant_polar: need a TQ_POLAR handle");
   if (N < 0) return set_error(TQ_EINVAL, "tq_dequant_polar: N < 0");
@@ -742,6 +753,7 @@ extern "C" int tq_dequant_polar(tq_handle h, const uint32_t* codes, const float*
 extern "C" int tq_quant_gather(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                                const int32_t* channels, uint32_t* codes, uint32_t* signs, float* norms,
                                float* rnorms, int64_t out_stride, void* stream) {
+  TQ_TRACE("tq_quant_gather");
   if (!h) return set_error(TQ_EINVAL, "tq_quant_gather: NULL handle");
   if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "tq_quant_gather: a TQ_POLAR handle");
   if (N < 0) return set_error(TQ_EINVAL, "tq_quant_gather: N < 0");
@@ -777,6 +789,7 @@ extern "C" int tq_quant_gather_groups(const tq_handle* h, int ngroups, const voi
                                       int64_t x_stride, const int32_t* channels, uint32_t* const* codes,
                                       uint32_t* const* signs, float* const* norms, float* const* rnorms,
                                       int64_t out_stride, void* stream) {
+  TQ_TRACE("tq_quant_gather_groups");
   const char* fn = "tq_quant_gather_groups";
   if (!h || ngroups < 1 || ngroups > 2) return set_error(TQ_EINVAL, "%s: need 1 or 2 groups", fn);
   if (N < 0 || N >= 65536) return set_error(TQ_EINVAL, "%s: N = %lld (need 0 <= N < 65536)", fn, (long long)N);
@@ -824,6 +837,7 @@ extern "C" int tq_attn_logits(const tq_handle* hk, int ngroups, const int32_t* c
                               const uint32_t* const* kcodes, const uint32_t* const* ksigns,
                               const float* const* knorms, const float* const* krnorms, float scale, float* logits,
                               void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_attn_logits");
   if (!hk || ngroups < 1 || ngroups > 2) return set_error(TQ_EINVAL, "tq_attn_logits: need 1 or 2 groups");
   int dsum = 0;
   for (int g = 0; g < ngroups; ++g) {

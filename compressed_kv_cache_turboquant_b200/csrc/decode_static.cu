@@ -58,6 +58,7 @@ extern "C" int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, 
                                      const float* knorms, const float* krnorms,
                                      const uint32_t* vcodes, const float* vnorms, float scale,
                                      float* out, void* stream) {
+  TQ_TRACE("tq_attn_decode_static");
   if (!hk || !hv) return set_error(TQ_EINVAL, "tq_attn_decode_static: NULL handle");
   if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)
     return set_error(TQ_EINVAL,

@@ -718,7 +718,7 @@ __global__ void __launch_bounds__(128) decode_tc_qtile_kernel(const float* qrot,
 
 bool decode_tc_supported(const tq_ctx* hk, const tq_ctx* hv, int Hq, int Hkv, int64_t kv_stride, int rn16) {
   return decode_mma_supported(hk, hv, Hq, Hkv, kv_stride) && hk->dev.ktab != nullptr && (!rn16 || kv_stride % 8 == 0) &&
-         !hk->debug_fixed_tables && !hk->legacy_mma;
+         !hk->debug_fixed_tables && hk->tc_attn;
 }
 
 int decode_tc_grid(int B, int Hkv, int64_t T, int sm_count) {

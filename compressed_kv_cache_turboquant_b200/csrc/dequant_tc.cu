@@ -4,28 +4,24 @@
 // (ttakun.com/news/45354, "KV缓存52GB瞬间爆内存？TurboQuant随机旋转+标量量化…")
 //
 // As a GEMM: X_hat[128 x d] = C[128 x d] . Pi (C = centroid values of a tile of
-// 128 vectors).  fp16 operands in two pieces each, both scaled by 2^6 and with
-// the low pieces true-valued (subnormal where small: their absolute rounding,
-// 2^-25 in the scaled units, is what matters), summed in one fp32 accumulator:
-//   2^6 C  = C_hi + C_lo,   2^6 Pi = P_hi + P_lo
-//   acc = C_hi . P_hi + C_lo . P_hi + C_hi . P_lo,   x_hat = n 2^-12 acc
-// (the dropped C_lo . P_lo term is ~2^-22 of the result).
+// 128 vectors).  fp16 operands in two pieces each, with the low pieces scaled
+// by 2^11 so they stay normal:
+//   C  = C_hi + 2^-11 C_lo',   Pi = P_hi + 2^-11 P_lo'
+//   acc0 = C_hi . P_hi,  acc1 = C_hi . P_lo' + C_lo' . P_hi
+//   x_hat = n * (acc0 + 2^-11 acc1)        (relative error ~2^-21)
 // Persistent CTA per SM; warps:
-//   0      TMEM allocation and the single-thread MMA issuer; A is read from
-//          tensor memory, B (the two pieces of Pi^T) from shared memory
-//   1..4   decoders: one thread per vector (its TMEM lane) unpacks its codes,
-//          looks the two fp16 pieces up in a 16-entry table and writes them
-//          into the vector's lane of the A stage (two stages)
-//   5..8   epilogue, one warp per TMEM lane quarter: one thread per vector
-//          reads the accumulator chunk by chunk, scales by n 2^-12, stages the
-//          warp's 32 rows x 128 B chunk in 128B-swizzled shared memory (eight
-//          boxes per warp: two tiles of chunks in flight) and writes it with
-//          one TMA tensor store: whole 128-byte lines
-// Tensor memory (4 d columns): A stage s at s d (hi d/2 columns, lo d/2), the
-// accumulator of buffer s at 2 d + s d.
+//   0      TMEM allocation and the single-thread MMA issuer
+//   1..4   decoders: one thread per vector unpacks its codes, looks the two
+//          fp16 pieces up in a 16-entry table and writes them into the
+//          128B-swizzled K-major A tiles (double-buffered)
+//   5..12  epilogue, two warps per TMEM lane quarter taking half of the column
+//          chunks each: one thread per vector reads both accumulators from TMEM,
+//          combines and scales by n; each warp stages its 32 rows x 128 B
+//          column chunk in 128B-swizzled shared memory (two buffers) and
+//          writes it with one TMA tensor store, so global writes are whole
+//          128-byte lines instead of 32 scattered 16-byte pieces per store
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "sm100_common.cuh"
@@ -37,29 +33,29 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 288;  // 9 warps: at most 3 per SM sub-partition, so ~168 registers a thread
+constexpr int kThreads = 416;  // 13 warps
 
 template <int D>
 struct DqShape {
   static constexpr int kSlabs = D / 64;
+  static constexpr int kSlabBytesA = kTileM * 128;
+  static constexpr int kABytes = kSlabs * kSlabBytesA;  // one piece of one A tile
   static constexpr int kSlabBytesB = D * 128;
   static constexpr int kBBytes = kSlabs * kSlabBytesB;  // one piece of Pi (as B, K-major)
-  static constexpr int kTmemCols = 4 * D;               // 2 A stages + 2 accumulators
+  static constexpr int kStages = 2;
+  static constexpr int kTmemCols = (4 * D <= 256) ? 256 : 512;  // 2 buffers x 2 accumulators
   static constexpr int kMiscBytes = 2048;
-  static constexpr int kStageOut = 32 * 128;            // one output box: 32 rows x 128 B
-  static constexpr int kOutBoxes = 8;                   // boxes per epilogue warp
-  static constexpr int kOutBytes = 4 * kOutBoxes * kStageOut;
-  static constexpr int kSmemBytes = 2 * kBBytes + kOutBytes + kMiscBytes + 1024;
+  static constexpr int kStageOut = 32 * 128;  // one warp's output chunk: 32 rows x 128 B
+  static constexpr int kOutBytes = 8 * kStageOut;  // one staging box per epilogue warp
+  static constexpr int kSmemBytes = 2 * kBBytes + kStages * 2 * kABytes + kOutBytes + kMiscBytes + 1024;
 };
-constexpr float kScale = 64.f;                // 2^6 on both operands
-constexpr float kInvScale2 = 1.f / 4096.f;    // 2^-12
 
 struct DqArgs {
   const uint32_t* codes;
   const float* norms;
   int64_t N;
-  const uint8_t* pit_f16;  // 2 pieces x [slab][row i][128 B swizzled] of 2^6 Pi^T (B[i][j] = Pi[j][i])
-  const float* cent;       // [2^b] centroids
+  const uint8_t* pit_f16;  // 2 pieces x [slab][row i][128 B swizzled] of Pi^T (B[i][j] = Pi[j][i])
+  const uint32_t* lut;     // [16]: fp16 hi | fp16 lo' << 16 of c_k
   int out_bf16;
   int* status;
   // PolarQuant codes (BM = 0): words per row, bits of level 1 / levels >= 2,
@@ -83,7 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* b_s = smem;                      // [2 pieces][kBBytes]
-  uint8_t* o_s = smem + 2 * S::kBBytes;     // [4 warps][kOutBoxes][kStageOut], 1024-aligned
+  uint8_t* a_s = smem + 2 * S::kBBytes;     // [stage][2 pieces][kABytes]
+  uint8_t* o_s = a_s + S::kStages * 2 * S::kABytes;  // [8 warps][kStageOut], 1024-aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(o_s + S::kOutBytes);
   uint64_t* a_full = bars;              // [2]  decoders -> MMA (count 128)
   uint64_t* a_empty = bars + 2;         // [2]  MMA commit -> decoders
@@ -92,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
   uint64_t* b_bar = bars + 8;
   uint64_t* done_bar = bars + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  uint32_t* lut_s = tmem_slot + 4;      // [16]: fp16 hi | fp16 lo << 16 of 2^6 c_k
+  uint32_t* lut_s = tmem_slot + 4;      // [16]
   float* pcs = reinterpret_cast<float*>(lut_s + 16);  // [2][8][16] (PolarQuant)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,18 +100,13 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       mbar_init(&a_full[s], 128);
       mbar_init(&a_empty[s], 1);
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);
+      mbar_init(&acc_empty[s], 8);
     }
     mbar_init(b_bar, 1);
     mbar_init(done_bar, 1);
     fence_mbar_init();
   }
-  if (BM > 0 && threadIdx.x < (1 << BM)) {
-    const float v = kScale * a.cent[threadIdx.x];
-    const __half hi = __float2half_rn(v);
-    const __half lo = __float2half_rn(v - __half2float(hi));
-    lut_s[threadIdx.x] = (uint32_t)__half_as_ushort(hi) | ((uint32_t)__half_as_ushort(lo) << 16);
-  }
+  if (threadIdx.x < 16) lut_s[threadIdx.x] = a.lut[threadIdx.x];
   if (BM == 0)
     for (int e = threadIdx.x; e < 256; e += blockDim.x) pcs[e] = a.polar_cs[e];
   if (warp == 0) tmem_alloc(tmem_slot, S::kTmemCols);
@@ -129,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       bulk_load(b_s, a.pit_f16, S::kBBytes, b_bar);
       bulk_load(b_s + S::kBBytes, a.pit_f16 + S::kBBytes, S::kBBytes, b_bar);
       constexpr uint32_t idesc = idesc_f16(kTileM, D, false);
-      const uint32_t p_hi = smem_u32(b_s), p_lo = p_hi + S::kBBytes;
+      const uint32_t b_addr = smem_u32(b_s), a_addr = smem_u32(a_s);
       bool ok = mbar_wait(b_bar, 0);
       int i = 0;
       for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++i) {
@@ -140,16 +132,19 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        const uint32_t acc = tmem_base + (uint32_t)(2 * D + s * D);
-        const uint32_t a_hi = tmem_base + (uint32_t)(s * D), a_lo = a_hi + D / 2;
+        const uint32_t acc0 = tmem_base + (uint32_t)(s * 2 * D), acc1 = acc0 + D;
+        const uint32_t a_hi = a_addr + s * 2 * S::kABytes, a_lo = a_hi + S::kABytes;
+        const uint32_t p_hi = b_addr, p_lo = b_addr + S::kBBytes;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t kb = (ks >> 2) * S::kSlabBytesB + (ks & 3) * 32;
-          const uint64_t bh = sw128_kmajor_desc(p_hi + kb), bl = sw128_kmajor_desc(p_lo + kb);
-          mma_f16_ta(acc, a_hi + 8 * ks, bh, idesc, ks ? 1u : 0u);
-          mma_f16_ta(acc, a_lo + 8 * ks, bh, idesc, 1u);
-          mma_f16_ta(acc, a_hi + 8 * ks, bl, idesc, 1u);
-        }
+        for (int sl = 0; sl < S::kSlabs; ++sl)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint32_t ka = sl * S::kSlabBytesA + k4 * 32, kb = sl * S::kSlabBytesB + k4 * 32;
+            const uint32_t first = (sl | k4) != 0 ? 1u : 0u;
+            mma_f16(acc0, sw128_kmajor_desc(a_hi + ka), sw128_kmajor_desc(p_hi + kb), idesc, first);
+            mma_f16(acc1, sw128_kmajor_desc(a_hi + ka), sw128_kmajor_desc(p_lo + kb), idesc, first);
+            mma_f16(acc1, sw128_kmajor_desc(a_lo + ka), sw128_kmajor_desc(p_hi + kb), idesc, 1u);
+          }
         mma_commit(&a_empty[s]);
         mma_commit(&acc_full[s]);
       }
@@ -157,10 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       mma_commit(done_bar);
     }
   } else if (warp <= 4) {
-    // decoders: thread r (TMEM lane r, warp % 4 = lane quarter) decodes vector
-    // r of the tile
-    const int r = (warp & 3) * 32 + lane;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    // decoders: thread r of the 128 decodes vector r of the tile; the codes of
+    // the next tile are loaded while this one is decoded
+    const int r = threadIdx.x - 32;
     auto load_codes = [&](int64_t tile, uint32_t (&w)[W]) {
       const int64_t vec = tile * kTileM + r;
       if (BM == 0) {
@@ -183,20 +177,22 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
         for (int q = 0; q < W; ++q) w[q] = 0u;
       }
     };
-    // the next tile's codes are loaded as soon as this tile's are decoded, so
-    // the loads are in flight while the decoder waits for its next A stage
-    uint32_t w[W];
-    load_codes(blockIdx.x, w);
+    uint32_t w_next[W];
+    load_codes(blockIdx.x, w_next);
     int i = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       const int s = i & 1;
       const uint32_t u = (uint32_t)(i >> 1);
+      uint32_t w[W];
+#pragma unroll
+      for (int q = 0; q < W; ++q) w[q] = w_next[q];
+      load_codes(tile + gridDim.x, w_next);
       if (!mbar_wait_warp(&a_empty[s], (u & 1u) ^ 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
-      tc_fence_after();
-      const uint32_t t_hi = tmem_base + lane_base + (uint32_t)(s * D), t_lo = t_hi + D / 2;
+      uint8_t* hi_tile = a_s + s * 2 * S::kABytes;
+      uint8_t* lo_tile = hi_tile + S::kABytes;
       if constexpr (BM == 0) {
         // the unit angle tree run back down: radii of the top levels, then one
         // 32-coordinate group at a time
@@ -233,68 +229,78 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
               rr[2 * i + 1] = r * sinl[lev * 16 + c];
             }
           }
+          float y[32];
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t hv[8], lv[8];
+          for (int p = 0; p < 16; ++p) {
+            const uint32_t c = polar_code(w, 0, 16 * g + p, a.b1);
+            y[2 * p] = rr[p] * cosl[16 + c];
+            y[2 * p + 1] = rr[p] * sinl[16 + c];
+          }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int p = 8 * hf + e;
-              const uint32_t c = polar_code(w, 0, 16 * g + p, a.b1);
-              const float v0 = kScale * rr[p] * cosl[16 + c], v1 = kScale * rr[p] * sinl[16 + c];
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int kglob = 32 * g + 8 * c4;
+            const int slab = kglob / 64, chunk = (kglob % 64) / 8;
+            uint32_t hv[4], lv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float v0 = y[8 * c4 + 2 * e], v1 = y[8 * c4 + 2 * e + 1];
               const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
-              const __half l0 = __float2half_rn(v0 - __half2float(h0));
-              const __half l1 = __float2half_rn(v1 - __half2float(h1));
+              const __half l0 = __float2half_rn((v0 - __half2float(h0)) * 2048.f);
+              const __half l1 = __float2half_rn((v1 - __half2float(h1)) * 2048.f);
               hv[e] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
               lv[e] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
             }
-            tmem_st8(t_hi + 16 * g + 8 * hf, hv);
-            tmem_st8(t_lo + 16 * g + 8 * hf, lv);
+            const int off = slab * S::kSlabBytesA + r * 128 + ((chunk ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
           }
         }
       } else {
 #pragma unroll
-        for (int g = 0; g < D / 32; ++g) {
-          uint32_t idx[32];
-          const uint32_t* p = w + g * BM;
+      for (int g = 0; g < D / 32; ++g) {
+        uint32_t idx[32];
+        const uint32_t* p = w + g * BM;
 #pragma unroll
-          for (int ii = 0; ii < 32; ++ii) {
-            if constexpr (BM == 1) idx[ii] = (p[0] >> ii) & 1u;
-            else if constexpr (BM == 2) idx[ii] = (p[ii >> 4] >> (2 * (ii & 15))) & 3u;
-            else if constexpr (BM == 4) idx[ii] = (p[ii >> 3] >> (4 * (ii & 7))) & 15u;
+        for (int ii = 0; ii < 32; ++ii) {
+          if constexpr (BM == 1) idx[ii] = (p[0] >> ii) & 1u;
+          else if constexpr (BM == 2) idx[ii] = (p[ii >> 4] >> (2 * (ii & 15))) & 3u;
+          else if constexpr (BM == 4) idx[ii] = (p[ii >> 3] >> (4 * (ii & 7))) & 15u;
+          else {
+            if (ii < 24) idx[ii] = (p[ii >> 3] >> (4 * (ii & 7))) & 7u;
             else {
-              if (ii < 24) idx[ii] = (p[ii >> 3] >> (4 * (ii & 7))) & 7u;
-              else {
-                const int sh = 4 * (ii - 24) + 3;
-                idx[ii] = ((p[0] >> sh) & 1u) | (((p[1] >> sh) & 1u) << 1) | (((p[2] >> sh) & 1u) << 2);
-              }
+              const int sh = 4 * (ii - 24) + 3;
+              idx[ii] = ((p[0] >> sh) & 1u) | (((p[1] >> sh) & 1u) << 1) | (((p[2] >> sh) & 1u) << 2);
             }
-          }
-          // column e of the group holds coordinates 32 g + 2 e, 32 g + 2 e + 1
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t hv[8], lv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t x0 = lut_s[idx[16 * hf + 2 * e]], x1 = lut_s[idx[16 * hf + 2 * e + 1]];
-              hv[e] = __byte_perm(x0, x1, 0x5410);
-              lv[e] = __byte_perm(x0, x1, 0x7632);
-            }
-            tmem_st8(t_hi + 16 * g + 8 * hf, hv);
-            tmem_st8(t_lo + 16 * g + 8 * hf, lv);
           }
         }
+        // 4 chunks of 8 coordinates: k = 32 g + 8 c4 + e
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int kglob = 32 * g + 8 * c4;
+          const int slab = kglob / 64, chunk = (kglob % 64) / 8;
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t x0 = lut_s[idx[8 * c4 + 2 * e]], x1 = lut_s[idx[8 * c4 + 2 * e + 1]];
+            hv[e] = __byte_perm(x0, x1, 0x5410);
+            lv[e] = __byte_perm(x0, x1, 0x7632);
+          }
+          const int off = slab * S::kSlabBytesA + r * 128 + ((chunk ^ (r & 7)) * 16);
+          *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
       }
-      load_codes(tile + gridDim.x, w);
-      // the stores must be complete before the MMA thread is told
-      tmem_wait_st();
-      tc_fence_before();
+      }
+      // generic-proxy writes must be visible to the tensor core's async proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&a_full[s]);
     }
   } else {
-    // epilogue: warp % 4 selects the TMEM lane quarter; every chunk of it
+    // epilogue: warp % 4 selects the TMEM lane quarter, (warp - 5) / 4 the half of the chunks
     const int quarter = warp & 3;
+    const int part = (warp - 5) >> 2;
     const int r = quarter * 32 + lane;
-    uint8_t* boxes = o_s + (warp - 5) * S::kOutBoxes * S::kStageOut;
+    uint8_t* buf = o_s + (warp - 5) * S::kStageOut;
     constexpr int kCols = 32;  // fp32 columns per 128-byte chunk (bf16: 64)
     int nst = 0;
     int i = 0;
@@ -303,38 +309,42 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
       const uint32_t u = (uint32_t)(i >> 1);
       const int64_t vec = tile * kTileM + r;
       const int64_t row0 = tile * kTileM + quarter * 32;
-      const float n = ((vec < a.N) ? a.norms[vec] : 0.f) * kInvScale2;  // issued before the wait
+      const float n = (vec < a.N) ? a.norms[vec] : 0.f;  // issued before the wait
       if (!mbar_wait_warp(&acc_full[s], u & 1u)) {
         atomicOr(a.status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(2 * D + s * D);
+      const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 2 * D);
       const int nchunks = a.out_bf16 ? D / 64 : D / 32;
-      for (int c = 0; c < nchunks; ++c, ++nst) {
-        uint8_t* buf = boxes + (nst % S::kOutBoxes) * S::kStageOut;
-        // the store that last used this box must have read it
-        if (lane == 0) bulk_wait_read<S::kOutBoxes - 1>();
+      const int c_lo = part * (nchunks / 2), c_hi = (nchunks == 1) ? (part == 0 ? 1 : 0) : c_lo + nchunks / 2;
+      for (int c = c_lo; c < c_hi; ++c, ++nst) {
+        // the previous store from this warp's buffer must have read it
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
         uint32_t pk[32];
         if (a.out_bf16) {
 #pragma unroll
           for (int hlf = 0; hlf < 2; ++hlf) {
-            float v[32];
-            tmem_ld32(t0 + c * 64 + hlf * 32, v);
+            float v0[32], v1[32];
+            tmem_ld32(t0 + c * 64 + hlf * 32, v0);
+            tmem_ld32(t0 + D + c * 64 + hlf * 32, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(n * v[2 * e], n * v[2 * e + 1]);
+              const float y0 = n * fmaf(v1[2 * e], 4.8828125e-4f, v0[2 * e]);
+              const float y1 = n * fmaf(v1[2 * e + 1], 4.8828125e-4f, v0[2 * e + 1]);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
               pk[16 * hlf + e] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
         } else {
-          float v[32];
-          tmem_ld32(t0 + c * kCols, v);
+          float v0[32], v1[32];
+          tmem_ld32(t0 + c * kCols, v0);
+          tmem_ld32(t0 + D + c * kCols, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(n * v[e]);
+          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
         }
         // row `lane` of the 128B-swizzled box: 16-byte unit j lands at j ^ (lane & 7)
 #pragma unroll
@@ -345,10 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
         __syncwarp();
         if (lane == 0 && row0 < a.N) {
           tma_store_2d(&omap, buf, c * (a.out_bf16 ? 64 : kCols), (int)row0);
+          bulk_commit();
         }
-        // one bulk group per chunk (empty past the end), so the count of
-        // groups in flight matches the boxes in use
-        if (lane == 0) bulk_commit();
       }
       tc_fence_before();
       __syncwarp();
@@ -361,7 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
   if (warp == 0) {
     if (!mbar_wait(done_bar, 0) && lane == 0) atomicOr(a.status, kStatusTimeout);
     __syncwarp();
-    tc_fence_after();
     tmem_dealloc(tmem_base, S::kTmemCols);
   }
 }
@@ -385,7 +392,7 @@ int launch_dq(const tq_ctx* h, const uint32_t* codes, const float* norms, int64_
     return (int)cudaErrorInvalidValue;
   auto kern = dequant_tc_kernel<D, BM>;
   if (int e = ensure_dyn_smem((const void*)kern, S::kSmemBytes)) return e;
-  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.centroids, out_bf16, h->dev.status};
+  DqArgs a{codes, norms, N, h->dev.pit_f16, h->dev.lut_dq, out_bf16, h->dev.status};
   if (BM == 0) {
     a.b1 = h->polar_b1;
     a.bh = h->polar_bh;

@@ -128,6 +128,7 @@ struct Law {
 using namespace tqi;
 
 extern "C" int tq_make_codebook(int b, int d, double* centroids, double* thresholds) {
+  TQ_TRACE("tq_make_codebook");
   if (!centroids) return set_error(TQ_EINVAL, "tq_make_codebook: centroids is NULL");
   if (b < 1 || b > 4 || d < 3 || d > TQ_MAX_DIM)
     return set_error(TQ_EUNSUPPORTED, "tq_make_codebook: need 1 <= b <= 4 and 3 <= d <= %d",
@@ -182,6 +183,7 @@ extern "C" int tq_make_codebook(int b, int d, double* centroids, double* thresho
 // The sign fix makes Pi Haar distributed (R gets a positive diagonal).
 // ---------------------------------------------------------------------------
 extern "C" int tq_make_rotation(int d, const double* G, double* Pi) {
+  TQ_TRACE("tq_make_rotation");
   if (!G || !Pi) return set_error(TQ_EINVAL, "tq_make_rotation: NULL pointer");
   if (d < 1 || d > TQ_MAX_DIM)
     return set_error(TQ_EUNSUPPORTED, "tq_make_rotation: need 1 <= d <= %d", TQ_MAX_DIM);
@@ -270,6 +272,7 @@ struct AngleLaw {
 }  // namespace tqi
 
 extern "C" int tq_polar_codebook(int b, int level, double* centroids, double* thresholds) {
+  TQ_TRACE("tq_polar_codebook");
   if (!centroids) return set_error(TQ_EINVAL, "tq_polar_codebook: NULL centroids");
   if (b < 1 || b > 8 || level < 1 || level > 12)
     return set_error(TQ_EUNSUPPORTED, "tq_polar_codebook: b = %d, level = %d", b, level);

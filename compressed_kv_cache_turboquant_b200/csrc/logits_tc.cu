@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(128) logits_tc_qtile_kernel(const float* qrot0
 }  // namespace
 
 bool logits_tc_supported(const tq_ctx* const* hk, int ngroups, int64_t kv_stride) {
-  return logits_mma_supported(hk, ngroups, kv_stride) && !hk[0]->debug_fixed_tables && !hk[0]->legacy_mma;
+  return logits_mma_supported(hk, ngroups, kv_stride) && !hk[0]->debug_fixed_tables && hk[0]->tc_attn;
 }
 
 size_t logits_tc_workspace(int B, int Hkv) {

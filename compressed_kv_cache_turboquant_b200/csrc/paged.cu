@@ -18,6 +18,7 @@ using namespace tqi;
 extern "C" int tq_quant_paged(tq_handle h, const void* x, int dtype, int64_t N, int64_t x_stride,
                               const int32_t* channels, const int64_t* slots, uint32_t* codes, uint32_t* signs,
                               float* norms, void* rnorms, int rn_dtype, void* stream) {
+  TQ_TRACE("tq_quant_paged");
   const char* fn = "tq_quant_paged";
   if (!h) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
   if (h->variant == TQ_POLAR) return set_error(TQ_EINVAL, "%s: a TQ_POLAR handle", fn);
@@ -45,6 +46,7 @@ extern "C" int tq_attn_decode_paged(tq_handle hk, tq_handle hv, const void* q, i
                                     const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
                                     const void* krnorms, int rn_dtype, const uint32_t* vcodes, const float* vnorms,
                                     float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_attn_decode_paged");
   const char* fn = "tq_attn_decode_paged";
   if (!hk || !hv) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
   if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)

@@ -585,6 +585,7 @@ extern "C" int tq_attn_prefill(tq_handle hk, tq_handle hv, const void* q, int q_
                                int64_t T, int64_t kv_stride, const uint32_t* kcodes, const uint32_t* ksigns,
                                const float* knorms, const float* krnorms, const uint32_t* vcodes, const float* vnorms,
                                float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_attn_prefill");
   const char* fn = "tq_attn_prefill";
   if (!hk || !hv) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
   if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)

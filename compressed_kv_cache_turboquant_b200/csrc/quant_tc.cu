@@ -13,9 +13,9 @@
 //   warp 1      TMEM allocation and the single-thread MMA issuer:
 //               Y[128 x d] = X[128 x d] . (Pi_hi + Pi_mid + Pi_lo)^T, three
 //               bf16 passes accumulated in fp32 in TMEM (double-buffered)
-//   warps 2-13  epilogue: three sets of four warps (one per TMEM lane
+//   warps 2-17  epilogue: four sets of four warps (one per TMEM lane
 //               quarter) take the tiles in turn, each set with its own
-//               accumulator buffer, so three tiles are in flight; one thread
+//               accumulator buffer, so four tiles are in flight; one thread
 //               per vector (TMEM lane) reads the vector's columns twice: once
 //               for n = ||y|| (= ||x||, Pi orthogonal), once for the cell of
 //               every coordinate against n * t_k, packing and stores.  Even
@@ -40,7 +40,7 @@ using namespace sm100;
 
 constexpr int kPieces = 3;
 constexpr int kTileM = 128;
-constexpr int kSets = 3;                  // epilogue warp sets = accumulator buffers
+constexpr int kSets = 4;                  // epilogue warp sets = accumulator buffers
 // warps: TMA producer, MMA issuer, kSets sets of 4 epilogue warps
 template <int D>
 constexpr int threads_for() { return 32 * (2 + 4 * kSets); }
@@ -299,13 +299,6 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     constexpr int H = 1 << (BM - 1);
-    // positive thresholds t_m (m = 1 .. H - 1) and the constants of the FMA-pipe count
-    float tp[8], Cf[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      tp[m] = (m >= 1 && m < H) ? thr_s[H - 1 + m] : 0.f;
-      Cf[m] = (m >= 1 && m < H) ? 1.f - 4294967296.f * tp[m] : -1.f;
-    }
     const uint32_t lb = (uint32_t)(quarter * 32) << 16;
     int i = set;
     for (int64_t tile = blockIdx.x + (int64_t)set * gridDim.x; tile < ntiles; tile += (int64_t)kSets * gridDim.x,
@@ -329,12 +322,15 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
         for (int c = 0; c < 32; ++c) ss = fmaf(v[c], v[c], ss);
       }
       const float n = sqrtf(ss);
-      // a zero vector has y = 0, which lies below every positive threshold
+      // positive thresholds t_m (m = 1 .. H - 1) scaled by n, and the
+      // constants of the FMA-pipe count; a zero vector has y = 0, which lies
+      // below every positive threshold
       float P[8], Cz[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        P[m] = n > 0.f ? n * tp[m] : INFINITY;
-        Cz[m] = n > 0.f ? Cf[m] : -1.f;
+        const float tm = (m >= 1 && m < H) ? thr_s[H - 1 + m] : 0.f;
+        P[m] = n > 0.f ? n * tm : INFINITY;
+        Cz[m] = (n > 0.f && m >= 1 && m < H) ? 1.f - 4294967296.f * tm : -1.f;
       }
       const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
       const int64_t vec = tile * kTileM + row;

@@ -84,6 +84,7 @@ extern "C" int tq_attn_decode_partial(tq_handle hk, tq_handle hv, const void* q,
                                       const float* knorms, const float* krnorms, const uint32_t* vcodes,
                                       const float* vnorms, float scale, float* partial, void* workspace,
                                       size_t ws_bytes, void* stream) {
+  TQ_TRACE("tq_attn_decode_partial");
   const char* fn = "tq_attn_decode_partial";
   if (!hk || !hv) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
   if (hk->variant != TQ_PROD || hv->variant != TQ_MSE)
@@ -117,6 +118,7 @@ extern "C" int tq_attn_decode_partial(tq_handle hk, tq_handle hv, const void* q,
 }
 
 extern "C" int tq_attn_merge(tq_handle hv, const float* partials, int R, int64_t rows, float* out, void* stream) {
+  TQ_TRACE("tq_attn_merge");
   const char* fn = "tq_attn_merge";
   if (!hv) return set_error(TQ_EINVAL, "%s: NULL handle", fn);
   if (hv->variant != TQ_MSE) return set_error(TQ_EINVAL, "%s: need the TQ_MSE value handle", fn);
@@ -132,6 +134,7 @@ extern "C" int tq_attn_merge(tq_handle hv, const float* partials, int R, int64_t
 
 extern "C" int tq_topk_merge(const float* val, const int32_t* idx, int R, int64_t nq, int k, const int64_t* offsets,
                              int32_t* out_idx, float* out_val, void* stream) {
+  TQ_TRACE("tq_topk_merge");
   const char* fn = "tq_topk_merge";
   if (R < 1 || R > TQ_MAX_SHARDS) return set_error(TQ_EINVAL, "%s: R = %d (need 1..%d)", fn, R, TQ_MAX_SHARDS);
   if (nq < 0 || k < 1 || k > TQ_MAX_TOPK) return set_error(TQ_EINVAL, "%s: nq = %lld, k = %d", fn, (long long)nq, k);

@@ -1,10 +1,24 @@
 // Internal declarations shared by the host API and the kernels.
 #pragma once
 
+#include <nvtx3/nvToolsExt.h>
 #include <cstddef>
 #include <cstdint>
 
 #include "tq.h"
+
+namespace tqi {
+// An NVTX range named after the C entry point for the duration of the call
+// (host side: argument checks and launches), so a profiler's timeline shows
+// the library's calls; free when no tool is attached.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+}  // namespace tqi
+#define TQ_TRACE(name) ::tqi::TraceRange tq_trace_range_(name)
 
 namespace tqi {
 
@@ -105,10 +119,10 @@ struct tq_ctx {
   float polar_tan2[8][3] = {};
   float* polar_cs = nullptr;  // device [2][8 levels][16]: cos, sin of centroid k of level l (level 1 at l = 1)
   bool debug_fixed_tables = false;  // TQ_DEBUG_DYN_BASE given: take the fixed-address kernels anyway
-  // TQ_LEGACY_MMA_SYNC=1 at creation: decode and split-cache logits take the
-  // mma.sync kernels instead of the tcgen05 ones (both stay covered by the
-  // parity tests)
-  bool legacy_mma = false;
+  // TQ_TCGEN05_ATTN=1 at creation: dense decode and split-cache logits take
+  // the tcgen05 kernels instead of the mma.sync ones (both are covered by the
+  // parity tests; the mma.sync kernels are faster today)
+  bool tc_attn = false;
   // 3-bit codebook as fp16 byte tables (register decoding): lo bytes of c0-3,
   // c4-7, hi bytes of c0-3, c4-7 (zero unless b = 3 mse bits)
   uint32_t host_ktab[4] = {0, 0, 0, 0};

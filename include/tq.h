@@ -150,9 +150,9 @@ TQ_API int tq_make_rotation(int d, const double* G, double* Pi);
  *   TQ_FUSED_REGISTER_LOADS=1  quantization at d <= 256 takes the kernel whose
  *                        producer threads load x themselves (the one a channel
  *                        gather always takes) instead of the TMA-staged one
- *   TQ_LEGACY_MMA_SYNC=1  tq_attn_decode on a dense cache and the two-group
- *                        tq_attn_logits take the mma.sync kernels instead of
- *                        the tcgen05 ones (a paged cache always takes the
+ *   TQ_TCGEN05_ATTN=1    tq_attn_decode on a dense cache and the two-group
+ *                        tq_attn_logits take the tcgen05 kernels instead of
+ *                        the mma.sync ones (a paged cache always takes the
  *                        mma.sync decode kernel)
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM, TQ_ECUDA.
  */

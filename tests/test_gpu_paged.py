@@ -90,8 +90,12 @@ def _paginate(c, B, Hkv, T, page, seed, spare=3):
 
 
 @pytest.mark.parametrize("page,rn16,Hq", [(16, False, 32), (64, True, 32), (256, False, 32), (64, True, 16)])
-def test_paged_decode_matches_oracle(page, rn16, Hq):
-    # Hq = 32 takes the tensor-core decode, Hq = 16 (2 q-heads per kv-head) the general kernel
+def test_paged_decode_matches_oracle(monkeypatch, page, rn16, Hq):
+    # Hq = 32 takes the mma.sync decode (the paged kernel), Hq = 16 (2 q-heads
+    # per kv-head) the general kernel.  The handles take the mma.sync kernel
+    # for dense caches as well, so the paged result can be compared with the
+    # dense one of the same arithmetic (only the addressing differs).
+    monkeypatch.delenv("TQ_TCGEN05_ATTN", raising=False)
     B, Hkv, T, d = 2, 8, 9000, 128
     sample = [(0, 2), (1, 5)]
     hk, hv, c, q64, refs = decode_cache(B, Hq, Hkv, T, d, sample, seed=9)

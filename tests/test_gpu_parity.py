@@ -358,16 +358,16 @@ def _decode_case(B, Hq, Hkv, T, d, sample, seed=0, stride_extra=0):
 
 
 # The dense 4-heads-per-kv-head decode and the two-group logits run on the
-# tcgen05 kernels; handles created with TQ_LEGACY_MMA_SYNC=1 take the mma.sync
+# mma.sync kernels; handles created with TQ_TCGEN05_ATTN=1 take the tcgen05
 # kernels instead.
 DECODE_KERNELS = ["tcgen05", "mma_sync"]
 
 
 def _pick_decode_kernel(monkeypatch, kernel):
-    if kernel == "mma_sync":
-        monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
+    if kernel == "tcgen05":
+        monkeypatch.setenv("TQ_TCGEN05_ATTN", "1")
     else:
-        monkeypatch.delenv("TQ_LEGACY_MMA_SYNC", raising=False)
+        monkeypatch.delenv("TQ_TCGEN05_ATTN", raising=False)
 
 
 @pytest.mark.parametrize("kernel", DECODE_KERNELS)
@@ -392,10 +392,11 @@ def test_decode_one_kv_head_long_context(monkeypatch, kernel):
     _decode_case(B=1, Hq=4, Hkv=1, T=70001, d=128, sample=[(0, 0)], seed=2)
 
 
-def test_decode_tc_short_contexts():
+def test_decode_tc_short_contexts(monkeypatch):
     """Contexts of one partial block, of a block and one token, and of many
     (batch, kv-head) pairs per CTA: segment starts and ends inside the
     tcgen05 kernel's pipeline, records of single-block segments."""
+    _pick_decode_kernel(monkeypatch, "tcgen05")
     _decode_case(B=3, Hq=8, Hkv=2, T=37, d=128, sample=[(0, 0), (2, 1)], seed=6, stride_extra=3)
     _decode_case(B=2, Hq=4, Hkv=1, T=129, d=128, sample=[(1, 0)], seed=7, stride_extra=3)
     _decode_case(B=64, Hq=16, Hkv=4, T=300, d=128, sample=[(0, 0), (31, 2), (63, 3)], seed=8)
@@ -412,7 +413,6 @@ def test_decode_runtime_table_addresses(monkeypatch):
     """The decode kernel instance that adds its table addresses at run time (taken when the
     dynamic shared window is not where the library expects it) agrees just the same."""
     monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
-    monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
     _decode_case(B=2, Hq=8, Hkv=2, T=1531, d=128, sample=[(0, 1), (1, 0)], seed=5, stride_extra=5)
 
 
@@ -566,7 +566,6 @@ def test_split_group_logits_ragged_tensor_core(monkeypatch, kernel):
 
 def test_split_group_logits_runtime_table_addresses(monkeypatch):
     monkeypatch.setenv("TQ_RUNTIME_TABLE_ADDRESSES", "1")
-    monkeypatch.setenv("TQ_LEGACY_MMA_SYNC", "1")
     _logits_case(B=2, Hq=8, Hkv=2, T=1001, sample=[(0, 1), (1, 0)], seed=2, stride_extra=3)
 
 
