@@ -49,8 +49,8 @@ METRIC = "vectors quantized/s; packed-KV logits keys/s and % of HBM-bandwidth ro
 # ran: when they differ from the files in this tree the figure is stale and
 # roofline.traffic is reported as null.
 MEASURED_TRAFFIC = {
-    "quant_mse": {"bytes": 299.6e6, "sources": "4823f0e5ed6de076", "capture": "profiles/sweep_traffic_bf16_d128.md"},
-    "dequant_mse": {"bytes": 521.1e6, "sources": "1fe914a60a9b05b0", "capture": "profiles/sweep_traffic_bf16_d128.md"},
+    "quant_mse": {"bytes": 299.4e6, "sources": "14acebe8f1133f32", "capture": "profiles/sweep_traffic_bf16_d128.md"},
+    "dequant_mse": {"bytes": 519.3e6, "sources": "1e172447f3500502", "capture": "profiles/sweep_traffic_bf16_d128.md"},
 }
 TRAFFIC_SOURCES = {
     "quant_mse": ["quant_tc.cu", "sm100_common.cuh"],

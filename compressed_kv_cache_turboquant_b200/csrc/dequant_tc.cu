@@ -322,35 +322,48 @@ __global__ void __launch_bounds__(kThreads, 1) dequant_tc_kernel(const __grid_co
         // the previous store from this warp's buffer must have read it
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        uint32_t pk[32];
+        // 16 columns of both accumulators at a time (a 32-column pair of
+        // loads plus the packed row does not fit the register budget of 13
+        // warps without spilling); each half fills four 16-byte units of the row
         if (a.out_bf16) {
 #pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            float v0[32], v1[32];
-            tmem_ld32(t0 + c * 64 + hlf * 32, v0);
-            tmem_ld32(t0 + D + c * 64 + hlf * 32, v1);
+          for (int q = 0; q < 4; ++q) {
+            float v0[16], v1[16];
+            tmem_ld16(t0 + c * 64 + q * 16, v0);
+            tmem_ld16(t0 + D + c * 64 + q * 16, v1);
             tmem_wait_ld();
+            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 8; ++e) {
               const float y0 = n * fmaf(v1[2 * e], 4.8828125e-4f, v0[2 * e]);
               const float y1 = n * fmaf(v1[2 * e + 1], 4.8828125e-4f, v0[2 * e + 1]);
               __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-              pk[16 * hlf + e] = *reinterpret_cast<uint32_t*>(&b2);
+              pk[e] = *reinterpret_cast<uint32_t*>(&b2);
             }
+#pragma unroll
+            for (int j = 2 * q; j < 2 * q + 2; ++j)
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                  make_uint4(pk[4 * (j - 2 * q)], pk[4 * (j - 2 * q) + 1], pk[4 * (j - 2 * q) + 2],
+                             pk[4 * (j - 2 * q) + 3]);
           }
         } else {
-          float v0[32], v1[32];
-          tmem_ld32(t0 + c * kCols, v0);
-          tmem_ld32(t0 + D + c * kCols, v1);
-          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
+          for (int hh = 0; hh < 2; ++hh) {
+            float v0[16], v1[16];
+            tmem_ld16(t0 + c * kCols + 16 * hh, v0);
+            tmem_ld16(t0 + D + c * kCols + 16 * hh, v1);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = __float_as_uint(n * fmaf(v1[e], 4.8828125e-4f, v0[e]));
+            // row `lane` of the 128B-swizzled box: 16-byte unit j lands at j ^ (lane & 7)
+#pragma unroll
+            for (int j = 4 * hh; j < 4 * hh + 4; ++j)
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                  make_uint4(pk[4 * (j - 4 * hh)], pk[4 * (j - 4 * hh) + 1], pk[4 * (j - 4 * hh) + 2],
+                             pk[4 * (j - 4 * hh) + 3]);
+          }
         }
-        // row `lane` of the 128B-swizzled box: 16-byte unit j lands at j ^ (lane & 7)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         fence_async_smem();
         __syncwarp();
         if (lane == 0 && row0 < a.N) {

@@ -334,7 +334,9 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       }
       const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
       const int64_t vec = tile * kTileM + row;
-#pragma unroll
+      // not unrolled: the two cell paths exist once each in the code (a
+      // fully unrolled loop outgrows the instruction cache at 4 bits)
+#pragma unroll 1
       for (int g = 0; g < kGroups; ++g) {
         float v[32];
         tmem_ld32(t0 + 32 * g, v);

@@ -180,7 +180,7 @@ def test_near_threshold_band_is_one_e_minus_5_over_sqrt_d(d):
     # exact band edge: thresholds (0, 0.25) and y = w are represented exactly
     edge = np.array([w, 0.25 + 2 * w, -w])
     assert np.array_equal(tq.near_threshold_mask(edge, np.array([0.0, 0.25]), d), [True, False, True])
-    # the mask keeps the shape of its input and judges each coordinate on its own
+    # the mask keeps the shape of its input and decides each coordinate on its own
     y = np.array([[t[0] + 0.5 * w, c[0]], [c[7], t[6] - 2 * w]])
     assert np.array_equal(tq.near_threshold_mask(y, t, d), [[True, False], [False, False]])
 
