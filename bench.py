@@ -49,7 +49,7 @@ METRIC = "vectors quantized/s; packed-KV logits keys/s and % of HBM-bandwidth ro
 # ran: when they differ from the files in this tree the figure is stale and
 # roofline.traffic is reported as null.
 MEASURED_TRAFFIC = {
-    "quant_mse": {"bytes": 299.4e6, "sources": "14acebe8f1133f32", "capture": "profiles/sweep_traffic_bf16_d128.md"},
+    "quant_mse": {"bytes": 299.5e6, "sources": "3c007b3786cd370d", "capture": "profiles/sweep_traffic_bf16_d128.md"},
     "dequant_mse": {"bytes": 519.3e6, "sources": "1e172447f3500502", "capture": "profiles/sweep_traffic_bf16_d128.md"},
 }
 TRAFFIC_SOURCES = {
@@ -889,6 +889,8 @@ PROFILE_CASES = {
     "search": "quantize + fused top-10 scoring: d = --search-d, --profile-n keys (default 200000), "
               "--profile-nq queries (default 1280)",
     "sweep": "the sweep step (quantize + dequantize at b = 1..4, 2^20 bf16 vectors)",
+    "prefill": "prefill of --profile-nq new tokens (default 128) over the config-4 cache at context --profile-t "
+               "(default 32768)",
 }
 
 
@@ -908,6 +910,11 @@ def run_profile_case(args):
     elif case == "logits":
         wl = Stream(tq, torch, 0, dev, T=args.profile_t or (1 << 18))
         call, size = wl.logits_only, {"T": wl.T}
+    elif case == "prefill":
+        DEC["T"] = args.profile_t or 32768
+        dec = Decode(tq, torch, 0, dev)
+        wl = Prefill(tq, torch, dec, nq=args.profile_nq or 128)
+        call, size = wl.step, {"T": DEC["T"], "nq": wl.nq}
     elif case == "search":
         n, nq = args.profile_n or 200000, args.profile_nq or 1280
         wl = Search(tq, torch, 0, dev, d=args.search_d, N=n, nq=nq)

@@ -13,9 +13,9 @@
 //   warp 1      TMEM allocation and the single-thread MMA issuer:
 //               Y[128 x d] = X[128 x d] . (Pi_hi + Pi_mid + Pi_lo)^T, three
 //               bf16 passes accumulated in fp32 in TMEM (double-buffered)
-//   warps 2-17  epilogue: four sets of four warps (one per TMEM lane
+//   warps 2-13  epilogue: three sets of four warps (one per TMEM lane
 //               quarter) take the tiles in turn, each set with its own
-//               accumulator buffer, so four tiles are in flight; one thread
+//               accumulator buffer, so three tiles are in flight; one thread
 //               per vector (TMEM lane) reads the vector's columns twice: once
 //               for n = ||y|| (= ||x||, Pi orthogonal), once for the cell of
 //               every coordinate against n * t_k, packing and stores.  Even
@@ -40,7 +40,7 @@ using namespace sm100;
 
 constexpr int kPieces = 3;
 constexpr int kTileM = 128;
-constexpr int kSets = 4;                  // epilogue warp sets = accumulator buffers
+constexpr int kSets = 3;                  // epilogue warp sets = accumulator buffers
 // warps: TMA producer, MMA issuer, kSets sets of 4 epilogue warps
 template <int D>
 constexpr int threads_for() { return 32 * (2 + 4 * kSets); }
@@ -311,15 +311,18 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       }
       tc_fence_after();
       const uint32_t t0 = tmem_base + lb + (uint32_t)(ab * D);
-      // n = ||y|| from all of the vector's columns
+      // n = ||y|| from all of the vector's columns, two 32-column loads per wait
       float ss = 0.f;
 #pragma unroll
-      for (int g = 0; g < kGroups; ++g) {
-        float v[32];
+      for (int g = 0; g < kGroups; g += 2) {
+        float v[32], w[32];
         tmem_ld32(t0 + 32 * g, v);
+        tmem_ld32(t0 + 32 * (g + 1), w);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) ss = fmaf(v[c], v[c], ss);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) ss = fmaf(w[c], w[c], ss);
       }
       const float n = sqrtf(ss);
       // positive thresholds t_m (m = 1 .. H - 1) scaled by n, and the
@@ -334,23 +337,28 @@ __global__ void __launch_bounds__(threads_for<D>(), 1)
       }
       const float Bf = n > 0.f ? 4294967296.f / n : 0.f;
       const int64_t vec = tile * kTileM + row;
-      // not unrolled: the two cell paths exist once each in the code (a
-      // fully unrolled loop outgrows the instruction cache at 4 bits)
+      // two groups per iteration, loaded together (one wait): the even group
+      // takes the ALU-pipe search, the odd one the FMA-pipe count, and the
+      // loop is not unrolled further, so each cell path exists once in the code
+      // (a fully unrolled loop outgrows the instruction cache at 4 bits)
 #pragma unroll 1
-      for (int g = 0; g < kGroups; ++g) {
-        float v[32];
+      for (int g = 0; g < kGroups; g += 2) {
+        float v[32], u[32];
         tmem_ld32(t0 + 32 * g, v);
+        tmem_ld32(t0 + 32 * (g + 1), u);
         tmem_wait_ld();
-        if (g + 1 == kGroups) {
+        if (g + 2 == kGroups) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
         if (vec < a.N) {
           uint32_t w[BM];
-          if (BM >= 2 && (g & 1)) pack_group_fma<BM>(v, P, Bf, Cz, w);
-          else pack_group<BM>(v, P, w);
+          pack_group<BM>(v, P, w);
           store_words<BM>(a.codes + vec * a.out_stride * W + g * BM, w);
+          if (BM >= 2) pack_group_fma<BM>(u, P, Bf, Cz, w);
+          else pack_group<BM>(u, P, w);
+          store_words<BM>(a.codes + vec * a.out_stride * W + (g + 1) * BM, w);
         }
       }
       if (vec < a.N) a.norms[vec * a.out_stride] = n;
