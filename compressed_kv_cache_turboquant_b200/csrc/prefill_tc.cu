@@ -57,7 +57,9 @@ constexpr int kRows = 128;               // query rows per CTA
 constexpr int kThreads = 320;
 constexpr int kKW = 12, kSW = 4, kVW = 16;
 constexpr int kOffK = 0, kOffS = kOffK + kTK * kKW * 4, kOffV = kOffS + kTK * kSW * 4;
-constexpr int kStage = kOffV + kTK * kVW * 4;   // 16384
+// the three norm arrays of the tile follow the codes (whole groups of 4 tokens)
+constexpr int kOffKN = kOffV + kTK * kVW * 4, kOffKR = kOffKN + kTK * 4, kOffVN = kOffKR + kTK * 4;
+constexpr int kStage = kOffVN + kTK * 4;   // 17920
 constexpr int kTile = 2 * kTK * 128;             // one [128 x 128] fp16 operand (two 64-wide slabs)
 constexpr uint32_t kColQ1 = 0, kColQ2 = 64, kColS1 = 128, kColS2 = 256, kColO = 384;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -183,10 +185,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
         const int n = (int)min((int64_t)kTK, a.T - t0);
         const int64_t r = bh * a.kv_stride + t0;
         uint8_t* st = ring + s * kStage;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)(n * (kKW + kSW + kVW) * 4));
+        const int n4 = n & ~3;  // norms in whole 16-byte units; a tail of up to 3 comes from global memory
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(n * (kKW + kSW + kVW) * 4 + 3 * n4 * 4));
         bulk_load(st + kOffK, a.kcodes + r * kKW, n * kKW * 4, &full[s]);
         bulk_load(st + kOffS, a.ksigns + r * kSW, n * kSW * 4, &full[s]);
         bulk_load(st + kOffV, a.vcodes + r * kVW, n * kVW * 4, &full[s]);
+        if (n4) {
+          bulk_load(st + kOffKN, a.knorms + r, n4 * 4, &full[s]);
+          bulk_load(st + kOffKR, a.krnorms + r, n4 * 4, &full[s]);
+          bulk_load(st + kOffVN, a.vnorms + r, n4 * 4, &full[s]);
+        }
         issued = it + 1;
       }
       for (int it = issued - 2 > 0 ? issued - 2 : 0; it < issued; ++it)
@@ -287,8 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
                 make_uint4(sp[4 * u], sp[4 * u + 1], sp[4 * u + 2], sp[4 * u + 3]);
         }
         float* nb = nrm + (it & 1) * 2 * kTK;
-        nb[t] = t < n ? a.knorms[row0 + t] : 0.f;
-        nb[kTK + t] = t < n ? a.krnorms[row0 + t] : 0.f;
+        const int n4 = n & ~3;
+        const float* skn = reinterpret_cast<const float*>(st + kOffKN);
+        const float* skr = reinterpret_cast<const float*>(st + kOffKR);
+        nb[t] = t < n4 ? skn[t] : (t < n ? a.knorms[row0 + t] : 0.f);
+        nb[kTK + t] = t < n4 ? skr[t] : (t < n ? a.krnorms[row0 + t] : 0.f);
       }
       fence_async_smem();
       __syncwarp();
@@ -301,8 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       }
       {
         const int k0 = 2 * m, k1 = 2 * m + 1;
-        const __half2 n0 = __float2half2_rn(k0 < n ? a.vnorms[row0 + k0] : 0.f);
-        const __half2 n1 = __float2half2_rn(k1 < n ? a.vnorms[row0 + k1] : 0.f);
+        const int n4 = n & ~3;
+        const float* svn = reinterpret_cast<const float*>(st + kOffVN);
+        const __half2 n0 = __float2half2_rn(k0 < n4 ? svn[k0] : (k0 < n ? a.vnorms[row0 + k0] : 0.f));
+        const __half2 n1 = __float2half2_rn(k1 < n4 ? svn[k1] : (k1 < n ? a.vnorms[row0 + k1] : 0.f));
         const uint32_t* v0 = reinterpret_cast<const uint32_t*>(st + kOffV) + k0 * kVW + 8 * ch;
         const uint32_t* v1 = v0 + kVW;
         const int slab = m >> 5, unit = (m & 31) >> 2, sub = (m & 3) * 4;
@@ -381,15 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       }
       tc_fence_after();
       const float* nb = nrm + (it & 1) * 2 * kTK;
-      // logits (base 2) of 16 keys from the two accumulators; keys past this
-      // row's position (or the context end) are -FLT_MAX
-      auto logits16 = [&](int c0, float (&x)[16]) {
-        float v1[16], v2[16];
-        tmem_ld16(tmem + lb + kColS1 + c0, v1);
-        tmem_ld16(tmem + lb + kColS2 + c0, v2);
+      // logits (base 2) of 32 keys from the two accumulators, one tensor-memory
+      // wait for both 32-column loads; keys past this row's position (or the
+      // context end) are -FLT_MAX
+      auto logits32 = [&](int c0, float (&x)[32]) {
+        float v1[32], v2[32];
+        tmem_ld32(tmem + lb + kColS1 + c0, v1);
+        tmem_ld32(tmem + lb + kColS2 + c0, v2);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 32; ++e) {
           const int k = c0 + e;
           const bool vis = live && t0 + k <= pos && t0 + k < a.T;
           x[e] = vis ? fmaf(nb[k] * c1, v1[e], nb[kTK + k] * c2 * v2[e]) : -FLT_MAX;
@@ -397,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       };
       // pass 1: the row max of the tile
       float mx = -FLT_MAX;
-#pragma unroll 2
-      for (int c0 = 0; c0 < kTK; c0 += 16) {
-        float x[16];
-        logits16(c0, x);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTK; c0 += 32) {
+        float x[32];
+        logits32(c0, x);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, x[e]);
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, x[e]);
       }
       // lazy rescale: a row's reference max moves only when one of its logits
       // passes it by kLazy.  The O rescale goes through warp-collective tensor
@@ -440,14 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       // columns written hold keys the earlier reads have consumed
 #pragma unroll 1
       for (int c0 = 0; c0 < kTK; c0 += 32) {
-        float x0[16], x1[16];
-        logits16(c0, x0);
-        logits16(c0 + 16, x1);
+        float x[32];
+        logits32(c0, x);
         uint32_t pu[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float xa = e < 8 ? x0[2 * e] : x1[2 * e - 16];
-          const float xb = e < 8 ? x0[2 * e + 1] : x1[2 * e - 15];
+          const float xa = x[2 * e];
+          const float xb = x[2 * e + 1];
           const float p0 = xa > -FLT_MAX ? exp2f(xa - m_run) : 0.f;
           const float p1 = xb > -FLT_MAX ? exp2f(xb - m_run) : 0.f;
           const __half2 ph = __floats2half2_rn(p0, p1);

@@ -156,12 +156,33 @@ __device__ __forceinline__ uint32_t code_of(const uint32_t* w /*BM words of the 
 }
 
 __global__ void gen_norms_kernel(const void* x, int xbf16, int64_t x_stride, int64_t N, int d, float* norms,
-                                 int64_t out_stride, const int32_t* channels, const int64_t* slots) {
+                                 int64_t out_stride, const int32_t* channels, const int64_t* slots, int vec16) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t v = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; v < N; v += warps) {
     double acc = 0.0;
-    if (xbf16) {
+    if (vec16) {
+      // 16-byte loads: rows start 16-byte aligned and d is a whole number of them
+      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + v * x_stride * (xbf16 ? 2 : 4));
+      const int nv = xbf16 ? d / 8 : d / 4;
+      for (int j = lane; j < nv; j += 32) {
+        const uint4 w = p[j];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        if (xbf16) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const double t0 = (double)__uint_as_float(ws[k] << 16), t1 = (double)__uint_as_float(ws[k] & 0xFFFF0000u);
+            acc = fma(t0, t0, fma(t1, t1, acc));
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const double t = (double)__uint_as_float(ws[k]);
+            acc = fma(t, t, acc);
+          }
+        }
+      }
+    } else if (xbf16) {
       const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(x) + v * x_stride;
       for (int j = lane; j < d; j += 32) {
         const double t = (double)__bfloat162float(p[channels ? channels[j] : j]);
@@ -602,8 +623,11 @@ int launch_gen_norms(const tq_ctx* h, const void* x, int dtype, int64_t N, int64
                      int64_t out_stride, void* stream, const int32_t* channels, const int64_t* slots) {
   const int64_t blocks = (N + 7) / 8;  // 8 warps per block, one vector per warp
   const int grid = (int)(blocks < (int64_t)h->sm_count * 16 ? blocks : (int64_t)h->sm_count * 16);
+  const int esz = dtype == TQ_BF16 ? 2 : 4;
+  const int vec16 = !channels && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (x_stride * esz) % 16 == 0 &&
+                    (h->d * esz) % 16 == 0;
   gen_norms_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, dtype == TQ_BF16 ? 1 : 0, x_stride, N, h->d, norms,
-                                                          out_stride, channels, slots);
+                                                          out_stride, channels, slots, vec16);
   return (int)cudaGetLastError();
 }
 
