@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cfloat>
 
 #include "tq_internal.h"
@@ -321,6 +322,65 @@ __global__ void query_prep_kernel(const TIn* q, int64_t nq, int d, const float* 
 }
 
 // One thread per (query, key): est = n <q', c[idx]> + rn sqrt(pi/2)/d <q'', sigma>.
+// q' = Pi q and q'' = S q for d = 128 as a tiled fp32 product: the block
+// (blockIdx.y = which matrix) keeps M^T in shared memory and loops over tiles
+// of 32 query rows; thread (ty, tx) accumulates rows 4 ty .. + 3 x outputs
+// 4 tx .. + 3, summing over the input coordinate in order.
+constexpr int kQpRows = 32;
+constexpr int kQpLd = 132;   // padded row length (floats) of the shared tiles
+constexpr int kQpSmem = (128 + kQpRows) * kQpLd * 4;
+
+template <typename TIn>
+__global__ void __launch_bounds__(256) query_prep_tiled_kernel(const TIn* q, int64_t nq, const float* Pi,
+                                                               const float* S, float* qrot, float* qproj) {
+  extern __shared__ __align__(16) float qp_smem[];
+  float* mt = qp_smem;                   // [i][j] = M[j][i]
+  float* qs = qp_smem + 128 * kQpLd;     // [row][i]
+  const float* M = blockIdx.y ? S : Pi;
+  float* out = blockIdx.y ? qproj : qrot;
+  for (int e = threadIdx.x; e < 128 * 128; e += 256) mt[(e & 127) * kQpLd + (e >> 7)] = M[e];
+  const int ty = threadIdx.x >> 5, tx = threadIdx.x & 31;
+  const int64_t tiles = (nq + kQpRows - 1) / kQpRows;
+  for (int64_t rt = blockIdx.x; rt < tiles; rt += gridDim.x) {
+    const int64_t r0 = rt * kQpRows;
+    __syncthreads();
+    for (int e = threadIdx.x; e < kQpRows * 128; e += 256) {
+      const int64_t row = r0 + (e >> 7);
+      qs[(e >> 7) * kQpLd + (e & 127)] = row < nq ? load_elem(q, row * 128 + (e & 127)) : 0.f;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < 128; i += 4) {
+      float4 xa[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) xa[r] = *reinterpret_cast<const float4*>(qs + (4 * ty + r) * kQpLd + i);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 mb = *reinterpret_cast<const float4*>(mt + (i + k) * kQpLd + 4 * tx);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float x = k == 0 ? xa[r].x : k == 1 ? xa[r].y : k == 2 ? xa[r].z : xa[r].w;
+          acc[r][0] = fmaf(mb.x, x, acc[r][0]);
+          acc[r][1] = fmaf(mb.y, x, acc[r][1]);
+          acc[r][2] = fmaf(mb.z, x, acc[r][2]);
+          acc[r][3] = fmaf(mb.w, x, acc[r][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int64_t row = r0 + 4 * ty + r;
+      if (row < nq)
+        *reinterpret_cast<float4*>(out + row * 128 + 4 * tx) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
+  }
+}
+
 __global__ void scores_simple_kernel(const float* qrot, const float* qproj, int64_t nq,
                                      const uint32_t* codes, const uint32_t* signs,
                                      const float* norms, const float* rnorms, int64_t N, int d,
@@ -571,6 +631,19 @@ int launch_query_prep(const tq_ctx* h, const float* q, int q_dtype, int64_t nq, 
   const int grid = grid_for((warps * 32 + 255) / 256, h->sm_count * 32);
   const float* S = qproj ? h->dev.S : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
+  const bool out16 = ((reinterpret_cast<uintptr_t>(qrot) | reinterpret_cast<uintptr_t>(qproj)) & 15u) == 0;
+  if (h->d == 128 && nq > 0 && out16) {
+    const void* kern = q_dtype == TQ_BF16 ? (const void*)query_prep_tiled_kernel<__nv_bfloat16>
+                                          : (const void*)query_prep_tiled_kernel<float>;
+    if (int e = ensure_dyn_smem(kern, kQpSmem)) return e;
+    const int64_t tiles = (nq + kQpRows - 1) / kQpRows;
+    const dim3 grid2((unsigned)std::min<int64_t>(tiles, h->sm_count), qproj ? 2u : 1u);
+    if (q_dtype == TQ_BF16)
+      query_prep_tiled_kernel<<<grid2, 256, kQpSmem, s>>>((const __nv_bfloat16*)q, nq, h->dev.Pi, S, qrot, qproj);
+    else
+      query_prep_tiled_kernel<<<grid2, 256, kQpSmem, s>>>(q, nq, h->dev.Pi, S, qrot, qproj);
+    return (int)cudaGetLastError();
+  }
   if (q_dtype == TQ_BF16)
     query_prep_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, nq, h->d, h->dev.Pi, S, qrot, qproj);
   else

@@ -8,34 +8,44 @@
 // position T - nq + i and sees keys t <= T - nq + i.
 //
 // With many queries per key the work is a pair of GEMMs per key tile, so every
-// product runs on tcgen05 with the decoded cache as the shared-memory operand:
-//   S1 = Q' C^T      Q' = Pi_K q (fp16, per-row power-of-two scale), C = the
-//                    key centroids c[idx] (fp16)
-//   S2 = Q'' Sg^T    Q'' = S_K q, Sg = the QJL signs as +-1
-//   logit = scale (n_k S1 / s' + rn_k sqrt(pi/2)/d S2 / s'')
-//   O   += P V^T-tile  P = e^(logit - m) (fp16, written back into tensor memory),
-//                    V = n_v c_V[idx] (fp16) in the rotated value frame
+// product runs on tcgen05 with the decoded cache as the shared-memory operand.
+// The estimator's two terms share one accumulator:
+//   S = Q' C^T + Q'' Sg^T
+//     Q'  = s Pi_K q                     C  = n_k c[idx]        (fp16)
+//     Q'' = s sqrt(pi/2)/d S_K q         Sg = rn_k sign(S_K r)  (fp16)
+//   with s a power of two per query row (the larger of the two rows' maxima
+//   placed at 2^13..2^14), so logit = scale S / s
+//   O += P V^T-tile   P = 2^(log2e logit - m) (fp16, written back into tensor
+//                     memory), V = n_v c_V[idx] (fp16) in the rotated value frame
 // One CTA per (batch, kv-head, tile of 128 query rows, slice of the context);
 // a query row is a (token, head of the kv-head's group) pair.  Q' and Q'' live
-// in tensor memory as the A operands of the two logit products, P overwrites
-// S1 as the A operand of the value product; the decoded key and value tiles
-// are the B operands in shared memory.  Each CTA writes its rows' softmax
-// records (acc in the rotated frame, m, l); the merge kernel combines the
-// slices and applies Pi_V^T once.
+// in tensor memory as the A operands of the logit product, P overwrites the
+// first half of its logit buffer as the A operand of the value product; the
+// decoded key and value tiles are the B operands in shared memory.  Two logit
+// buffers let the product of key tile i + 1 run while the softmax warps work
+// on tile i.  Each CTA writes its rows' softmax records (acc in the rotated
+// frame, m, l); the merge kernel combines the slices and applies Pi_V^T once.
 //
 // Warps (320 threads, one CTA per SM):
-//   0      bulk copies of each 128-token tile of packed K codes, QJL signs and
-//          V codes into a two-stage ring
+//   0      bulk copies of each 128-token tile of packed K codes, QJL signs,
+//          V codes and the three norms into a three-stage ring
 //   1      TMEM allocation and the single-thread MMA issuer
-//   2-5    decoders: thread t decodes key t into the centroid and sign tiles
-//          (byte-table lookups, one shift and one logic op per sign pair), then
-//          key pairs into the transposed value tile (keys as the K dimension)
-//   6-9    softmax: thread = query row (TMEM lane), online softmax in base 2
-//          with a lazy rescale of O
-// Tensor memory: Q' [0, 64) | Q'' [64, 128) | S1 / P [128, 256) | S2 [256, 384)
-// | O [384, 512).  The sign tile pairs coordinates (32g + c, 32g + 16 + c) in
-// each 32-bit element, and Q'' is written with the same pairing (a consistent
-// reordering of the K dimension of one product).
+//   2-5    decoders: thread t decodes key t of tile i + 1 into the centroid and
+//          sign tiles (centroids from register byte tables by byte permutes,
+//          the norms multiplied in), then key t of tile i into its row of one
+//          of two value tiles (an MN-major B operand, so each key's decoded row
+//          is stored whole; byte-table lookups in a per-lane copy of the table)
+//          once the value product of tile i - 2 is done with that tile
+//   6-9    softmax: thread = query row (TMEM lane); a tile's 128 logits stay in
+//          registers for both passes (row max, then weights), online softmax in
+//          base 2 with a lazy rescale of O
+// Tensor memory: Q' [0, 64) | Q'' [64, 128) | S/P buffer 0 [128, 256) |
+// S/P buffer 1 [256, 384) | O [384, 512).  The sign tile pairs coordinates
+// (32g + c, 32g + 16 + c) in each 32-bit element, and Q'' is written with the
+// same pairing (a consistent reordering of the K dimension of one product).
+//
+// Range: the fp16 key and value tiles hold n_k c, rn_k and n_v c_V, so key and
+// value norms must stay below 65504 / max|c| (about 3e5 for these codebooks).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -55,23 +65,23 @@ constexpr int D = 128;
 constexpr int kTK = 128;                 // keys per tile
 constexpr int kRows = 128;               // query rows per CTA
 constexpr int kThreads = 320;
+constexpr int kStages = 3;               // ring stages of packed tiles
 constexpr int kKW = 12, kSW = 4, kVW = 16;
 constexpr int kOffK = 0, kOffS = kOffK + kTK * kKW * 4, kOffV = kOffS + kTK * kSW * 4;
 // the three norm arrays of the tile follow the codes (whole groups of 4 tokens)
 constexpr int kOffKN = kOffV + kTK * kVW * 4, kOffKR = kOffKN + kTK * 4, kOffVN = kOffKR + kTK * 4;
 constexpr int kStage = kOffVN + kTK * 4;   // 17920
 constexpr int kTile = 2 * kTK * 128;             // one [128 x 128] fp16 operand (two 64-wide slabs)
-constexpr uint32_t kColQ1 = 0, kColQ2 = 64, kColS1 = 128, kColS2 = 256, kColO = 384;
+constexpr uint32_t kColQ1 = 0, kColQ2 = 64, kColS = 128, kColO = 384;   // S/P buffers at 128 and 256
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;            // rescale O only when the max grows by 2^8
-// shared layout
-constexpr int kOffRing = 0;
-constexpr int kOffC = kOffRing + 2 * kStage;
+// shared layout: the swizzled operand tiles first (1024-byte aligned)
+constexpr int kOffC = 0;
 constexpr int kOffSg = kOffC + kTile;
-constexpr int kOffVt = kOffSg + kTile;
-constexpr int kOffTab = kOffVt + kTile;          // K table [256] + V table [256] fp16 pairs
-constexpr int kOffNorm = kOffTab + 2 * 1024;     // [2][2][128] kn, kr
-constexpr int kOffBar = kOffNorm + 2 * 2 * kTK * 4;
+constexpr int kOffVt = kOffSg + kTile;                 // two value tiles
+constexpr int kOffRing = kOffVt + 2 * kTile;
+constexpr int kOffTab = kOffRing + kStages * kStage;   // value byte table, one copy per lane: [256][32]
+constexpr int kOffBar = kOffTab + 256 * 32 * 4;
 constexpr int kSmem = kOffBar + 256 + 1024;
 
 struct PfArgs {
@@ -83,7 +93,7 @@ struct PfArgs {
   const float* vnorms;
   const float* qrot;       // [rows][d] fp32, rows = (b nq + i) Hq + j
   const float* qproj;
-  const float* kcent;      // [8]
+  uint32_t ktab[4];        // key codebook (8 entries) as fp16 byte tables: lo bytes c0-3, c4-7, hi bytes c0-3, c4-7
   const float* vcent;      // [16]
   int B, nq, Hq, Hkv, g;   // g = Hq / Hkv query heads per kv-head
   int64_t T, kv_stride;
@@ -98,6 +108,69 @@ struct PfArgs {
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// 2^x by the hardware's approximate exponential (subnormal results flush to 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// An empty statement that the compiler sees as redefining r: placed right after
+// tcgen05.wait::ld, it keeps every use of the loaded registers behind the wait
+// (the load's results are asynchronous, which the compiler does not know).
+__device__ __forceinline__ void regs_after_wait(float (&r)[32]) {
+  asm volatile(""
+               : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]), "+f"(r[6]), "+f"(r[7]), "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]), "+f"(r[12]), "+f"(r[13]), "+f"(r[14]), "+f"(r[15]), "+f"(r[16]), "+f"(r[17]), "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]), "+f"(r[22]), "+f"(r[23]), "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]), "+f"(r[30]), "+f"(r[31])::"memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// eight 3-bit codes in the nibbles of x (bit 3 of each nibble ignored) -> four
+// fp16 pairs (codes 0,1 | 2,3 | 4,5 | 6,7) through register byte tables: one
+// byte permute picks the low bytes of four centroids, another the high bytes
+__device__ __forceinline__ void decode8(uint32_t x, const uint32_t (&t)[4], uint32_t* out) {
+  const uint32_t s0 = x & 0x7777u, s1 = (x >> 16) & 0x7777u;
+  const uint32_t l0 = prmt(t[0], t[1], s0), h0 = prmt(t[2], t[3], s0);
+  const uint32_t l1 = prmt(t[0], t[1], s1), h1 = prmt(t[2], t[3], s1);
+  out[0] = prmt(l0, h0, 0x5140);
+  out[1] = prmt(l0, h0, 0x7362);
+  out[2] = prmt(l1, h1, 0x5140);
+  out[3] = prmt(l1, h1, 0x7362);
+}
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzled
+// canonical layout: 64-element (128-byte) rows along N, 8-row atoms along K
+// `sbo` bytes apart, the next 64 N elements `lbo` bytes further.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // byte offset of 16-byte unit u (8 fp16) of row r in slab s of a [128 x 128] K-major 128B-swizzled tile
 __device__ __forceinline__ uint32_t tile_off(int s, int r, int u) {
   return (uint32_t)(s * kTK * 128 + r * 128 + ((u ^ (r & 7)) << 4));
@@ -110,21 +183,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
   uint8_t* ctile = smem + kOffC;
   uint8_t* stile = smem + kOffSg;
   uint8_t* vtile = smem + kOffVt;
-  uint32_t* ktab = reinterpret_cast<uint32_t*>(smem + kOffTab);
-  uint32_t* vtab = ktab + 256;
-  float* nrm = reinterpret_cast<float*>(smem + kOffNorm);     // [2 buffers][kn 128 | kr 128]
+  uint32_t* vtab = reinterpret_cast<uint32_t*>(smem + kOffTab);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* full = bars;          // [2] ring, tx
-  uint64_t* empty = bars + 2;     // [2] ring, 4 decoder warps
-  uint64_t* cs_ready = bars + 4;  // 4 decoder warps
-  uint64_t* cs_free = bars + 5;   // MMA commit
-  uint64_t* v_ready = bars + 6;   // 4 decoder warps
-  uint64_t* pv_done = bars + 7;   // MMA commit
-  uint64_t* s_full = bars + 8;    // MMA commit
-  uint64_t* p_ready = bars + 9;   // 4 softmax warps
-  uint64_t* q_ready = bars + 10;  // 4 softmax warps
-  uint64_t* done = bars + 11;     // MMA commit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* full = bars;          // [kStages] ring, tx
+  uint64_t* empty = bars + 3;     // [kStages] ring, 4 decoder warps
+  uint64_t* cs_ready = bars + 6;  // 4 decoder warps: centroid and sign tiles written
+  uint64_t* cs_free = bars + 7;   // MMA commit: logit product done with them
+  uint64_t* v_ready = bars + 8;   // [2] 4 decoder warps: value tile written
+  uint64_t* v_free = bars + 10;   // [2] MMA commit: the value product done with the value tile
+  uint64_t* pv_done = bars + 12;  // MMA commit: value product done
+  uint64_t* s_full = bars + 13;   // [2] MMA commit: logit buffer holds S
+  uint64_t* p_ready = bars + 15;  // [2] 4 softmax warps: P written into the buffer
+  uint64_t* q_ready = bars + 17;  // 4 softmax warps
+  uint64_t* done = bars + 18;     // MMA commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // this CTA's (batch, kv-head, query tile, context slice)
@@ -146,24 +218,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
   const int nkt = kt_hi > kt_lo ? (int)(kt_hi - kt_lo) : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 4);
     }
     mbar_init(cs_ready, 4);
     mbar_init(cs_free, 1);
-    mbar_init(v_ready, 4);
     mbar_init(pv_done, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_ready, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&v_ready[s], 4);
+      mbar_init(&v_free[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_ready[s], 4);
+    }
     mbar_init(q_ready, 4);
     mbar_init(done, 1);
     fence_mbar_init();
   }
-  // byte tables: K byte -> (c[B & 7], c[(B >> 4) & 7]), V byte -> (c[B & 15], c[B >> 4]) as fp16 pairs
-  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
-    ktab[e] = h2u(__floats2half2_rn(a.kcent[e & 7], a.kcent[(e >> 4) & 7]));
-    vtab[e] = h2u(__floats2half2_rn(a.vcent[e & 15], a.vcent[e >> 4]));
+  // value byte table: byte B -> (c[B & 15], c[B >> 4]) as an fp16 pair, one
+  // copy per lane (entry B of lane l at word 32 B + l), so that lookups of a
+  // warp never share a bank
+  for (int e = threadIdx.x; e < 256 * 32; e += blockDim.x) {
+    const int byte = e >> 5;
+    vtab[e] = h2u(__floats2half2_rn(a.vcent[byte & 15], a.vcent[byte >> 4]));
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -176,8 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
     if (lane == 0) {
       int issued = 0;
       for (int it = 0; it < nkt; ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(&empty[s], (uint32_t)(((it >> 1) & 1) ^ 1))) {
+        const int s = it % kStages;
+        if (!mbar_wait(&empty[s], (uint32_t)(((it / kStages) & 1) ^ 1))) {
           atomicOr(a.status, kStatusTimeout);
           break;
         }
@@ -197,147 +274,186 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
         }
         issued = it + 1;
       }
-      for (int it = issued - 2 > 0 ? issued - 2 : 0; it < issued; ++it)
-        if (!mbar_wait(&full[it & 1], (uint32_t)((it >> 1) & 1))) atomicOr(a.status, kStatusTimeout);
+      // no bulk copy may still be in flight when the CTA exits
+      for (int it = issued - kStages > 0 ? issued - kStages : 0; it < issued; ++it)
+        if (!mbar_wait(&full[it % kStages], (uint32_t)((it / kStages) & 1))) atomicOr(a.status, kStatusTimeout);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(kRows, kTK, false);
+      const uint32_t idesc_pv = idesc | (1u << 16);   // B (the value tile) MN-major
       const uint32_t cbase = smem_u32(ctile), sbase = smem_u32(stile), vbase = smem_u32(vtile);
-      bool ok = mbar_wait(q_ready, 0u);
-      for (int it = 0; ok && it < nkt; ++it) {
-        if (!mbar_wait(cs_ready, (uint32_t)(it & 1)) || (it > 0 && !mbar_wait(pv_done, (uint32_t)((it - 1) & 1)))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // S1 = Q' C^T, S2 = Q'' Sg^T: K = 128 coordinates in 8 steps of 16
+      // S(i) = Q' C^T + Q'' Sg^T into buffer i & 1: K = 2 x 128 in 16 steps of 16
+      auto logit_product = [&](int it) {
+        const uint32_t sc = tmem + kColS + (uint32_t)(it & 1) * 128;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t boff = (uint32_t)((ks >> 2) * kTK * 128 + (ks & 3) * 32);
-          mma_f16_ta(tmem + kColS1, tmem + kColQ1 + 8 * ks, sw128_kmajor_desc(cbase + boff), idesc, ks ? 1u : 0u);
-          mma_f16_ta(tmem + kColS2, tmem + kColQ2 + 8 * ks, sw128_kmajor_desc(sbase + boff), idesc, ks ? 1u : 0u);
+          mma_f16_ta(sc, tmem + kColQ1 + 8 * ks, sw128_kmajor_desc(cbase + boff), idesc, ks ? 1u : 0u);
         }
-        mma_commit(s_full);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t boff = (uint32_t)((ks >> 2) * kTK * 128 + (ks & 3) * 32);
+          mma_f16_ta(sc, tmem + kColQ2 + 8 * ks, sw128_kmajor_desc(sbase + boff), idesc, 1u);
+        }
+        mma_commit(&s_full[it & 1]);
         mma_commit(cs_free);
-        if (!mbar_wait(p_ready, (uint32_t)(it & 1)) || !mbar_wait(v_ready, (uint32_t)(it & 1))) {
+      };
+      bool ok = nkt == 0 || (mbar_wait(q_ready, 0u) && mbar_wait(cs_ready, 0u));
+      if (ok && nkt > 0) {
+        tc_fence_after();
+        logit_product(0);
+      }
+      for (int it = 0; ok && it < nkt; ++it) {
+        if (it + 1 < nkt) {
+          // buffer (it + 1) & 1 last held P(it - 1): the value product of tile it - 1 must be done with it
+          if (!mbar_wait(cs_ready, (uint32_t)((it + 1) & 1)) ||
+              (it > 0 && !mbar_wait(pv_done, (uint32_t)((it - 1) & 1)))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          logit_product(it + 1);
+        }
+        if (!mbar_wait(&p_ready[it & 1], (uint32_t)((it >> 1) & 1)) ||
+            !mbar_wait(&v_ready[it & 1], (uint32_t)((it >> 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // O += P Vt: K = 128 keys in 8 steps of 16 (P pairs keys 2m, 2m+1 in column m)
+        // O += P V: K = 128 keys in 8 steps of 16 (P pairs keys 2m, 2m+1 in
+        // column m); the value tile is MN-major (key rows of 128 bytes, 8-row
+        // atoms 1024 bytes apart, coordinates 64..127 one slab further)
+        const uint32_t pc = tmem + kColS + (uint32_t)(it & 1) * 128;
+        const uint32_t vt = vbase + (uint32_t)(it & 1) * kTile;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t boff = (uint32_t)((ks >> 2) * kTK * 128 + (ks & 3) * 32);
-          mma_f16_ta(tmem + kColO, tmem + kColS1 + 8 * ks, sw128_kmajor_desc(vbase + boff), idesc,
-                 (it | ks) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_f16_ta(tmem + kColO, pc + 8 * ks, sw128_mnmajor_desc(vt + ks * 2048, kTK * 128, 1024), idesc_pv,
+                     (it | ks) ? 1u : 0u);
+        mma_commit(&v_free[it & 1]);
         mma_commit(pv_done);
       }
       if (!ok) atomicOr(a.status, kStatusTimeout);
       mma_commit(done);
     }
   } else if (warp < 6) {
-    // ---------------- decoders
-    const int t = threadIdx.x - 64;          // key of the tile (centroid and sign rows)
-    const int m = t & 63, ch = t >> 6;       // key pair (2m, 2m+1) and coordinate half for the value tile
-    bool ok = true;
-    for (int it = 0; ok && it < nkt; ++it) {
-      const int s = it & 1;
+    // ---------------- decoders: thread t = key t of the tile
+    const int t = threadIdx.x - 64;
+    const uint32_t rb = smem_u32(ring);
+    const uint32_t ctb = smem_u32(ctile), stb = smem_u32(stile), vtb = smem_u32(vtile);
+    const uint32_t tab = smem_u32(vtab) + (uint32_t)lane * 4u;
+    const uint32_t ktab[4] = {a.ktab[0], a.ktab[1], a.ktab[2], a.ktab[3]};
+    // centroid row n_k c[idx] and sign row rn_k sign of key t (zeros past the context end)
+    auto decode_keys = [&](int it) -> bool {
+      const int s = it % kStages;
       const int64_t t0 = (kt_lo + it) * kTK;
       const int n = (int)min((int64_t)kTK, a.T - t0);
       const int64_t row0 = bh * a.kv_stride + t0;
-      if (!mbar_wait_warp(&full[s], (uint32_t)((it >> 1) & 1)) ||
-          (it > 0 && !mbar_wait_warp(cs_free, (uint32_t)((it - 1) & 1)))) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait_warp(&full[s], (uint32_t)((it / kStages) & 1)) ||
+          (it > 0 && !mbar_wait_warp(cs_free, (uint32_t)((it - 1) & 1))))
+        return false;
       const uint8_t* st = ring + s * kStage;
-      // centroid row and sign row of key t (zeros past the context end)
+      const uint32_t sb = rb + (uint32_t)(s * kStage);
+      const int n4 = n & ~3;
+      const bool kin = t < n;
+      const float kn = t < n4 ? reinterpret_cast<const float*>(st + kOffKN)[t] : (kin ? a.knorms[row0 + t] : 0.f);
+      const float kr = t < n4 ? reinterpret_cast<const float*>(st + kOffKR)[t] : (kin ? a.krnorms[row0 + t] : 0.f);
+      const __half2 kn2 = __float2half2_rn(kn);
+      // -rn_k in both halves; a set sign bit of the code flips a half to +rn_k
+      const uint32_t neg_rn = 0x80008000u | (0x00010001u * (uint32_t)__half_as_ushort(__float2half_rn(kr)));
+      uint32_t w[kKW], sg[kSW];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const uint4 v = kin ? lds128(sb + kOffK + (uint32_t)(t * kKW * 4 + 16 * q)) : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * q] = v.x, w[4 * q + 1] = v.y, w[4 * q + 2] = v.z, w[4 * q + 3] = v.w;
+      }
       {
-        uint32_t w[kKW], sg[kSW];
-        if (t < n) {
+        const uint4 v = kin ? lds128(sb + kOffS + (uint32_t)(t * kSW * 4)) : make_uint4(0u, 0u, 0u, 0u);
+        sg[0] = v.x, sg[1] = v.y, sg[2] = v.z, sg[3] = v.w;
+      }
 #pragma unroll
-          for (int q = 0; q < kKW; ++q) w[q] = reinterpret_cast<const uint32_t*>(st + kOffK)[t * kKW + q];
+      for (int gq = 0; gq < 4; ++gq) {  // 32-coordinate groups
+        // nibbles of w0, w1, w2 hold coordinates 0-23, their fourth bits coordinates 24-31
+        const uint32_t w0 = w[3 * gq], w1 = w[3 * gq + 1], w2 = w[3 * gq + 2];
+        const uint32_t s3 = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
+        uint32_t pr[16];
+        decode8(w0, ktab, pr);
+        decode8(w1, ktab, pr + 4);
+        decode8(w2, ktab, pr + 8);
+        decode8(s3, ktab, pr + 12);
 #pragma unroll
-          for (int q = 0; q < kSW; ++q) sg[q] = reinterpret_cast<const uint32_t*>(st + kOffS)[t * kSW + q];
-        } else {
+        for (int e = 0; e < 16; ++e) pr[e] = h2u(__hmul2(u2h(pr[e]), kn2));
+        // 32 coordinates = 4 units of 8; group gq is slab gq / 2, units 4 (gq & 1) .. + 3
 #pragma unroll
-          for (int q = 0; q < kKW; ++q) w[q] = 0u;
+        for (int u = 0; u < 4; ++u)
+          sts128(ctb + tile_off(gq >> 1, t, 4 * (gq & 1) + u), pr[4 * u], pr[4 * u + 1], pr[4 * u + 2],
+                 pr[4 * u + 3]);
+        // signs: element c of the group pairs coordinates (c, c + 16)
+        uint32_t sp[16];
+        const uint32_t x = sg[gq];
 #pragma unroll
-          for (int q = 0; q < kSW; ++q) sg[q] = 0u;
-        }
+        for (int c = 0; c < 16; ++c) sp[c] = neg_rn ^ ((x << (15 - c)) & 0x80008000u);
 #pragma unroll
-        for (int gq = 0; gq < 4; ++gq) {  // 32-coordinate groups
-          const uint32_t w0 = w[3 * gq], w1 = w[3 * gq + 1], w2 = w[3 * gq + 2];
-          const uint32_t s3 = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
-          const uint32_t src[4] = {w0, w1, w2, s3};
-          uint32_t pr[16];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int by = 0; by < 4; ++by) pr[4 * q + by] = t < n ? ktab[(src[q] >> (8 * by)) & 0xFFu] : 0u;
-          // 32 coordinates = 4 units of 8; group gq is slab gq / 2, units 4 (gq & 1) .. + 3
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(ctile + tile_off(gq >> 1, t, 4 * (gq & 1) + u)) =
-                make_uint4(pr[4 * u], pr[4 * u + 1], pr[4 * u + 2], pr[4 * u + 3]);
-          // signs: element c of the group pairs coordinates (c, c + 16): +1.0 = 0x3C00, -1.0 = 0xBC00
-          uint32_t sp[16];
-          const uint32_t x = sg[gq];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            sp[c] = t < n ? (0xBC00BC00u ^ ((x << (15 - c)) & 0x80008000u)) : 0u;
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(stile + tile_off(gq >> 1, t, 4 * (gq & 1) + u)) =
-                make_uint4(sp[4 * u], sp[4 * u + 1], sp[4 * u + 2], sp[4 * u + 3]);
-        }
-        float* nb = nrm + (it & 1) * 2 * kTK;
-        const int n4 = n & ~3;
-        const float* skn = reinterpret_cast<const float*>(st + kOffKN);
-        const float* skr = reinterpret_cast<const float*>(st + kOffKR);
-        nb[t] = t < n4 ? skn[t] : (t < n ? a.knorms[row0 + t] : 0.f);
-        nb[kTK + t] = t < n4 ? skr[t] : (t < n ? a.krnorms[row0 + t] : 0.f);
+        for (int u = 0; u < 4; ++u)
+          sts128(stb + tile_off(gq >> 1, t, 4 * (gq & 1) + u), sp[4 * u], sp[4 * u + 1], sp[4 * u + 2],
+                 sp[4 * u + 3]);
       }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(cs_ready);
-      // transposed value tile: row = coordinate, K = keys; thread (m, ch) writes
-      // the words (v[2m][c], v[2m+1][c]) for coordinates c of half ch
-      if (it > 0 && !mbar_wait_warp(pv_done, (uint32_t)((it - 1) & 1))) {
-        ok = false;
-        break;
+      return true;
+    };
+    // row t of value tile it & 1 (MN-major: key rows of 128 bytes, 8-row atoms
+    // 1024 bytes apart, coordinates 64..127 one slab further): n_v c_V[idx]
+    const uint32_t row_off = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128);
+    const uint32_t sw = (uint32_t)(t & 7);
+    auto decode_values = [&](int it) -> bool {
+      // the tile's buffer was last read by the value product of tile it - 2
+      if (it > 1 && !mbar_wait_warp(&v_free[it & 1], (uint32_t)(((it >> 1) - 1) & 1))) return false;
+      const int s = it % kStages;
+      const int64_t t0 = (kt_lo + it) * kTK;
+      const int n = (int)min((int64_t)kTK, a.T - t0);
+      const int64_t row0 = bh * a.kv_stride + t0;
+      const uint8_t* st = ring + s * kStage;
+      const uint32_t sb = rb + (uint32_t)(s * kStage) + kOffV + (uint32_t)(t * kVW * 4);
+      const int n4 = n & ~3;
+      const bool kin = t < n;
+      const float vn = t < n4 ? reinterpret_cast<const float*>(st + kOffVN)[t] : (kin ? a.vnorms[row0 + t] : 0.f);
+      const __half2 vn2 = __float2half2_rn(vn);
+      uint32_t w[kVW];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = kin ? lds128(sb + 16 * q) : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * q] = v.x, w[4 * q + 1] = v.y, w[4 * q + 2] = v.z, w[4 * q + 3] = v.w;
       }
-      {
-        const int k0 = 2 * m, k1 = 2 * m + 1;
-        const int n4 = n & ~3;
-        const float* svn = reinterpret_cast<const float*>(st + kOffVN);
-        const __half2 n0 = __float2half2_rn(k0 < n4 ? svn[k0] : (k0 < n ? a.vnorms[row0 + k0] : 0.f));
-        const __half2 n1 = __float2half2_rn(k1 < n4 ? svn[k1] : (k1 < n ? a.vnorms[row0 + k1] : 0.f));
-        const uint32_t* v0 = reinterpret_cast<const uint32_t*>(st + kOffV) + k0 * kVW + 8 * ch;
-        const uint32_t* v1 = v0 + kVW;
-        const int slab = m >> 5, unit = (m & 31) >> 2, sub = (m & 3) * 4;
+      const uint32_t vt = vtb + (uint32_t)((it & 1) * kTile) + row_off;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {           // code word q: coordinates 64 ch + 8 q .. + 7
-          const uint32_t a0 = k0 < n ? v0[q] : 0u, a1 = k1 < n ? v1[q] : 0u;
-#pragma unroll
-          for (int by = 0; by < 4; ++by) {      // byte: coordinates 2 by, 2 by + 1 of the word
-            const uint32_t p0 = h2u(__hmul2(u2h(vtab[(a0 >> (8 * by)) & 0xFFu]), n0));
-            const uint32_t p1 = h2u(__hmul2(u2h(vtab[(a1 >> (8 * by)) & 0xFFu]), n1));
-            const int c = 64 * ch + 8 * q + 2 * by;
-            *reinterpret_cast<uint32_t*>(vtile + tile_off(slab, c, unit) + sub) = __byte_perm(p0, p1, 0x5410);
-            *reinterpret_cast<uint32_t*>(vtile + tile_off(slab, c + 1, unit) + sub) = __byte_perm(p0, p1, 0x7632);
-          }
-        }
+      for (int q = 0; q < kVW; ++q) {
+        // word q: coordinates 8 q .. 8 q + 7, two per byte
+        const uint32_t x = w[q];
+        const uint32_t e0 = h2u(__hmul2(u2h(lds32(tab + ((x << 7) & 0x7F80u))), vn2));
+        const uint32_t e1 = h2u(__hmul2(u2h(lds32(tab + ((x >> 1) & 0x7F80u))), vn2));
+        const uint32_t e2 = h2u(__hmul2(u2h(lds32(tab + ((x >> 9) & 0x7F80u))), vn2));
+        const uint32_t e3 = h2u(__hmul2(u2h(lds32(tab + ((x >> 17) & 0x7F80u))), vn2));
+        const uint32_t m = (uint32_t)(q >> 3), j = (uint32_t)(q & 7);
+        sts128(vt + m * (kTK * 128) + ((j ^ sw) << 4), e0, e1, e2, e3);
       }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(v_ready);
+        mbar_arrive(&v_ready[it & 1]);
         mbar_arrive(&empty[s]);
       }
+      return true;
+    };
+    // keys run one tile ahead of values: the logit product of tile i + 1 needs
+    // only the logit product of tile i to be done, and with two value tiles
+    // the value tile of tile i waits for the value product of tile i - 2
+    bool ok = nkt == 0 || decode_keys(0);
+    for (int it = 0; ok && it < nkt; ++it) {
+      if (it + 1 < nkt) ok = decode_keys(it + 1);
+      if (ok) ok = decode_values(it);
     }
     if (!ok) atomicOr(a.status, kStatusTimeout);
   } else {
@@ -348,22 +464,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
     const int il = r / a.g, jl = r % a.g;
     const int tok = i0 + il;
     const bool live = il < tok_per_tile && tok < a.nq;
-    const int64_t grow = ((int64_t)b * a.nq + tok) * a.Hq + (int64_t)h * a.g + jl;   // global query row
+    const int64_t qrow = ((int64_t)b * a.nq + tok) * a.Hq + (int64_t)h * a.g + jl;   // global query row
     const int64_t pos = a.T - a.nq + tok;                                            // this row's position
-    // queries into tensor memory: Q' natural pairs, Q'' pairs (32 g + c, 32 g + 16 + c)
-    float inv1, inv2;
+    // queries into tensor memory: Q' natural pairs, Q'' pairs (32 g + c, 32 g + 16 + c), both with the
+    // row's power-of-two scale s so that the two products add in one accumulator
+    float inv;
     {
-      const float* q1 = a.qrot + grow * D;
-      const float* q2 = a.qproj + grow * D;
-      float mx1 = 0.f, mx2 = 0.f;
+      const float* q1 = a.qrot + qrow * D;
+      const float* q2 = a.qproj + qrow * D;
+      const float cq = a.qjl_coef;
+      float mx = 0.f;
       if (live)
-        for (int j = 0; j < D; ++j) mx1 = fmaxf(mx1, fabsf(q1[j])), mx2 = fmaxf(mx2, fabsf(q2[j]));
-      int e1 = 0, e2 = 0;
-      if (mx1 > 0.f) (void)frexpf(mx1, &e1);
-      if (mx2 > 0.f) (void)frexpf(mx2, &e2);
-      const float s1 = mx1 > 0.f ? ldexpf(1.f, 14 - e1) : 1.f, s2 = mx2 > 0.f ? ldexpf(1.f, 14 - e2) : 1.f;
-      inv1 = 1.f / s1;
-      inv2 = 1.f / s2;
+        for (int j = 0; j < D; ++j) mx = fmaxf(mx, fmaxf(fabsf(q1[j]), fabsf(q2[j]) * cq));
+      int e1 = 0;
+      if (mx > 0.f) (void)frexpf(mx, &e1);
+      const float s1 = mx > 0.f ? ldexpf(1.f, 14 - e1) : 1.f, s2 = s1 * cq;
+      inv = 1.f / s1;
       for (int c0 = 0; c0 < 64; c0 += 16) {
         uint32_t u1[16], u2[16];
 #pragma unroll
@@ -383,59 +499,112 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
-    const float c1 = inv1 * a.scale_log2, c2 = inv2 * a.qjl_coef * a.scale_log2;
+    const float cl = inv * a.scale_log2;    // base-2 logit = cl S
     float m_run = -FLT_MAX, l_run = 0.f;
     bool ok = true;
     for (int it = 0; ok && it < nkt; ++it) {
       const int64_t t0 = (kt_lo + it) * kTK;
-      if (!mbar_wait_warp(s_full, (uint32_t)(it & 1))) {
+      const uint32_t sc = tmem + lb + kColS + (uint32_t)(it & 1) * 128;
+      if (!mbar_wait_warp(&s_full[it & 1], (uint32_t)((it >> 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* nb = nrm + (it & 1) * 2 * kTK;
-      // logits (base 2) of 32 keys from the two accumulators, one tensor-memory
-      // wait for both 32-column loads; keys past this row's position (or the
-      // context end) are -FLT_MAX
-      auto logits32 = [&](int c0, float (&x)[32]) {
-        float v1[32], v2[32];
-        tmem_ld32(tmem + lb + kColS1 + c0, v1);
-        tmem_ld32(tmem + lb + kColS2 + c0, v2);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int k = c0 + e;
-          const bool vis = live && t0 + k <= pos && t0 + k < a.T;
-          x[e] = vis ? fmaf(nb[k] * c1, v1[e], nb[kTK + k] * c2 * v2[e]) : -FLT_MAX;
-        }
-      };
-      // pass 1: the row max of the tile
-      float mx = -FLT_MAX;
+      // keys past this row's position (or the context end) take no part; only
+      // a tile that some row of the warp does not see whole needs the test
+      const int64_t rel = pos - t0;
+      const int lim = live ? (int)(rel < 0 ? -1 : (rel > kTK - 1 ? kTK - 1 : rel)) : -1;
+      const bool masked = __any_sync(0xffffffffu, lim < kTK - 1);
+      // pass 1: the row max of the tile (four independent chains), 64 columns per tensor-memory wait
+      float m4[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll 1
-      for (int c0 = 0; c0 < kTK; c0 += 32) {
-        float x[32];
-        logits32(c0, x);
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[2][32];
+        tmem_ld32(sc + 64 * hf, v[0]);
+        tmem_ld32(sc + 64 * hf + 32, v[1]);
+        tmem_wait_ld();
+        regs_after_wait(v[0]);
+        regs_after_wait(v[1]);
+        if (masked) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, x[e]);
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[c][e] = 64 * hf + 32 * c + e <= lim ? v[c][e] : -FLT_MAX;
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], v[c][e]);
       }
+      const float smx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mx = smx > -FLT_MAX ? smx * cl : -FLT_MAX;
       // lazy rescale: a row's reference max moves only when one of its logits
-      // passes it by kLazy.  The O rescale goes through warp-collective tensor
-      // memory loads and stores, so the whole warp takes it when any row needs
-      // it (rows that do not rescale by 1).
-      const bool grow = mx > m_run + kLazy || (it == 0 && mx > -FLT_MAX);
-      const float mn = grow ? mx : m_run;
+      // passes it by kLazy (or on its first visible key)
+      const bool grow = mx > m_run + kLazy || (m_run == -FLT_MAX && mx > -FLT_MAX);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = m_run > -FLT_MAX ? ex2(m_run - mx) : 0.f;
+        l_run *= alpha;
+        m_run = mx;
+      }
+      // pass 2: P = 2^(cl S - m) as fp16 pairs of consecutive keys, written over
+      // the first 64 columns of the buffer (chunk c of 32 keys goes to columns
+      // 16 c .. 16 c + 15, which hold logits already read); the load of the next
+      // chunk is in flight while a chunk is weighted
+      const float mref = m_run > -FLT_MAX ? m_run : 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      auto weights = [&](const float (&x)[32], int c) {
+        float p[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) p[e] = ex2(fmaf(cl, x[e], -mref));
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) p[e] = 32 * c + e <= lim ? p[e] : 0.f;
+        }
+        uint32_t pu[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          ls[e & 3] += p[2 * e] + p[2 * e + 1];
+          pu[e] = h2u(__floats2half2_rn(p[2 * e], p[2 * e + 1]));
+        }
+        tmem_st16(sc + 16 * c, pu);
+      };
+      {
+        float va[32], vb[32];
+        tmem_ld32(sc, va);
+        tmem_wait_ld();
+        regs_after_wait(va);
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld32(sc + 32 * (c + 1), vb);
+          weights(va, c);
+          tmem_wait_ld();
+          regs_after_wait(vb);
+          if (c + 2 < 4) tmem_ld32(sc + 32 * (c + 2), va);
+          weights(vb, c + 1);
+          if (c + 2 < 4) {
+            tmem_wait_ld();
+            regs_after_wait(va);
+          }
+        }
+      }
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // O carries the value products of tiles before this one: once the last
+      // of them is done, the rows whose reference max moved scale it by alpha.
+      // The loads and stores are warp-collective, so the whole warp takes the
+      // step when any of its rows needs it (the others scale by 1).
       if (it > 0 && __any_sync(0xffffffffu, grow)) {
-        const float alpha = grow ? exp2f(m_run - mn) : 1.f;
         if (!mbar_wait_warp(pv_done, (uint32_t)((it - 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           float o[32];
           tmem_ld32(tmem + lb + kColO + c0, o);
           tmem_wait_ld();
+          regs_after_wait(o);
           uint32_t ou[16];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -444,49 +613,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PfArgs a) {
             tmem_st16(tmem + lb + kColO + c0 + 16 * hh, ou);
           }
         }
-        tmem_wait_st();
       }
-      if (grow) {
-        l_run *= (it > 0) ? exp2f(m_run - mn) : 0.f;
-        m_run = mn;
-      }
-      // pass 2: P (fp16 pairs of consecutive keys), 32 keys at a time; the 16
-      // columns written hold keys the earlier reads have consumed
-#pragma unroll 1
-      for (int c0 = 0; c0 < kTK; c0 += 32) {
-        float x[32];
-        logits32(c0, x);
-        uint32_t pu[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float xa = x[2 * e];
-          const float xb = x[2 * e + 1];
-          const float p0 = xa > -FLT_MAX ? exp2f(xa - m_run) : 0.f;
-          const float p1 = xb > -FLT_MAX ? exp2f(xb - m_run) : 0.f;
-          const __half2 ph = __floats2half2_rn(p0, p1);
-          l_run += __low2float(ph) + __high2float(ph);
-          pu[e] = h2u(ph);
-        }
-        tmem_st16(tmem + lb + kColS1 + c0 / 2, pu);
-        tmem_wait_st();
-      }
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
+      if (lane == 0) mbar_arrive(&p_ready[it & 1]);
     }
-    // the record of this row: acc (rotated frame), m (natural units), l
-    if (ok && nkt > 0 && !mbar_wait_warp(pv_done, (uint32_t)((nkt - 1) & 1))) ok = false;
+    // the record of this row: acc (rotated frame), m (natural units), l.  The
+    // last value products are awaited through the issuer's final commit: the
+    // parity of pv_done alone cannot tell phase nkt - 1 from phase nkt - 3 when
+    // the value product of tile nkt - 2 is still running
+    if (ok && nkt > 0 && !mbar_wait_warp(done, 0u)) ok = false;
     if (!ok) atomicOr(a.status, kStatusTimeout);
     tc_fence_after();
     // records are d + 2 = 130 floats apart, so a record starts on an 8-byte
     // (not always a 16-byte) boundary: two-float stores
-    float* rec = a.partials + (grow * a.splits + split) * (D + 2);
+    float* rec = a.partials + (qrow * a.splits + split) * (D + 2);
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
       float o[32];
       if (nkt > 0) {
         tmem_ld32(tmem + lb + kColO + c0, o);
         tmem_wait_ld();
+        regs_after_wait(o);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0.f;
@@ -546,7 +695,7 @@ int launch_prefill(const tq_ctx* hk, const tq_ctx* hv, const float* qrot, const 
   a.vnorms = vnorms;
   a.qrot = qrot;
   a.qproj = qproj;
-  a.kcent = hk->dev.centroids;
+  for (int k = 0; k < 4; ++k) a.ktab[k] = hk->host_ktab[k];
   a.vcent = hv->dev.centroids;
   a.B = B;
   a.nq = nq;
