@@ -322,31 +322,41 @@ __global__ void query_prep_kernel(const TIn* q, int64_t nq, int d, const float* 
 }
 
 // One thread per (query, key): est = n <q', c[idx]> + rn sqrt(pi/2)/d <q'', sigma>.
-// q' = Pi q and q'' = S q for d = 128 as a tiled fp32 product: the block
-// (blockIdx.y = which matrix) keeps M^T in shared memory and loops over tiles
-// of 32 query rows; thread (ty, tx) accumulates rows 4 ty .. + 3 x outputs
-// 4 tx .. + 3, summing over the input coordinate in order.
+// q' = Pi q and q'' = S q as a tiled fp32 product (d <= 256, d % 4 == 0): a
+// block takes one matrix and one chunk of 128 output coordinates (blockIdx.y =
+// matrix * chunks + chunk), keeps that chunk of M^T in shared memory and loops
+// over tiles of 32 query rows; thread (ty, tx) accumulates rows 4 ty .. + 3 x
+// outputs 4 tx .. + 3 of the chunk, summing over the input coordinate in order.
 constexpr int kQpRows = 32;
-constexpr int kQpLd = 132;   // padded row length (floats) of the shared tiles
-constexpr int kQpSmem = (128 + kQpRows) * kQpLd * 4;
+constexpr int kQpLd = 132;   // padded row length (floats) of the transposed matrix chunk
+
+inline int qp_smem_bytes(int d) { return (d * kQpLd + kQpRows * (d + 4)) * 4; }
 
 template <typename TIn>
-__global__ void __launch_bounds__(256) query_prep_tiled_kernel(const TIn* q, int64_t nq, const float* Pi,
-                                                               const float* S, float* qrot, float* qproj) {
+__global__ void __launch_bounds__(256) query_prep_tiled_kernel(const TIn* q, int64_t nq, int d, int chunks,
+                                                               const float* Pi, const float* S, float* qrot,
+                                                               float* qproj) {
   extern __shared__ __align__(16) float qp_smem[];
-  float* mt = qp_smem;                   // [i][j] = M[j][i]
-  float* qs = qp_smem + 128 * kQpLd;     // [row][i]
-  const float* M = blockIdx.y ? S : Pi;
-  float* out = blockIdx.y ? qproj : qrot;
-  for (int e = threadIdx.x; e < 128 * 128; e += 256) mt[(e & 127) * kQpLd + (e >> 7)] = M[e];
+  const int ld = d + 4;                  // row length of the query tile
+  float* mt = qp_smem;                   // [i][jj] = M[c0 + jj][i]
+  float* qs = qp_smem + d * kQpLd;       // [row][i]
+  const int which = (int)blockIdx.y / chunks, c0 = ((int)blockIdx.y % chunks) * 128;
+  const float* M = which ? S : Pi;
+  float* out = which ? qproj : qrot;
+  for (int e = threadIdx.x; e < 128 * d; e += 256) {
+    const int jj = e / d, i = e - jj * d;
+    mt[i * kQpLd + jj] = c0 + jj < d ? M[(int64_t)(c0 + jj) * d + i] : 0.f;
+  }
   const int ty = threadIdx.x >> 5, tx = threadIdx.x & 31;
+  const bool col_ok = c0 + 4 * tx < d;
   const int64_t tiles = (nq + kQpRows - 1) / kQpRows;
   for (int64_t rt = blockIdx.x; rt < tiles; rt += gridDim.x) {
     const int64_t r0 = rt * kQpRows;
     __syncthreads();
-    for (int e = threadIdx.x; e < kQpRows * 128; e += 256) {
-      const int64_t row = r0 + (e >> 7);
-      qs[(e >> 7) * kQpLd + (e & 127)] = row < nq ? load_elem(q, row * 128 + (e & 127)) : 0.f;
+    for (int e = threadIdx.x; e < kQpRows * d; e += 256) {
+      const int rr = e / d, i = e - rr * d;
+      const int64_t row = r0 + rr;
+      qs[rr * ld + i] = row < nq ? load_elem(q, row * d + i) : 0.f;
     }
     __syncthreads();
     float acc[4][4];
@@ -355,10 +365,10 @@ __global__ void __launch_bounds__(256) query_prep_tiled_kernel(const TIn* q, int
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
 #pragma unroll 2
-    for (int i = 0; i < 128; i += 4) {
+    for (int i = 0; i < d; i += 4) {
       float4 xa[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) xa[r] = *reinterpret_cast<const float4*>(qs + (4 * ty + r) * kQpLd + i);
+      for (int r = 0; r < 4; ++r) xa[r] = *reinterpret_cast<const float4*>(qs + (4 * ty + r) * ld + i);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float4 mb = *reinterpret_cast<const float4*>(mt + (i + k) * kQpLd + 4 * tx);
@@ -372,12 +382,14 @@ __global__ void __launch_bounds__(256) query_prep_tiled_kernel(const TIn* q, int
         }
       }
     }
+    if (col_ok)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int64_t row = r0 + 4 * ty + r;
-      if (row < nq)
-        *reinterpret_cast<float4*>(out + row * 128 + 4 * tx) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-    }
+      for (int r = 0; r < 4; ++r) {
+        const int64_t row = r0 + 4 * ty + r;
+        if (row < nq)
+          *reinterpret_cast<float4*>(out + row * d + c0 + 4 * tx) =
+              make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      }
   }
 }
 
@@ -632,16 +644,21 @@ int launch_query_prep(const tq_ctx* h, const float* q, int q_dtype, int64_t nq, 
   const float* S = qproj ? h->dev.S : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
   const bool out16 = ((reinterpret_cast<uintptr_t>(qrot) | reinterpret_cast<uintptr_t>(qproj)) & 15u) == 0;
-  if (h->d == 128 && nq > 0 && out16) {
+  if (h->d <= 256 && h->d % 4 == 0 && nq > 0 && out16) {
     const void* kern = q_dtype == TQ_BF16 ? (const void*)query_prep_tiled_kernel<__nv_bfloat16>
                                           : (const void*)query_prep_tiled_kernel<float>;
-    if (int e = ensure_dyn_smem(kern, kQpSmem)) return e;
+    const int smem = qp_smem_bytes(h->d);
+    if (int e = ensure_dyn_smem(kern, smem)) return e;
+    const int chunks = (h->d + 127) / 128;
+    const int ys = chunks * (qproj ? 2 : 1);
     const int64_t tiles = (nq + kQpRows - 1) / kQpRows;
-    const dim3 grid2((unsigned)std::min<int64_t>(tiles, h->sm_count), qproj ? 2u : 1u);
+    const int64_t xs = std::max<int64_t>(1, std::min<int64_t>(tiles, 2 * (int64_t)h->sm_count / ys));
+    const dim3 grid2((unsigned)xs, (unsigned)ys);
     if (q_dtype == TQ_BF16)
-      query_prep_tiled_kernel<<<grid2, 256, kQpSmem, s>>>((const __nv_bfloat16*)q, nq, h->dev.Pi, S, qrot, qproj);
+      query_prep_tiled_kernel<<<grid2, 256, smem, s>>>((const __nv_bfloat16*)q, nq, h->d, chunks, h->dev.Pi, S,
+                                                       qrot, qproj);
     else
-      query_prep_tiled_kernel<<<grid2, 256, kQpSmem, s>>>(q, nq, h->dev.Pi, S, qrot, qproj);
+      query_prep_tiled_kernel<<<grid2, 256, smem, s>>>(q, nq, h->d, chunks, h->dev.Pi, S, qrot, qproj);
     return (int)cudaGetLastError();
   }
   if (q_dtype == TQ_BF16)
