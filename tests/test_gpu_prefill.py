@@ -74,6 +74,15 @@ def test_prefill_whole_prompt():
     _prefill_case(B=1, nq=700, Hq=8, Hkv=2, T=700, sample=[(0, 0)], seed=3)
 
 
+def test_prefill_empty_context_slices_and_ragged_tail():
+    """nq = 600 of T = 1203 (a 3-token tail past the last whole group of four,
+    whose norms the kernel reads from global memory): with two context slices
+    per query tile, the early tokens' tiles see no key of the second slice, so
+    those CTAs write empty softmax records (m = -inf, l = 0) that the merge must
+    ignore, and tiles of several keys run through both logit buffers."""
+    _prefill_case(B=1, nq=600, Hq=4, Hkv=1, T=1203, sample=[(0, 0)], seed=4)
+
+
 def test_prefill_config4_cache_sampled():
     """A block of 128 tokens at the end of the decode configuration's cache
     (B = 8, Hq = 32, Hkv = 8, d = 128, T = 131072): the full launch, one
