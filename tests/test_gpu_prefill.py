@@ -75,12 +75,13 @@ def test_prefill_whole_prompt():
 
 
 def test_prefill_empty_context_slices_and_ragged_tail():
-    """nq = 600 of T = 1203 (a 3-token tail past the last whole group of four,
-    whose norms the kernel reads from global memory): with two context slices
-    per query tile, the early tokens' tiles see no key of the second slice, so
-    those CTAs write empty softmax records (m = -inf, l = 0) that the merge must
-    ignore, and tiles of several keys run through both logit buffers."""
-    _prefill_case(B=1, nq=600, Hq=4, Hkv=1, T=1203, sample=[(0, 0)], seed=4)
+    """nq = 600 of T = 1203 in rows of 1204 (the row stride stays a multiple of
+    four; the 3-token tail past the last whole group of four has its norms read
+    from global memory): with two context slices per query tile, the early
+    tokens' tiles see no key of the second slice, so those CTAs write empty
+    softmax records (m = -inf, l = 0) that the merge must ignore, and tiles of
+    several keys run through both logit buffers."""
+    _prefill_case(B=1, nq=600, Hq=4, Hkv=1, T=1203, sample=[(0, 0)], seed=4, stride_extra=1)
 
 
 def test_prefill_config4_cache_sampled():
