@@ -644,7 +644,9 @@ int launch_query_prep(const tq_ctx* h, const float* q, int q_dtype, int64_t nq, 
   const float* S = qproj ? h->dev.S : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
   const bool out16 = ((reinterpret_cast<uintptr_t>(qrot) | reinterpret_cast<uintptr_t>(qproj)) & 15u) == 0;
-  if (h->d <= 256 && h->d % 4 == 0 && nq > 0 && out16) {
+  // the tiled product pays a copy of the matrix into shared memory per block; a few hundred query rows (a decode
+  // step) finish sooner one warp per output
+  if (h->d <= 256 && h->d % 4 == 0 && nq >= 1024 && out16) {
     const void* kern = q_dtype == TQ_BF16 ? (const void*)query_prep_tiled_kernel<__nv_bfloat16>
                                           : (const void*)query_prep_tiled_kernel<float>;
     const int smem = qp_smem_bytes(h->d);
