@@ -36,9 +36,10 @@
 //          of two value tiles (an MN-major B operand, so each key's decoded row
 //          is stored whole; byte-table lookups in a per-lane copy of the table)
 //          once the value product of tile i - 2 is done with that tile
-//   6-9    softmax: thread = query row (TMEM lane); a tile's 128 logits stay in
-//          registers for both passes (row max, then weights), online softmax in
-//          base 2 with a lazy rescale of O
+//   6-9    softmax: thread = query row (TMEM lane); a tile's logits are read
+//          twice from tensor memory (the row max, 64 columns per wait; then
+//          the weights, the next 32 columns' load in flight while a chunk is
+//          weighted), online softmax in base 2 with a lazy rescale of O
 // Tensor memory: Q' [0, 64) | Q'' [64, 128) | S/P buffer 0 [128, 256) |
 // S/P buffer 1 [256, 384) | O [384, 512).  The sign tile pairs coordinates
 // (32g + c, 32g + 16 + c) in each 32-bit element, and Q'' is written with the
