@@ -492,3 +492,39 @@ def test_channel_split_takes_largest_scales():
     assert len(hi) == 64 and len(lo) == 64
     assert np.min(sc[hi]) > np.max(sc[lo])
     assert np.array_equal(np.sort(np.concatenate([hi, lo])), np.arange(128))
+
+
+def test_pack_signs_layout_by_hand():
+    """QJL sign bits use the b = 1 code layout of include/tq.h: bit i of word g is
+    coordinate 32 g + i, set for a non-negative projection."""
+    bits = np.zeros((2, 40), dtype=bool)
+    bits[0, [0, 31, 32, 39]] = True
+    bits[1, 5] = True
+    w = tq.pack_signs(bits)
+    assert w.shape == (2, 2)
+    assert [int(v) for v in w[0]] == [1 | (1 << 31), 1 | (1 << 7)]
+    assert [int(v) for v in w[1]] == [1 << 5, 0]
+    assert np.array_equal(tq.unpack_signs(w, 40), bits)
+    # a random round trip at a width that leaves a partial last word
+    r = synth.rng(0, 99).random((5, 77)) < 0.5
+    assert np.array_equal(tq.unpack_signs(tq.pack_signs(r), 77), r)
+
+
+def test_mse_estimate_by_hand():
+    """<q, x_hat> with x_hat = n Pi^T c[idx]: with Pi = I it is n sum_j q_j c[idx_j];
+    with a quarter-turn Pi = [[0, 1], [-1, 0]], Pi^T c = (-c_1, c_0)."""
+    c = np.array([-1.5, -0.5, 0.5, 1.5])
+    est = tq.mse_estimate(np.array([1.0, 2.0, -1.0, 0.5]), np.array([[0, 3, 1, 2]]), np.array([2.0]),
+                          np.eye(4), c)
+    assert est.shape == (1, 1)
+    assert abs(est[0, 0] - 2.0 * (-1.5 + 3.0 + 0.5 + 0.25)) < 1e-12
+    Pi = np.array([[0.0, 1.0], [-1.0, 0.0]])
+    q = np.array([[3.0, -2.0], [1.0, 1.0]])
+    idx = np.array([[0, 1], [1, 1]])
+    cc = np.array([0.25, -0.75])
+    n = np.array([1.0, 4.0])
+    est = tq.mse_estimate(q, idx, n, Pi, cc)
+    for i in range(2):
+        for k in range(2):
+            c0, c1 = cc[idx[k, 0]], cc[idx[k, 1]]
+            assert abs(est[i, k] - n[k] * (-q[i, 0] * c1 + q[i, 1] * c0)) < 1e-12
