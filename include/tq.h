@@ -345,6 +345,9 @@ TQ_API int tq_attn_decode_static(tq_handle hk, tq_handle hv, const void* q, int 
  *   workspace dev scratch of at least tq_attn_prefill_workspace(...) bytes
  * Supported: d = 128, keys TQ_PROD b = 4, values TQ_MSE b = 4, Hq / Hkv a
  * divisor of 128, kv_stride % 4 == 0 (TQ_EUNSUPPORTED otherwise).
+ * Range: the decoded operands are fp16 products n_k c[idx], rn_k and
+ * n_v c_V[idx], so key norms, residual norms and value norms must stay below
+ * 65504 / max|c| (about 3e5 for these codebooks); the kernel does not check it.
  * Errors: TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EALIGN, TQ_EWORKSPACE, TQ_ECUDA.
  */
 TQ_API int tq_attn_prefill(tq_handle hk, tq_handle hv, const void* q, int q_dtype, int B, int nq, int Hq, int Hkv,
