@@ -102,8 +102,11 @@ def test_hot_path_calls_reject_null_handle():
                           None) == _lib.TQ_EINVAL
     assert L.tq_attn_decode(None, None, None, 0, 1, 1, 1, 1, 1, None, None, None, None, None, None,
                             1.0, None, None, 0, None) == _lib.TQ_EINVAL
+    assert L.tq_attn_prefill(None, None, None, 0, 1, 1, 4, 1, 8, 8, None, None, None, None, None, None, 1.0, None,
+                             None, 0, None) == _lib.TQ_EINVAL
     assert L.tq_ip_scores_workspace(None, 1, 1, 0) == 0
     assert L.tq_attn_decode_workspace(None, 1, 1, 1, 1) == 0
+    assert L.tq_attn_prefill_workspace(None, 1, 1, 4, 1, 8) == 0
     assert L.tq_destroy(None) == _lib.TQ_OK
 
 
